@@ -1,0 +1,327 @@
+"""CPU oracle of the sequence-parallel boundary (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (``sp_region_b200``)
+never imports, links or runs anything here, and this package never imports the
+product: the two share nothing but the seeded input generators in ``sp_synth``.
+
+The arithmetic lives in ``sp_oracle.c`` (plain scalar C, double precision);
+this module only builds it with gcc and marshals tensors through ctypes.
+Inputs are CPU tensors in the I/O dtype (float32 or bfloat16), outputs are
+tensors in the I/O dtype plus float64 numpy arrays for the statistics and the
+parameter gradients.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sp_oracle.c")
+_LIB = os.path.join(_HERE, "liborc.so")
+
+F32, BF16 = 0, 1
+LAYERNORM, RMSNORM = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (IEEE double, no contraction into FMA).
+
+    ``SP_ORACLE_LIB`` names an already built library to load instead; the
+    mutation tests use it to run the pins against deliberately broken copies.
+    """
+    override = os.environ.get("SP_ORACLE_LIB")
+    if override:
+        return override
+    if (not force and os.path.exists(_LIB)
+            and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+        return _LIB
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
+           "-fno-fast-math", "-o", _LIB + ".tmp", _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(_LIB + ".tmp", _LIB)
+    return _LIB
+
+
+class Cfg(ctypes.Structure):
+    _fields_ = [("s", ctypes.c_int64), ("b", ctypes.c_int64),
+                ("h", ctypes.c_int64), ("t", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("norm", ctypes.c_int32),
+                ("eps", ctypes.c_float), ("p_drop", ctypes.c_float),
+                ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
+
+
+_lib_handle = None
+
+
+def _lib():
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = ctypes.CDLL(build())
+        L = _lib_handle
+        vp, i64, i32, dp = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
+                            ctypes.c_void_p)
+        L.orc_philox4x32_10.argtypes = [vp, vp, vp]
+        L.orc_round.argtypes = [ctypes.c_double, ctypes.c_int]
+        L.orc_round.restype = ctypes.c_double
+        L.orc_drop_threshold.argtypes = [ctypes.c_float]
+        L.orc_drop_threshold.restype = ctypes.c_uint32
+        L.orc_keep.argtypes = [ctypes.c_uint64, ctypes.c_uint64, i64, i64,
+                               ctypes.c_float]
+        L.orc_keep.restype = ctypes.c_int
+        L.orc_mask_words.argtypes = [i64]
+        L.orc_mask_words.restype = i64
+        L.orc_all_reduce.argtypes = [ctypes.c_int, i64, ctypes.c_int, vp, dp]
+        L.orc_reduce_scatter.argtypes = [ctypes.c_int, i64, i64, ctypes.c_int,
+                                         vp, ctypes.c_int, dp]
+        L.orc_all_gather.argtypes = [ctypes.c_int, i64, i64, vp, dp]
+        L.orc_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int,
+                              vp, dp, dp]
+        L.orc_fwd.restype = ctypes.c_int
+        L.orc_fwd_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
+                                   vp, dp, dp]
+        L.orc_fwd_rows.restype = ctypes.c_int
+        L.orc_bwd.argtypes = [vp, vp, vp, vp, vp, vp, dp, dp, vp, vp, dp, dp,
+                              dp]
+        L.orc_bwd.restype = ctypes.c_int
+        L.orc_bwd_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, dp, dp, vp, vp]
+        L.orc_bwd_rows.restype = ctypes.c_int
+        L.orc_activation_bytes.argtypes = [i64, i64, i64, i64, i32, i32,
+                                           ctypes.c_double]
+        L.orc_activation_bytes.restype = ctypes.c_double
+        L.orc_ring_bytes.argtypes = [i32, i32, ctypes.c_double]
+        L.orc_ring_bytes.restype = ctypes.c_double
+    return _lib_handle
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------
+
+def _dtype_code(dt) -> int:
+    if dt in ("f32", torch.float32):
+        return F32
+    if dt in ("bf16", torch.bfloat16):
+        return BF16
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+def _torch_dtype(code: int) -> torch.dtype:
+    return torch.float32 if code == F32 else torch.bfloat16
+
+
+def make_cfg(s, b, h, t, dtype, norm, eps, p_drop, seed=0, offset=0) -> Cfg:
+    return Cfg(s=s, b=b, h=h, t=t, dtype=_dtype_code(dtype),
+               norm=LAYERNORM if norm in ("layernorm", LAYERNORM) else RMSNORM,
+               eps=eps, p_drop=p_drop, seed=seed, offset=offset)
+
+
+def cfg_from(w, **over) -> Cfg:
+    """Oracle configuration from a workload description (``sp_synth``)."""
+    d = dict(s=w.s, b=w.b, h=w.h, t=w.t, dtype=w.dtype, norm=w.norm,
+             eps=w.eps, p_drop=w.p_drop, seed=w.drop_seed,
+             offset=w.drop_offset)
+    d.update(over)
+    return make_cfg(**d)
+
+
+def _cpu(x: Optional[torch.Tensor], dt_code: int) -> Optional[torch.Tensor]:
+    if x is None:
+        return None
+    x = x.detach().to("cpu").contiguous()
+    if x.dtype != _torch_dtype(dt_code):
+        raise TypeError(f"expected {_torch_dtype(dt_code)}, got {x.dtype}")
+    return x
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return x.data_ptr()
+    return x.ctypes.data
+
+
+def _ptr_array(ts: Sequence) -> ctypes.Array:
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, x in enumerate(ts):
+        arr[i] = _ptr(x)
+    return arr
+
+
+# ----------------------------------------------------------------------------
+# primitives
+# ----------------------------------------------------------------------------
+
+def philox(ctr: Sequence[int], key: Sequence[int]) -> List[int]:
+    c = np.array(ctr, dtype=np.uint32)
+    k = np.array(key, dtype=np.uint32)
+    o = np.zeros(4, dtype=np.uint32)
+    _lib().orc_philox4x32_10(c.ctypes.data, k.ctypes.data, o.ctypes.data)
+    return [int(v) for v in o]
+
+
+def round_to(x: float, dtype) -> float:
+    return _lib().orc_round(float(x), _dtype_code(dtype))
+
+
+def drop_threshold(p: float) -> int:
+    return int(_lib().orc_drop_threshold(p))
+
+
+def keep(seed: int, offset: int, n: int, j: int, p: float) -> bool:
+    return bool(_lib().orc_keep(seed, offset, n, j, p))
+
+
+def mask_words(h: int) -> int:
+    return int(_lib().orc_mask_words(h))
+
+
+def all_reduce(parts: Sequence[torch.Tensor]) -> np.ndarray:
+    dt = _dtype_code(parts[0].dtype)
+    ps = [_cpu(p, dt) for p in parts]
+    out = np.zeros(ps[0].numel(), dtype=np.float64)
+    _lib().orc_all_reduce(len(ps), ps[0].numel(), dt, _ptr_array(ps),
+                          out.ctypes.data)
+    return out.reshape(tuple(ps[0].shape))
+
+
+def reduce_scatter(parts: Sequence[torch.Tensor], rank: int) -> np.ndarray:
+    """parts: t tensors [rows, h]; returns rank's [rows/t, h] float64."""
+    dt = _dtype_code(parts[0].dtype)
+    ps = [_cpu(p, dt) for p in parts]
+    rows, h = ps[0].shape
+    t = len(ps)
+    out = np.zeros((rows // t, h), dtype=np.float64)
+    _lib().orc_reduce_scatter(t, rows, h, dt, _ptr_array(ps), rank,
+                              out.ctypes.data)
+    return out
+
+
+def all_gather(shards: Sequence[np.ndarray]) -> np.ndarray:
+    sh = [np.ascontiguousarray(s, dtype=np.float64) for s in shards]
+    rows, h = sh[0].shape
+    out = np.zeros((rows * len(sh), h), dtype=np.float64)
+    _lib().orc_all_gather(len(sh), rows, h, _ptr_array(sh), out.ctypes.data)
+    return out
+
+
+def activation_bytes(s, b, h, a, t, mode, bytes_per_elem) -> float:
+    return float(_lib().orc_activation_bytes(s, b, h, a, t, mode,
+                                             bytes_per_elem))
+
+
+def ring_bytes(t: int, kind: str, V: float) -> float:
+    k = {"reduce_scatter": 0, "all_gather": 1, "all_reduce": 2}[kind]
+    return float(_lib().orc_ring_bytes(t, k, V))
+
+
+# ----------------------------------------------------------------------------
+# the boundary
+# ----------------------------------------------------------------------------
+
+def fwd(cfg: Cfg, parts, bias, residual, gamma, beta, n_out: int = 1,
+        want_mask: bool = True) -> dict:
+    """Forward on all t emulated ranks.  Tensors are [s*b, h] / [h]."""
+    dt = cfg.dtype
+    tdt = _torch_dtype(dt)
+    ps = [_cpu(p, dt) for p in parts]
+    bias, residual, gamma, beta = (_cpu(x, dt) for x in
+                                   (bias, residual, gamma, beta))
+    N, h = cfg.s * cfg.b, cfg.h
+    rout = torch.empty((N, h), dtype=tdt)
+    gathered = [torch.empty((N, h), dtype=tdt) for _ in range(n_out)]
+    mask = (np.zeros((N, mask_words(h)), dtype=np.uint32) if want_mask
+            else None)
+    mean = np.zeros(N, dtype=np.float64)
+    rstd = np.zeros(N, dtype=np.float64)
+    rc = _lib().orc_fwd(ctypes.byref(cfg), _ptr_array(ps), _ptr(bias),
+                        _ptr(residual), _ptr(gamma), _ptr(beta), _ptr(rout),
+                        _ptr_array(gathered), n_out, _ptr(mask),
+                        mean.ctypes.data, rstd.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle forward rejected the configuration ({rc})")
+    return dict(residual_out=rout, gathered=gathered, mask=mask,
+                mean=mean if cfg.norm == LAYERNORM else None, rstd=rstd)
+
+
+def fwd_rows(cfg: Cfg, row_ids, part_rows, bias, residual_rows, gamma,
+             beta) -> dict:
+    """Forward on selected global token rows; inputs are [nrows, h]."""
+    dt = cfg.dtype
+    tdt = _torch_dtype(dt)
+    ids = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64))
+    ps = [_cpu(p, dt) for p in part_rows]
+    bias, residual_rows, gamma, beta = (_cpu(x, dt) for x in
+                                        (bias, residual_rows, gamma, beta))
+    n, h = len(ids), cfg.h
+    rout = torch.empty((n, h), dtype=tdt)
+    out = torch.empty((n, h), dtype=tdt)
+    mask = np.zeros((n, mask_words(h)), dtype=np.uint32)
+    mean = np.zeros(n, dtype=np.float64)
+    rstd = np.zeros(n, dtype=np.float64)
+    rc = _lib().orc_fwd_rows(ctypes.byref(cfg), n, ids.ctypes.data,
+                             _ptr_array(ps), _ptr(bias), _ptr(residual_rows),
+                             _ptr(gamma), _ptr(beta), _ptr(rout), _ptr(out),
+                             mask.ctypes.data, mean.ctypes.data,
+                             rstd.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle forward rejected the configuration ({rc})")
+    return dict(residual_out=rout, norm_out=out, mask=mask,
+                mean=mean if cfg.norm == LAYERNORM else None, rstd=rstd)
+
+
+def bwd(cfg: Cfg, dparts, drnext, x, gamma, mask, mean, rstd,
+        with_dbeta: bool = True, with_dbias: bool = True) -> dict:
+    """Backward on all t emulated ranks (mask None: nothing was dropped)."""
+    dt = cfg.dtype
+    tdt = _torch_dtype(dt)
+    ps = [_cpu(p, dt) for p in dparts]
+    drnext, x, gamma = (_cpu(v, dt) for v in (drnext, x, gamma))
+    N, h = cfg.s * cfg.b, cfg.h
+    mask = None if mask is None else np.ascontiguousarray(mask, np.uint32)
+    mean = (np.zeros(N) if mean is None
+            else np.ascontiguousarray(mean, np.float64))
+    rstd = np.ascontiguousarray(rstd, np.float64)
+    dres = torch.empty((N, h), dtype=tdt)
+    dY = torch.empty((N, h), dtype=tdt)
+    dg = np.zeros(h)
+    db = np.zeros(h) if with_dbeta else None
+    dc = np.zeros(h) if with_dbias else None
+    rc = _lib().orc_bwd(ctypes.byref(cfg), _ptr_array(ps), _ptr(drnext),
+                        _ptr(x), _ptr(gamma), _ptr(mask), mean.ctypes.data,
+                        rstd.ctypes.data, _ptr(dres), _ptr(dY), dg.ctypes.data,
+                        _ptr(db), _ptr(dc))
+    if rc != 0:
+        raise ValueError(f"oracle backward rejected the configuration ({rc})")
+    return dict(dresidual_in=dres, dY=dY, dgamma=dg, dbeta=db, dbias=dc)
+
+
+def bwd_rows(cfg: Cfg, dpart_rows, drnext_rows, x_rows, gamma, mask_rows,
+             mean, rstd) -> dict:
+    """Backward on selected rows (per-row outputs only)."""
+    dt = cfg.dtype
+    tdt = _torch_dtype(dt)
+    ps = [_cpu(p, dt) for p in dpart_rows]
+    drnext_rows, x_rows, gamma = (_cpu(v, dt) for v in
+                                  (drnext_rows, x_rows, gamma))
+    n, h = x_rows.shape
+    mask_rows = (None if mask_rows is None
+                 else np.ascontiguousarray(mask_rows, np.uint32))
+    mean = (np.zeros(n) if mean is None
+            else np.ascontiguousarray(mean, np.float64))
+    rstd = np.ascontiguousarray(rstd, np.float64)
+    dres = torch.empty((n, h), dtype=tdt)
+    dY = torch.empty((n, h), dtype=tdt)
+    rc = _lib().orc_bwd_rows(ctypes.byref(cfg), n, _ptr_array(ps),
+                             _ptr(drnext_rows), _ptr(x_rows), _ptr(gamma),
+                             _ptr(mask_rows), mean.ctypes.data,
+                             rstd.ctypes.data, _ptr(dres), _ptr(dY))
+    if rc != 0:
+        raise ValueError(f"oracle backward rejected the configuration ({rc})")
+    return dict(dresidual_in=dres, dY=dY)
