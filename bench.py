@@ -1,0 +1,540 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 sequence-parallel boundary (forward + backward).
+
+One step is one pass of the whole hot path over one batch of synthetic input
+(the C2 workload: s=2048, b=4, h=6144, t=8 emulated ranks, bf16 I/O, fp32
+arithmetic, LayerNorm, dropout p=0.1, bias):
+
+  forward   sp_rs_bias_dropout_add_norm_fwd: reduce-scatter of the 8 partial
+            sums + bias + dropout + residual + LayerNorm + all-gather write
+  backward  sp_rs_norm_dropout_bwd: reduce-scatter of the 8 upstream gradient
+            partials + LayerNorm / residual / dropout backward + all-gathered
+            dY + dgamma / dbeta / dbias
+
+The metric is achieved HBM bandwidth on the algorithmic bytes of both calls
+(GB/s), with tokens/s and the fraction of the measured HBM peak beside it.
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs an independent
+replica on its own GPU (weak scaling; the path has no exchange between
+replicas); the time is the maximum over ranks.  ``--impl reference`` times the
+CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SP-boundary fwd+bwd achieved HBM GB/s (% of B200 peak); tokens/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------------------
+# algorithmic bytes (per call), from the data each call must move
+# ----------------------------------------------------------------------------
+
+def fwd_bytes(w, n_gathered=1):
+    E, N, h = w.elem_bytes, w.rows, w.h
+    sbh = N * h
+    W = (h + 31) // 32
+    params = h * E * (1 + (1 if w.has_bias else 0) +
+                      (1 if (w.has_beta and w.norm == "layernorm") else 0))
+    rd = (w.t + 1) * E * sbh + params
+    stats = (8 if w.norm == "layernorm" else 4) * N
+    wr = E * sbh * (1 + n_gathered) + 4 * W * N + stats
+    return rd + wr
+
+
+def bwd_bytes(w, with_drnext=False):
+    E, N, h = w.elem_bytes, w.rows, w.h
+    sbh = N * h
+    W = (h + 31) // 32
+    stats = (8 if w.norm == "layernorm" else 4) * N
+    rd = w.t * E * sbh + E * sbh + 4 * W * N + stats + h * E
+    if with_drnext:
+        rd += E * sbh
+    ngrad = 1 + (1 if w.norm == "layernorm" else 0) + (1 if w.has_bias else 0)
+    wr = 2 * E * sbh + 4 * h * ngrad
+    return rd + wr
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def kernel_sources_sha():
+    h = hashlib.sha1()
+    for f in ("sp_region.cu", "sp_device.cuh", "sp_fwd.cuh", "sp_bwd.cuh",
+              "sp_gather.cuh"):
+        with open(os.path.join(ROOT, "sp_region_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def recorded_traffic(kernel_key):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    sha = kernel_sources_sha()
+    for line in open(p):
+        if line.startswith("#") or "=" not in line:
+            continue
+        kv = dict(x.split("=", 1) for x in line.split())
+        if kv.get("key") == kernel_key and kv.get("src_sha1") == sha:
+            return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,"
+              "clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples = []   # (host time, sm, max, power, reasons...)
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev),
+                 f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append((time.time(), *parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed"
+        if not win:
+            win = self.samples
+            window = "whole run (timed region shorter than the sampling period)"
+        if not win:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "samples": 0, "note": "nvidia-smi unavailable"}
+        sm = [num(s[1]) for s in win if num(s[1]) is not None]
+        mx = [num(s[2]) for s in win if num(s[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for s in win for i in range(4)
+                          if s[4 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(win), "window": window}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import sp_synth
+    import sp_region_b200 as sp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    w = sp_synth.WORKLOADS[args.workload]
+    w = w.replace(seed=w.seed + 1000 * rank)   # each replica its own batch
+    N, h, t = w.rows, w.h, w.t
+    dt = w.torch_dtype
+    cfg = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm, eps=w.eps,
+                      p_drop=w.p_drop, seed=w.drop_seed, offset=w.drop_offset)
+
+    parts = sp_synth.draw_partials(w, dev)
+    bias, gamma, beta = sp_synth.draw_params(w, dev)
+    if not w.has_bias:
+        bias = None
+    if not w.has_beta or w.norm == "rmsnorm":
+        beta = None
+    res = sp_synth.draw_residual(w, dev)
+    dparts = sp_synth.draw_grad_partials(w, dev)
+    rout = torch.empty((N, h), dtype=dt, device=dev)
+    out = torch.empty((N, h), dtype=dt, device=dev)
+    mask = torch.empty((N, (h + 31) // 32), dtype=torch.int32, device=dev)
+    mean = torch.empty(N, dtype=torch.float32, device=dev)
+    rstd = torch.empty(N, dtype=torch.float32, device=dev)
+    dres = torch.empty((N, h), dtype=dt, device=dev)
+    dY = torch.empty((N, h), dtype=dt, device=dev)
+    dg = torch.empty(h, dtype=torch.float32, device=dev)
+    db = torch.empty(h, dtype=torch.float32, device=dev) \
+        if w.norm == "layernorm" else None
+    dc = torch.empty(h, dtype=torch.float32, device=dev) if bias is not None \
+        else None
+    ws = torch.empty(sp.sp_bwd_workspace_bytes(cfg, local) // 4,
+                     dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        sp.sp_rs_bias_dropout_add_norm_fwd(cfg, parts, bias, res, gamma, beta,
+                                           rout, [out], mask, mean, rstd,
+                                           stream=stream)
+
+    def bwd():
+        sp.sp_rs_norm_dropout_bwd(cfg, dparts, None, rout, gamma, mask, mean,
+                                  rstd, dres, dY, dg, db, dc, ws,
+                                  stream=stream)
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)]
+           for _ in range(K)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)   # let the sampler start before the timed region
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    h0 = time.time()
+    e0.record(stream)
+    for i in range(K):
+        evs[i][0].record(stream)
+        fwd()
+        evs[i][1].record(stream)
+        bwd()
+        evs[i][2].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    h1 = time.time()
+    if world > 1:
+        dist.barrier()
+    clocks.stop()
+    assert sp.sp_device_error(local) == 0, "device-side wait timed out"
+
+    total_ms = e0.elapsed_time(e1)
+    fwd_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
+    bwd_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
+    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    total_ms = float(tmax.item())
+
+    fb, bb = fwd_bytes(w), bwd_bytes(w)
+    step_bytes = fb + bb
+    value = step_bytes * world * K / (total_ms * 1e-3) / 1e9
+    ms_step = total_ms / K
+    peak, peak_src = measured_peak()
+    f_avg = statistics.mean(fwd_ms)
+    b_avg = statistics.mean(bwd_ms)
+    kern = {
+        "fwd": {"kernel": "k_fwd_tma", "bytes_per_launch": fb,
+                "avg_ms": f_avg, "gbs": fb / (f_avg * 1e-3) / 1e9},
+        "bwd": {"kernel": "k_bwd_tma + k_colreduce", "bytes_per_launch": bb,
+                "avg_ms": b_avg, "gbs": bb / (b_avg * 1e-3) / 1e9},
+    }
+    dom = "fwd" if f_avg >= b_avg else "bwd"
+    dk = kern[dom]
+    traffic = recorded_traffic(f"{dom}:{args.workload}")
+    roofline = {"bound": "hbm", "achieved": round(dk["gbs"], 1),
+                "peak": peak, "unit": "GB/s",
+                "frac": round(dk["gbs"] / peak, 4), "traffic": traffic,
+                "kernel": dk["kernel"], "call": dom,
+                "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": dk["bytes_per_launch"]}
+
+    e2e = run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+        cpu = cpu_baseline(w, fb, bb, budget_s=args.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "io_dtype": w.dtype, "data": "synthetic",
+        "config": {
+            "workload": (f"{w.name}: SP boundary fwd+bwd, s={w.s} b={w.b} "
+                         f"h={h} t={t} emulated ranks, {w.dtype} I/O, "
+                         f"{w.norm}, p={w.p_drop}, bias"),
+            "s": w.s, "b": w.b, "h": h, "t": t,
+            "global_batch": w.b * world, "seq_len": w.s,
+            "parallelism": f"{world} independent replicas (t={t} ranks "
+                           "emulated in one GPU's HBM each)",
+            "l2": "inputs larger than L2: each step streams "
+                  f"{step_bytes / 1e9:.2f} GB of distinct buffers (L2 126 MB)"},
+        "tokens_per_s": round(N * world / (ms_step * 1e-3), 1),
+        "pct_of_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_peak": round(100 * value / world / peak, 2),
+        "roofline": roofline,
+        "kernels": kern,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 3 * K,
+        "clocks": clocks.summary(h0, h1),
+    }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
+    """Same metric through the public API with host buffers: every step copies
+    its inputs from pinned host memory, runs forward and backward, and reads
+    every output back to pinned host memory, inside the timed region."""
+    import sp_synth
+    N, h = w.rows, w.h
+    dt = w.torch_dtype
+    pin = lambda x: None if x is None else x.cpu().pin_memory()
+    hp = [pin(p) for p in sp_synth.draw_partials(w, dev)]
+    bias, gamma, beta = sp_synth.draw_params(w, dev)
+    if not w.has_bias:
+        bias = None
+    if not w.has_beta or w.norm == "rmsnorm":
+        beta = None
+    hb, hg, hbe = pin(bias), pin(gamma), pin(beta)
+    hr = pin(sp_synth.draw_residual(w, dev))
+    hd = [pin(p) for p in sp_synth.draw_grad_partials(w, dev)]
+    ins = [*hp, hb, hg, hbe, hr, *hd]
+    h2d = sum(x.numel() * x.element_size() for x in ins if x is not None)
+    dev_in = [None if x is None else torch.empty_like(x, device=dev)
+              for x in ins]
+    t = w.t
+    d_parts, d_b, d_g, d_be, d_r = (dev_in[:t], dev_in[t], dev_in[t + 1],
+                                    dev_in[t + 2], dev_in[t + 3])
+    d_dp = dev_in[t + 4:]
+    outs_d = dict(rout=torch.empty((N, h), dtype=dt, device=dev),
+                  out=torch.empty((N, h), dtype=dt, device=dev),
+                  mask=torch.empty((N, (h + 31) // 32), dtype=torch.int32,
+                                   device=dev),
+                  mean=torch.empty(N, dtype=torch.float32, device=dev),
+                  rstd=torch.empty(N, dtype=torch.float32, device=dev),
+                  dres=torch.empty((N, h), dtype=dt, device=dev),
+                  dY=torch.empty((N, h), dtype=dt, device=dev),
+                  dg=torch.empty(h, dtype=torch.float32, device=dev),
+                  db=torch.empty(h, dtype=torch.float32, device=dev),
+                  dc=torch.empty(h, dtype=torch.float32, device=dev))
+    if w.norm != "layernorm":
+        outs_d["db"] = None
+    if bias is None:
+        outs_d["dc"] = None
+    outs_h = {k: (None if v is None else
+                  torch.empty_like(v, device="cpu").pin_memory())
+              for k, v in outs_d.items()}
+    d2h = sum(v.numel() * v.element_size() for v in outs_h.values()
+              if v is not None)
+    ws = torch.empty(sp.sp_bwd_workspace_bytes(cfg, dev.index) // 4,
+                     dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for d_, h_ in zip(dev_in, ins):
+            if h_ is not None:
+                d_.copy_(h_, non_blocking=True)
+        o = outs_d
+        sp.sp_rs_bias_dropout_add_norm_fwd(cfg, d_parts, d_b, d_r, d_g, d_be,
+                                           o["rout"], [o["out"]], o["mask"],
+                                           o["mean"], o["rstd"], stream=stream)
+        sp.sp_rs_norm_dropout_bwd(cfg, d_dp, None, o["rout"], d_g, o["mask"],
+                                  o["mean"], o["rstd"], o["dres"], o["dY"],
+                                  o["dg"], o["db"], o["dc"], ws, stream=stream)
+        for k, v in o.items():
+            if v is not None:
+                outs_h[k].copy_(v, non_blocking=True)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.e2e_steps
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        import torch.distributed as dist
+        tm = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms = float(tm.item())
+    return {"value": round(step_bytes * world * K / (ms * 1e-3) / 1e9, 2),
+            "unit": "GB/s", "ms_per_step": round(ms / K, 3), "steps": K,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "path": "pinned host -> device copies, fwd + bwd through the C "
+                    "ABI, every output copied back to pinned host"}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle (baseline leg and reference arm)
+# ----------------------------------------------------------------------------
+
+def _oracle_rows(w, row0, nrows, orc, sp_synth, cfg):
+    """Oracle forward + backward on token rows [row0, row0 + nrows), inputs
+    drawn on the host with the workload's recipe (rows seeded by row0)."""
+    ww = w.replace(seed=w.seed + 7919 * (row0 + 1))
+    parts = sp_synth.draw_partials(ww, rows=nrows)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    res = sp_synth.draw_residual(ww, rows=nrows)
+    dparts = sp_synth.draw_grad_partials(ww, rows=nrows)
+    ids = list(range(row0, row0 + nrows))
+    t0 = time.perf_counter()
+    fo = orc.fwd_rows(cfg, ids, parts, bias, res, gamma, beta)
+    orc.bwd_rows(cfg, dparts, None, fo["residual_out"], gamma, fo["mask"],
+                 fo["mean"], fo["rstd"])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, fb, bb, budget_s=10.0):
+    import oracle as orc
+    import sp_synth
+    orc.build()
+    cfg = orc.cfg_from(w)
+    per_row = (fb + bb) / w.rows
+    rows_done, secs, row0 = 0, 0.0, 0
+    chunk = 64
+    while secs < budget_s and row0 < w.rows:
+        n = min(chunk, w.rows - row0)
+        secs += _oracle_rows(w, row0, n, orc, sp_synth, cfg)
+        rows_done += n
+        row0 += n
+    return {"value": round(per_row * rows_done / secs / 1e9, 4),
+            "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": (f"{w.name} token rows 0..{rows_done - 1} of {w.rows} "
+                       f"(forward + backward per row, {secs:.1f} s of "
+                       "single-threaded C oracle time)"),
+            "tokens_per_s": round(rows_done / secs, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle as orc
+    import sp_synth
+    orc.build()
+    w = sp_synth.WORKLOADS[args.workload]
+    cfg = orc.cfg_from(w)
+    fb, bb = fwd_bytes(w), bwd_bytes(w)
+    per_row = (fb + bb) / w.rows
+    # per-step sample sized so that warm-up + timed steps take ~2 minutes
+    t_row = _oracle_rows(w, 0, 8, orc, sp_synth, cfg) / 8
+    rows = int(max(1, min(256, 120.0 / max(1, args.steps + args.warmup)
+                          / max(t_row, 1e-6))))
+    for i in range(args.warmup):
+        _oracle_rows(w, (i * rows) % w.rows, min(rows, w.rows), orc, sp_synth,
+                     cfg)
+    secs = 0.0
+    for i in range(args.steps):
+        r0 = ((args.warmup + i) * rows) % max(1, w.rows - rows + 1)
+        secs += _oracle_rows(w, r0, rows, orc, sp_synth, cfg)
+    value = per_row * rows * args.steps / secs / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(secs / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "io_dtype": w.dtype, "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": (f"{w.name}: SP boundary fwd+bwd, s={w.s} "
+                                f"b={w.b} h={w.h} t={w.t}, {w.dtype} I/O, "
+                                f"{w.norm}, p={w.p_drop}, bias"),
+                   "s": w.s, "b": w.b, "h": w.h, "t": w.t,
+                   "sample_rows_per_step": rows},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
+                         "cores": 1, "kind": "oracle",
+                         "sample": f"{rows} token rows of {w.name} per step, "
+                                   "forward + backward"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s",
+                "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "tokens_per_s": round(rows * args.steps / secs, 2),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="C2")
+    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,260 @@
+/*
+ * sp_region.h -- C ABI of the B200 (sm_100a) sequence-parallel boundary.
+ *
+ * The boundary sits where a tensor-parallel (TP) region hands its output to a
+ * sequence-parallel (SP) region and back:
+ *
+ *   t partial sums of a row-parallel linear
+ *     -> reduce-scatter along the sequence (each rank keeps s/t tokens)
+ *     -> + bias -> dropout -> + residual -> LayerNorm / RMSNorm
+ *     -> all-gather back to the full [s, b, h] input of the next
+ *        column-parallel linear
+ *
+ * and its backward, in which the all-gather and the reduce-scatter swap
+ * places.  Sources (web pages on Megatron sequence parallelism):
+ *   "Sequence Parallelism math" (aicassindra.com transformer-math), sections
+ *     "The move", "The collective substitution", "Why the byte count is
+ *     identical" and equations A_layer, A_TP, A_TP+SP;
+ *   "SP: Partition Activations Alongside TP" (llm-systems-engineering),
+ *     sections "Normalize and add residuals by token", "Change layouts
+ *     between SP and TP", "Connect SP and TP across a layer";
+ *   "TP and SP explained with pictures" (medium), section "Add Sequence
+ *     parallelism".
+ *
+ * On one GPU the t ranks are emulated: rank k's partial sum is its own
+ * buffer in the same HBM, and rank r's token shard is rows
+ * [r*N/t, (r+1)*N/t) of the [s, b, h] tensors (N = s*b).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout      [s, b, h] with h fastest, stored as N = s*b token rows of h
+ *             elements; token row n = s_idx*b + b_idx.  Rank r owns rows
+ *             [r*N/t, (r+1)*N/t), which is contiguous because the shard is
+ *             along s, the outermost dimension.
+ * Dtypes      cfg->dtype applies to partial sums, residual, gamma, beta,
+ *             bias and every [s,b,h] output; mean, rstd and the parameter
+ *             gradients are always fp32.  Arithmetic is fp32.
+ * Memory      every pointer argument named "device" is a CUDA device
+ *             pointer on the current device; arrays of pointers
+ *             (partials, gathered, dn_partials, shards, outs) are HOST arrays
+ *             of device pointers.  The caller owns every buffer; the library
+ *             allocates nothing.
+ * Execution   device work is enqueued on `stream` (a cudaStream_t passed as
+ *             void*; NULL is the legacy default stream) and is asynchronous.
+ *             No call synchronises.  The return value reports argument
+ *             validation and launch only.
+ * Errors      a call that returns anything but SP_OK enqueued nothing.
+ *             Arguments are validated before any launch: NULL required
+ *             pointers, s % t != 0, t outside [1, SP_MAX_T], h < 1,
+ *             p_drop outside [0, 1), eps <= 0 or not finite, unknown dtype
+ *             or norm codes, and s*b or h beyond the 32-bit Philox counter
+ *             give SP_ERR_INVALID_ARG.  A failed launch gives SP_ERR_CUDA.
+ *             Device-side waits are bounded in time; a wait that runs out
+ *             records a code that sp_device_error() reports, and the kernel
+ *             returns instead of hanging.
+ * Alignment   the fast kernels need 16-byte aligned [s,b,h] pointers and
+ *             h*elem_bytes a multiple of 16; other shapes take a slower
+ *             general kernel with the same results.  Nothing is rejected for
+ *             alignment except pointers not aligned to their element size.
+ */
+#ifndef SP_REGION_H
+#define SP_REGION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SP_MAX_T 64
+
+typedef enum {
+    SP_OK = 0,
+    SP_ERR_INVALID_ARG = 1,
+    SP_ERR_UNSUPPORTED = 2,
+    SP_ERR_CUDA = 3,
+    SP_ERR_DEVICE_TIMEOUT = 4
+} sp_status;
+
+typedef enum { SP_F32 = 0, SP_BF16 = 1 } sp_dtype;
+typedef enum { SP_LAYERNORM = 0, SP_RMSNORM = 1 } sp_norm;
+
+/* Problem description.
+ *   s, b, h  sequence length, micro-batch, hidden size
+ *   t        tensor/sequence-parallel degree (number of emulated ranks)
+ *   dtype    sp_dtype of the I/O tensors
+ *   norm     sp_norm
+ *   eps      added to the variance (LayerNorm) or the mean square (RMSNorm)
+ *            inside the square root
+ *   p_drop   dropout probability in [0, 1)
+ *   seed, offset   Philox4x32-10 key and counter offset of the dropout mask */
+typedef struct {
+    int64_t s, b, h;
+    int32_t t;
+    int32_t dtype;
+    int32_t norm;
+    float eps;
+    float p_drop;
+    uint64_t seed, offset;
+} sp_cfg;
+
+/*
+ * Forward of the boundary: reduce-scatter + bias + dropout + residual add +
+ * norm, with the all-gather fused into the output write.
+ *
+ * Defined by: "Sequence Parallelism math", section "The collective
+ * substitution" (leaving a TP region the all-reduce becomes a reduce-scatter
+ * that sums the partials and scatters sequence shards; entering the next, an
+ * all-gather); section "The move" (LayerNorm per token, dropout elementwise);
+ * "SP: Partition Activations Alongside TP", sections "Normalize and add
+ * residuals by token" and "Connect SP and TP across a layer" (residual add in
+ * the token layout, its result is what the norm consumes).
+ *
+ * For every token row n (rank r = n / (N/t) owns it):
+ *   y       = sum_{k=0..t-1} partials[k][n, :]      fp32, k ascending
+ *   y      += bias                                   (once, if bias != NULL)
+ *   z       = keep(n, j) ? y / (1 - p_drop) : 0      inverted dropout
+ *   r_out   = round(residual[n, :] + z)              stored in cfg->dtype
+ *   LN:  o  = (r_out - mean) * rstd * gamma + beta,
+ *        mean, var = mean and biased variance of r_out over h,
+ *        rstd = 1 / sqrt(var + eps)
+ *   RMS: o  = r_out * rstd * gamma, rstd = 1 / sqrt(mean(r_out^2) + eps)
+ *   gathered[q][n, :] = round(o) for every q < n_gathered   (all-gather)
+ * keep(n, j): Philox4x32-10 with key (seed lo, seed hi) and counter
+ * (j >> 2, n, offset lo, offset hi); word j & 3 is compared with
+ * floor(p_drop * 2^32) and the element is dropped iff it is smaller.  n is
+ * the global row, so results do not depend on t.
+ *
+ * Arguments (device unless stated):
+ *   partials     HOST array of t device pointers, each [s,b,h]
+ *   bias         [h] or NULL
+ *   residual     [s,b,h]
+ *   gamma        [h]
+ *   beta         [h] or NULL (LayerNorm without shift; ignored for RMSNorm)
+ *   residual_out [s,b,h], may alias residual (in-place update)
+ *   gathered     HOST array of n_gathered device pointers, each [s,b,h]; on
+ *                one GPU the shard-major norm output is already the gathered
+ *                tensor, so n_gathered = 1 is the plain case and n_gathered
+ *                = t writes per-rank replicas.  Must not alias the inputs.
+ *   n_gathered   1 .. SP_MAX_T
+ *   mask_bits    [N][ceil(h/32)] uint32 or NULL: bit j&31 of word
+ *                n*ceil(h/32) + (j>>5) is 1 iff element j was kept; padding
+ *                bits are 0.  With p_drop = 0 every valid bit is 1.
+ *   mean, rstd   [N] fp32 or NULL (mean is not written for RMSNorm)
+ *   stream       cudaStream_t
+ */
+int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg,
+                                    const void* const* partials,
+                                    const void* bias, const void* residual,
+                                    const void* gamma, const void* beta,
+                                    void* residual_out,
+                                    void* const* gathered, int32_t n_gathered,
+                                    uint32_t* mask_bits, float* mean,
+                                    float* rstd, void* stream);
+
+/*
+ * All-gather of t sequence shards into n_out full [s,b,h] tensors.
+ *
+ * Defined by: "SP: Partition Activations Alongside TP", section "Change
+ * layouts between SP and TP" (the token shards of the SP region combine into
+ * the same input X on every GPU); "Sequence Parallelism math", section "The
+ * collective substitution".
+ *
+ *   shards  HOST array of t device pointers; shard r is [N/t, h] rows of
+ *           rank r (they may be consecutive slices of one buffer)
+ *   outs    HOST array of n_out device pointers, each [s,b,h]; out[q] rows
+ *           [r*N/t, (r+1)*N/t) receive shard r.  Must not overlap shards.
+ *   n_out   1 .. SP_MAX_T
+ */
+int sp_all_gather(const sp_cfg* cfg, const void* const* shards,
+                  void* const* outs, int32_t n_out, void* stream);
+
+/*
+ * Backward of the boundary: reduce-scatter of the upstream gradient partials
+ * + norm backward + residual-stream gradient + dropout backward, with the
+ * all-gather of the gradient w.r.t. the partial sums fused into its write.
+ *
+ * Defined by: "Sequence Parallelism math", section "The collective
+ * substitution" (the backward swaps all-gather and reduce-scatter, their
+ * conjugates); the norm and dropout derivatives are the textbook ones.
+ *
+ * For every token row n:
+ *   dn   = sum_k dn_partials[k][n, :]            (all-gather's backward)
+ *   xhat = (x - mean) * rstd (LN) or x * rstd (RMS), x = residual_out
+ *   g    = dn * gamma
+ *   LN:  dx = rstd * (g - mean_j(g) - xhat * mean_j(g * xhat))
+ *   RMS: dx = rstd * (g - xhat * mean_j(g * xhat))
+ *   dr   = dx + dR_next (if given)
+ *   dresidual_in[n, :] = round(dr)
+ *   dz   = keep ? dr / (1 - p_drop) : 0,  keep read from mask_bits
+ *   dY[n, :] = round(dz)                         (reduce-scatter's backward)
+ *   dgamma += dn * xhat, dbeta += dn, dbias += dz   summed over all N rows
+ *
+ * Arguments (device unless stated):
+ *   dn_partials  HOST array of t device pointers, each [s,b,h]
+ *   dR_next      [s,b,h] or NULL
+ *   residual_out, mask_bits, mean, rstd   the forward's outputs (mask_bits
+ *                may be NULL only when p_drop == 0; mean unused for RMS)
+ *   gamma        [h]
+ *   dresidual_in [s,b,h]; dY [s,b,h]
+ *   dgamma [h] fp32; dbeta [h] fp32 or NULL; dbias [h] fp32 or NULL
+ *   workspace    device scratch of at least sp_bwd_workspace_bytes() bytes,
+ *                16-byte aligned; no initial contents needed
+ * The parameter gradients are deterministic: per-CTA partial sums in a
+ * fixed order, then one fixed-order sum over CTAs.
+ */
+int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
+                           const void* dR_next, const void* residual_out,
+                           const void* gamma, const uint32_t* mask_bits,
+                           const float* mean, const float* rstd,
+                           void* dresidual_in, void* dY, float* dgamma,
+                           float* dbeta, float* dbias, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Bytes of device scratch sp_rs_norm_dropout_bwd needs for cfg on CUDA
+ * device `device` (it depends on the device's SM count).  Host-only. */
+int sp_bwd_workspace_bytes(const sp_cfg* cfg, int32_t device, size_t* bytes);
+
+/*
+ * Activation memory of one transformer layer per device, host-only.
+ *
+ * Defined by: "Sequence Parallelism math", equation A_layer (section "The
+ * problem: activation memory") and equations A_TP and A_TP+SP (section "The
+ * activation-memory saving"); "TP and SP explained with pictures" and the
+ * anthology record summarise the same accounting.
+ *   mode 0: A_layer  = s*b*h * (34 + 5*a*s/h)
+ *   mode 1: A_TP     = s*b*h * (10 + 24/t + 5*a*s/(h*t))
+ *   mode 2: A_TP+SP  = (s*b*h / t) * (34 + 5*a*s/h)
+ * *out = coefficient * s*b*h * bytes_per_elem (the page's worked example
+ * multiplies by 2 bytes for fp16).  SP_ERR_INVALID_ARG for non-positive
+ * sizes, an unknown mode or out == NULL.
+ */
+int sp_activation_bytes(int64_t s, int64_t b, int64_t h, int64_t a,
+                        int32_t t, int32_t mode, double bytes_per_elem,
+                        double* out);
+
+/* Static text for a status code. */
+const char* sp_status_string(int status);
+
+/* Reads the device-side error word of CUDA device `device` (0: none; else
+ * the code of the first bounded wait that ran out: 1 a consumer waiting for a
+ * staged row, 2 the producer waiting for a free stage, 3 an aborted CTA
+ * draining its copies, 9 the diagnostic below) and clears it when
+ * clear != 0.  Synchronises the device.  No counterpart on the pages: this
+ * is the library's failure detection. */
+int sp_device_error(int32_t device, int32_t* code, int32_t clear);
+
+/* Failure-detection diagnostic, no counterpart on the pages: launches one
+ * CTA that waits on an mbarrier nothing will complete, through the same
+ * bounded wait the streaming kernels use, with a limit of limit_ns
+ * (0 .. 10^10).  The wait must run out: the kernel writes *status = 1 (a
+ * device int32) and records code 9, and the context stays usable.  *status
+ * = 0 would mean the wait completed. */
+int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP_REGION_H */

@@ -1,0 +1,343 @@
+// Device helpers shared by the sm_100a kernels of the SP boundary:
+// mbarrier / bulk-copy wrappers with time-bounded waits, Philox4x32-10,
+// I/O-dtype packing, and fp32 reductions in a fixed order.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace spk {
+
+// ---------------------------------------------------------------------------
+// Device-side error word.  A bounded wait that runs out records its code here
+// (first error wins) and the kernel winds down instead of hanging; the host
+// reads it with sp_device_error().
+// ---------------------------------------------------------------------------
+__device__ unsigned int g_error;
+
+enum : unsigned {
+    ERR_WAIT_FULL = 1,      // a consumer waited too long for a staged row
+    ERR_WAIT_EMPTY = 2,     // the producer waited too long for a free stage
+    ERR_DRAIN = 3,          // an aborted CTA could not drain its copies
+    ERR_SELFTEST = 9,       // the diagnostic wait of sp_debug_wait_timeout
+};
+
+// Long enough that no legitimate wait on a B200 comes near it (a whole row
+// stream of the largest workload takes microseconds), short enough that a
+// lost copy surfaces as an error well inside any process timeout.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void record_error(unsigned code)
+{
+    atomicCAS(&g_error, 0u, code);
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier and bulk copy (PTX ISA: mbarrier.*, cp.async.bulk)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete.  Returns
+// false, without waiting further, once *abort is set or the time limit runs
+// out (which sets *abort and records `code`).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile int* abort, unsigned code,
+                                          unsigned long long limit_ns = kWaitLimitNs)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            record_error(code);
+            return false;
+        }
+    }
+}
+
+// One bulk copy global -> this CTA's shared memory, completing `bytes`
+// transaction bytes on `bar`.  dst and src 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+// L2 policy for data read exactly once.
+__device__ __forceinline__ uint64_t policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// Named barrier over the first `nthreads` threads of the CTA (the consumer
+// warps); the producer warp never takes part.
+__device__ __forceinline__ void consumer_sync(int nthreads)
+{
+    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
+// Easy as 1, 2, 3", SC'11).  Each round multiplies counter words 0 and 2 by
+// the two Philox constants; the new words are (hi1 ^ w1 ^ k0, lo1,
+// hi0 ^ w3 ^ k1, lo0), and the key advances by the two Weyl constants.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 philox4x32_10(uint4 w, uint32_t k0, uint32_t k1)
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const uint32_t lo0 = 0xD2511F53u * w.x;
+        const uint32_t hi0 = __umulhi(0xD2511F53u, w.x);
+        const uint32_t lo1 = 0xCD9E8D57u * w.z;
+        const uint32_t hi1 = __umulhi(0xCD9E8D57u, w.z);
+        w = make_uint4(hi1 ^ w.y ^ k0, lo1, hi0 ^ w.w ^ k1, lo0);
+        k0 += 0x9E3779B9u;
+        k1 += 0xBB67AE85u;
+    }
+    return w;
+}
+
+// Keep bits of the 8 features [8v, 8v+8) of token row n: counter
+// (q, n, offset lo, offset hi) for q = 2v and 2v+1, word j & 3 of each;
+// kept iff the word is >= thr.  Bit e of the result is feature 8v+e.
+__device__ __forceinline__ uint32_t keep_bits8(uint32_t v, uint32_t n, uint32_t off_lo,
+                                               uint32_t off_hi, uint32_t k0, uint32_t k1,
+                                               uint32_t thr)
+{
+    const uint4 a = philox4x32_10(make_uint4(2u * v, n, off_lo, off_hi), k0, k1);
+    const uint4 b = philox4x32_10(make_uint4(2u * v + 1u, n, off_lo, off_hi), k0, k1);
+    return (uint32_t)(a.x >= thr) | (uint32_t)(a.y >= thr) << 1 |
+           (uint32_t)(a.z >= thr) << 2 | (uint32_t)(a.w >= thr) << 3 |
+           (uint32_t)(b.x >= thr) << 4 | (uint32_t)(b.y >= thr) << 5 |
+           (uint32_t)(b.z >= thr) << 6 | (uint32_t)(b.w >= thr) << 7;
+}
+
+// Keep bit of one feature j of row n (general kernels).
+__device__ __forceinline__ uint32_t keep_bit(uint32_t j, uint32_t n, uint32_t off_lo,
+                                             uint32_t off_hi, uint32_t k0, uint32_t k1,
+                                             uint32_t thr)
+{
+    const uint4 a = philox4x32_10(make_uint4(j >> 2, n, off_lo, off_hi), k0, k1);
+    const uint32_t w = (j & 3) == 0 ? a.x : (j & 3) == 1 ? a.y : (j & 3) == 2 ? a.z : a.w;
+    return w >= thr ? 1u : 0u;
+}
+
+// ---------------------------------------------------------------------------
+// I/O dtype: 8 consecutive elements are one "vector" (16 B of bf16, 32 B of
+// fp32).  Arithmetic is always fp32; stores round to nearest-even.
+// ---------------------------------------------------------------------------
+template <typename T>
+struct IO;
+
+template <>
+struct IO<__nv_bfloat16> {
+    static constexpr int kBytes = 2;
+    static constexpr int kWords = 1;   // uint4 per vector
+    struct Vec {
+        uint4 u[1];
+    };
+
+    __device__ static __forceinline__ void unpack(const Vec& v, float f[8])
+    {
+        const uint32_t w[4] = {v.u[0].x, v.u[0].y, v.u[0].z, v.u[0].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+    __device__ static __forceinline__ uint32_t pack2(float a, float b)
+    {
+        __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // .x (low half) = a
+        return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ static __forceinline__ Vec pack(const float f[8])
+    {
+        Vec v;
+        v.u[0] = make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]),
+                            pack2(f[6], f[7]));
+        return v;
+    }
+    __device__ static __forceinline__ float load1(const void* p, long long i)
+    {
+        const uint16_t b = static_cast<const uint16_t*>(p)[i];
+        return __uint_as_float(static_cast<uint32_t>(b) << 16);
+    }
+    __device__ static __forceinline__ void store1(void* p, long long i, float x)
+    {
+        static_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
+    }
+    __device__ static __forceinline__ float round1(float x)
+    {
+        return __bfloat162float(__float2bfloat16_rn(x));
+    }
+};
+
+template <>
+struct IO<float> {
+    static constexpr int kBytes = 4;
+    static constexpr int kWords = 2;
+    struct Vec {
+        uint4 u[2];
+    };
+
+    __device__ static __forceinline__ void unpack(const Vec& v, float f[8])
+    {
+        f[0] = __uint_as_float(v.u[0].x);
+        f[1] = __uint_as_float(v.u[0].y);
+        f[2] = __uint_as_float(v.u[0].z);
+        f[3] = __uint_as_float(v.u[0].w);
+        f[4] = __uint_as_float(v.u[1].x);
+        f[5] = __uint_as_float(v.u[1].y);
+        f[6] = __uint_as_float(v.u[1].z);
+        f[7] = __uint_as_float(v.u[1].w);
+    }
+    __device__ static __forceinline__ Vec pack(const float f[8])
+    {
+        Vec v;
+        v.u[0] = make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
+                            __float_as_uint(f[2]), __float_as_uint(f[3]));
+        v.u[1] = make_uint4(__float_as_uint(f[4]), __float_as_uint(f[5]),
+                            __float_as_uint(f[6]), __float_as_uint(f[7]));
+        return v;
+    }
+    __device__ static __forceinline__ float load1(const void* p, long long i)
+    {
+        return static_cast<const float*>(p)[i];
+    }
+    __device__ static __forceinline__ void store1(void* p, long long i, float x)
+    {
+        static_cast<float*>(p)[i] = x;
+    }
+    __device__ static __forceinline__ float round1(float x) { return x; }
+};
+
+template <typename T>
+__device__ __forceinline__ typename IO<T>::Vec load_vec(const void* base, long long v)
+{
+    typename IO<T>::Vec r;
+    const uint4* p = static_cast<const uint4*>(base) + v * IO<T>::kWords;
+#pragma unroll
+    for (int i = 0; i < IO<T>::kWords; ++i) r.u[i] = p[i];
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ void store_vec(void* base, long long v, const typename IO<T>::Vec& x)
+{
+    uint4* p = static_cast<uint4*>(base) + v * IO<T>::kWords;
+#pragma unroll
+    for (int i = 0; i < IO<T>::kWords; ++i) p[i] = x.u[i];
+}
+
+// ---------------------------------------------------------------------------
+// fp32 sums, deterministic: butterfly within the warp, then every consumer
+// thread adds the per-warp totals in warp order.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    return x;
+}
+
+// Sum over the C consumer threads; `red` holds >= C/32 floats and must not be
+// reused by the next call before every consumer has passed this one's barrier
+// (callers alternate two buffers).
+__device__ __forceinline__ float consumer_sum(float x, float* red, int C)
+{
+    x = warp_sum(x);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) red[warp] = x;
+    consumer_sync(C);
+    float s = 0.f;
+    for (int w = 0; w < (C >> 5); ++w) s += red[w];
+    return s;
+}
+
+__device__ __forceinline__ float2 consumer_sum2(float2 x, float2* red, int C)
+{
+    x.x = warp_sum(x.x);
+    x.y = warp_sum(x.y);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) red[warp] = x;
+    consumer_sync(C);
+    float2 s = make_float2(0.f, 0.f);
+    for (int w = 0; w < (C >> 5); ++w) {
+        s.x += red[w].x;
+        s.y += red[w].y;
+    }
+    return s;
+}
+
+// Block-wide sum for the general kernels (all threads take part).
+__device__ __forceinline__ float block_sum(float x, float* red)
+{
+    x = warp_sum(x);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    __syncthreads();   // red may still be read by a previous call
+    if (lane == 0) red[warp] = x;
+    __syncthreads();
+    float s = 0.f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];
+    return s;
+}
+
+}  // namespace spk

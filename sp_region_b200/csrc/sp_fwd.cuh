@@ -1,0 +1,367 @@
+// Forward of the SP boundary on sm_100a.
+//
+// Per token row n (rank r = n / (N/t) owns it), as the Megatron SP pages
+// describe the exit of a tensor-parallel region ("Sequence Parallelism
+// math", sections "The collective substitution" and "The move"; "SP:
+// Partition Activations Alongside TP", sections "Normalize and add residuals
+// by token" and "Connect SP and TP across a layer"):
+//   reduce-scatter of the t partial sums -> + bias -> inverted dropout ->
+//   + residual (stored in the I/O dtype) -> LayerNorm / RMSNorm -> written to
+//   every gathered replica (the all-gather).
+//
+// k_fwd_tma: persistent, one CTA per SM.  The last warp is a producer: one
+// lane streams whole row segments (partial k of row n, then the residual row)
+// from HBM into a ring of shared-memory stages with cp.async.bulk, each stage
+// completing on its own "full" mbarrier.  The other warps are consumers: each
+// thread owns V vectors of 8 features of the row, accumulates the t partials
+// from shared memory in fp32 registers, applies bias / dropout / residual,
+// and runs the two-pass mean / variance with fixed-order reductions.  The
+// ring keeps the next rows' segments in flight while a row is normalised.
+#pragma once
+
+#include "sp_device.cuh"
+
+namespace spk {
+
+constexpr int kMaxT = 64;
+constexpr int kFwdMaxConsumers = 512;
+
+struct FwdArgs {
+    const void* parts[kMaxT];
+    void* gathered[kMaxT];
+    const void* bias;
+    const void* residual;
+    const void* gamma;
+    const void* beta;
+    void* residual_out;
+    uint8_t* mask;          // bytes: [rows][mask_row_bytes]
+    float* mean;
+    float* rstd;
+    long long rows;
+    int h;
+    int hv;                 // h / 8 (fast kernel)
+    int t;
+    int n_gathered;
+    int stages;
+    uint32_t seg_bytes;     // h * elem bytes
+    uint32_t stage_stride;  // seg_bytes rounded up to 128
+    int mask_row_bytes;     // 4 * ceil(h / 32)
+    uint32_t param_off;     // shared-memory offsets (fast kernel): parameters,
+    uint32_t param_stride;  //   one slot of param_stride bytes each,
+    uint32_t tail_off;      //   then the barriers / scratch
+    float eps;
+    float h_f;
+    float scale;            // 1 / (1 - p)
+    uint32_t thr;           // floor(p * 2^32)
+    uint32_t seed_lo, seed_hi, off_lo, off_hi;
+    int dropout;            // p > 0
+};
+
+// Shared-memory tail after the ring: barriers, reduction scratch, abort flag.
+struct RingTail {
+    uint64_t full[64];
+    uint64_t empty[64];
+    float red0[32];
+    float red1[32];
+    int abort;
+};
+
+template <typename T, int V, bool LN>
+__global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
+    k_fwd_tma(const __grid_constant__ FwdArgs a)
+{
+    using Vec = typename IO<T>::Vec;
+    extern __shared__ __align__(128) unsigned char smem[];
+    RingTail* tail = reinterpret_cast<RingTail*>(smem + a.tail_off);
+    volatile int* abort = &tail->abort;
+    // gamma, beta, bias copies: each consumer thread stores and later reads
+    // only its own vectors, so no barrier orders them
+    unsigned char* sg = smem + a.param_off;
+    unsigned char* sb = sg + a.param_stride;
+    unsigned char* sc = sb + a.param_stride;
+
+    const int C = blockDim.x - 32;   // consumer threads
+    const int tid = threadIdx.x;
+    const int S = a.stages;
+
+    if (tid == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_addr(&tail->full[s]), 1);
+            mbar_init(smem_addr(&tail->empty[s]), C / 32);
+        }
+        tail->abort = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+
+    const int nsrc = a.t + 1;   // t partials, then the residual row
+
+    // ------------------------------------------------------------------ producer
+    if (tid >= C) {
+        if (tid != C) return;
+        const uint64_t pol = policy_evict_first();
+        uint32_t stage = 0, phase = 1;   // a fresh "empty" barrier counts as released
+        long long issued = 0;
+        bool ok = true;
+        for (long long n = blockIdx.x; n < a.rows && ok; n += gridDim.x) {
+            for (int k = 0; k < nsrc; ++k) {
+                if (!mbar_wait(smem_addr(&tail->empty[stage]), phase, abort, ERR_WAIT_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                const unsigned char* src =
+                    static_cast<const unsigned char*>(k < a.t ? a.parts[k] : a.residual) +
+                    (size_t)n * a.seg_bytes;
+                const uint32_t bar = smem_addr(&tail->full[stage]);
+                mbar_arrive_expect_tx(bar, a.seg_bytes);
+                bulk_load(smem_addr(smem + (size_t)stage * a.stage_stride), src, a.seg_bytes,
+                          bar, pol);
+                ++issued;
+                if (++stage == (uint32_t)S) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+        if (!ok) {
+            // wind down: let every copy already issued land before the CTA
+            // exits (its shared memory must not be released under a copy)
+            long long first = issued > S ? issued - S : 0;
+            for (long long i = first; i < issued; ++i) {
+                const uint32_t s = (uint32_t)(i % S);
+                const uint32_t par = (uint32_t)((i / S) & 1);
+                volatile int no_abort = 0;
+                if (!mbar_wait(smem_addr(&tail->full[s]), par, &no_abort, ERR_DRAIN)) break;
+            }
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------------ consumers
+    const int lane = tid & 31;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+        const int v = tid + i * C;
+        if (v < a.hv) {
+            store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
+            if (a.beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));
+            if (a.bias) store_vec<T>(sc, v, load_vec<T>(a.bias, v));
+        }
+    }
+
+    uint32_t stage = 0, phase = 0;
+    auto advance = [&]() {
+        if (++stage == (uint32_t)S) {
+            stage = 0;
+            phase ^= 1;
+        }
+    };
+    auto release = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&tail->empty[stage]));
+        advance();
+    };
+
+    for (long long n = blockIdx.x; n < a.rows; n += gridDim.x) {
+        float acc[V][8];
+        // reduce-scatter: sum of the t partial rows, k ascending
+        for (int k = 0; k < a.t; ++k) {
+            mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
+            const unsigned char* buf = smem + (size_t)stage * a.stage_stride;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int v = tid + i * C;
+                if (v < a.hv) {
+                    float f[8];
+                    IO<T>::unpack(load_vec<T>(buf, v), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[i][e] = (k == 0) ? f[e] : acc[i][e] + f[e];
+                }
+            }
+            release();
+        }
+
+        // bias once, then inverted dropout with the packed keep bits
+        uint8_t* mrow = a.mask ? a.mask + (size_t)n * a.mask_row_bytes : nullptr;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int v = tid + i * C;
+            if (v < a.hv) {
+                if (a.bias) {
+                    float f[8];
+                    IO<T>::unpack(load_vec<T>(sc, v), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
+                }
+                uint32_t kb = 0xFFu;
+                if (a.dropout) {
+                    kb = keep_bits8((uint32_t)v, (uint32_t)n, a.off_lo, a.off_hi, a.seed_lo,
+                                    a.seed_hi, a.thr);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        acc[i][e] = ((kb >> e) & 1u) ? acc[i][e] * a.scale : 0.f;
+                }
+                if (mrow) mrow[v] = (uint8_t)kb;
+            }
+        }
+        if (mrow && tid == 0)
+            for (int pbyte = a.hv; pbyte < a.mask_row_bytes; ++pbyte) mrow[pbyte] = 0;
+
+        // residual add; the sum is stored in the I/O dtype and the norm reads
+        // the stored (rounded) value
+        mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
+        {
+            const unsigned char* buf = smem + (size_t)stage * a.stage_stride;
+            unsigned char* rout = static_cast<unsigned char*>(a.residual_out) +
+                                  (size_t)n * a.seg_bytes;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int v = tid + i * C;
+                if (v < a.hv) {
+                    float f[8];
+                    IO<T>::unpack(load_vec<T>(buf, v), f);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] += acc[i][e];
+                    const Vec r = IO<T>::pack(f);
+                    store_vec<T>(rout, v, r);
+                    IO<T>::unpack(r, acc[i]);
+                }
+            }
+        }
+        release();
+
+        // per-token norm, two passes over the row held in registers
+        float mean = 0.f, rstd;
+        if (LN) {
+            float s = 0.f;
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                if (tid + i * C < a.hv)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) s += acc[i][e];
+            mean = consumer_sum(s, tail->red0, C) / a.h_f;
+            float q = 0.f;
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                if (tid + i * C < a.hv)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float d = acc[i][e] - mean;
+                        q += d * d;
+                    }
+            const float var = consumer_sum(q, tail->red1, C) / a.h_f;
+            rstd = 1.0f / sqrtf(var + a.eps);
+        } else {
+            float q = 0.f;
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                if (tid + i * C < a.hv)
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) q += acc[i][e] * acc[i][e];
+            const float ms = consumer_sum(q, tail->red0, C) / a.h_f;
+            rstd = 1.0f / sqrtf(ms + a.eps);
+        }
+
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int v = tid + i * C;
+            if (v < a.hv) {
+                float g[8], b[8], o[8];
+                IO<T>::unpack(load_vec<T>(sg, v), g);
+                if (LN && a.beta) {
+                    IO<T>::unpack(load_vec<T>(sb, v), b);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) b[e] = 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    o[e] = LN ? (acc[i][e] - mean) * rstd * g[e] + b[e]
+                              : acc[i][e] * rstd * g[e];
+                const Vec ov = IO<T>::pack(o);
+                for (int q = 0; q < a.n_gathered; ++q)
+                    store_vec<T>(static_cast<unsigned char*>(a.gathered[q]) +
+                                     (size_t)n * a.seg_bytes,
+                                 v, ov);
+            }
+        }
+        if (tid == 0) {
+            if (LN && a.mean) a.mean[n] = mean;
+            if (a.rstd) a.rstd[n] = rstd;
+        }
+    }
+}
+
+// General forward: any h, element-aligned pointers.  One CTA per row (grid
+// stride); the row's residual sum is kept in shared memory as fp32.
+template <typename T, bool LN>
+__global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ FwdArgs a)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    float* xs = reinterpret_cast<float*>(smem);
+    uint32_t* mw = reinterpret_cast<uint32_t*>(xs + a.h);
+    const int W = a.mask_row_bytes / 4;
+    __shared__ float red[32];
+    const int h = a.h;
+
+    for (long long n = blockIdx.x; n < a.rows; n += gridDim.x) {
+        for (int w = threadIdx.x; w < W; w += blockDim.x) mw[w] = 0u;
+        __syncthreads();
+        const long long base = n * (long long)h;
+        for (int j = threadIdx.x; j < h; j += blockDim.x) {
+            float y = 0.f;
+            for (int k = 0; k < a.t; ++k) y = (k == 0) ? IO<T>::load1(a.parts[k], base + j)
+                                                       : y + IO<T>::load1(a.parts[k], base + j);
+            if (a.bias) y += IO<T>::load1(a.bias, j);
+            uint32_t keep = 1u;
+            if (a.dropout) {
+                keep = keep_bit((uint32_t)j, (uint32_t)n, a.off_lo, a.off_hi, a.seed_lo,
+                                a.seed_hi, a.thr);
+                y = keep ? y * a.scale : 0.f;
+            }
+            if (keep) atomicOr(&mw[j >> 5], 1u << (j & 31));
+            const float r = IO<T>::round1(IO<T>::load1(a.residual, base + j) + y);
+            IO<T>::store1(a.residual_out, base + j, r);
+            xs[j] = r;
+        }
+        __syncthreads();
+        if (a.mask) {
+            uint32_t* mrow = reinterpret_cast<uint32_t*>(a.mask + (size_t)n * a.mask_row_bytes);
+            for (int w = threadIdx.x; w < W; w += blockDim.x) mrow[w] = mw[w];
+        }
+        float mean = 0.f, rstd;
+        if (LN) {
+            float s = 0.f;
+            for (int j = threadIdx.x; j < h; j += blockDim.x) s += xs[j];
+            mean = block_sum(s, red) / a.h_f;
+            float q = 0.f;
+            for (int j = threadIdx.x; j < h; j += blockDim.x) {
+                const float d = xs[j] - mean;
+                q += d * d;
+            }
+            rstd = 1.0f / sqrtf(block_sum(q, red) / a.h_f + a.eps);
+        } else {
+            float q = 0.f;
+            for (int j = threadIdx.x; j < h; j += blockDim.x) q += xs[j] * xs[j];
+            rstd = 1.0f / sqrtf(block_sum(q, red) / a.h_f + a.eps);
+        }
+        for (int j = threadIdx.x; j < h; j += blockDim.x) {
+            const float g = IO<T>::load1(a.gamma, j);
+            float o;
+            if (LN) {
+                const float b = a.beta ? IO<T>::load1(a.beta, j) : 0.f;
+                o = (xs[j] - mean) * rstd * g + b;
+            } else {
+                o = xs[j] * rstd * g;
+            }
+            for (int q = 0; q < a.n_gathered; ++q) IO<T>::store1(a.gathered[q], base + j, o);
+        }
+        if (threadIdx.x == 0) {
+            if (LN && a.mean) a.mean[n] = mean;
+            if (a.rstd) a.rstd[n] = rstd;
+        }
+        __syncthreads();   // xs / mw are reused by the next row
+    }
+}
+
+}  // namespace spk

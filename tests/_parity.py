@@ -1,0 +1,260 @@
+"""Helpers for the GPU-vs-oracle parity tests: guarded output buffers,
+GPU calls through the C ABI, and the tolerance bounds.
+
+Tolerances.  The oracle computes in float64 and rounds once to the I/O dtype;
+the kernels compute in fp32 and round once.  An output that is a short fp32
+expression of terms bounded by M carries an absolute fp32 error of at most
+k * 2^-24 * M before its final rounding, and the final rounding can then land
+on the neighbouring value of the I/O dtype.  So an element passes when
+
+    |gpu - ref| <= ulp_io(ref) + k * 2^-24 * M        (bf16)
+    |gpu - ref| <= 1e-5 |ref| + 1e-6 + k * 2^-24 * M  (fp32)
+
+with M computed per element from the inputs' magnitudes and k = 16.  Sums over
+all tokens (dgamma, dbeta, dbias) pass when |gpu - ref| <= 1e-5 * sum|terms|
++ 1e-6.  Masks, layouts and shard offsets must match bit for bit.
+"""
+import numpy as np
+import torch
+
+import sp_region_b200 as sp
+
+GUARD = 64          # elements of canary on each side of every output
+K_FP32 = 16
+
+
+def _canary(dtype):
+    # a NaN payload no kernel writes
+    if dtype == torch.bfloat16:
+        return torch.tensor([0x7FA5], dtype=torch.int16).view(torch.bfloat16)
+    if dtype == torch.float32:
+        return torch.tensor([0x7FA5A5A5], dtype=torch.int32).view(torch.float32)
+    if dtype == torch.int32:
+        return torch.tensor([0x5A5AA5A5], dtype=torch.int32)
+    raise TypeError(dtype)
+
+
+class Guarded:
+    """A device buffer with canary bands; ``.t`` is the usable view."""
+
+    def __init__(self, shape, dtype, device="cuda", offset_elems=0):
+        n = int(np.prod(shape))
+        self.full = torch.empty(n + 2 * GUARD + offset_elems, dtype=dtype,
+                                device=device)
+        self.full.view(torch.uint8).fill_(0)
+        c = _canary(dtype).to(device)
+        self.full[:GUARD + offset_elems] = c
+        self.full[GUARD + offset_elems + n:] = c
+        self.lo = GUARD + offset_elems
+        self.n = n
+        self.t = self.full[self.lo:self.lo + n].view(shape)
+        self.dtype = dtype
+
+    def intact(self):
+        c = _canary(self.dtype).to(self.full.device)
+        iv = torch.int16 if self.dtype == torch.bfloat16 else torch.int32
+        cb = c.view(iv)
+        head = self.full[:self.lo].view(iv)
+        tail = self.full[self.lo + self.n:].view(iv)
+        return bool((head == cb).all()) and bool((tail == cb).all())
+
+
+def ulp_io(x, dtype):
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    bits = 8 if dtype == torch.bfloat16 else 24
+    e = np.floor(np.log2(np.maximum(x, 2.0 ** -126)))
+    return 2.0 ** (e - (bits - 1))
+
+
+def assert_close(name, gpu, ref, mag, dtype, k=K_FP32):
+    g = np.asarray(gpu.double().cpu() if isinstance(gpu, torch.Tensor)
+                   else gpu, dtype=np.float64)
+    r = np.asarray(ref.double().cpu() if isinstance(ref, torch.Tensor)
+                   else ref, dtype=np.float64)
+    m = np.asarray(mag, dtype=np.float64)
+    d = np.abs(g - r)
+    if dtype == torch.bfloat16:
+        tol = ulp_io(r, dtype) + k * 2.0 ** -24 * m
+    else:
+        tol = 1e-5 * np.abs(r) + 1e-6 + k * 2.0 ** -24 * m
+    bad = ~(d <= tol)
+    if bad.any():
+        idx = np.argwhere(bad)[:5]
+        lines = [f"{name}: {int(bad.sum())} of {bad.size} outside tolerance"]
+        for i in idx:
+            i = tuple(i)
+            lines.append(f"  at {i}: gpu={g[i]!r} ref={r[i]!r} tol={tol[i]!r}")
+        raise AssertionError("\n".join(lines))
+
+
+def assert_sum_close(name, gpu, ref, abs_terms):
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    tol = 1e-5 * np.asarray(abs_terms, dtype=np.float64) + 1e-6
+    bad = ~(np.abs(g - r) <= tol)
+    if bad.any():
+        i = int(np.argwhere(bad)[0][0])
+        raise AssertionError(f"{name}: {int(bad.sum())} outside; at {i} "
+                             f"gpu={g[i]} ref={r[i]} tol={tol[i]}")
+
+
+def unpack_mask(words, h):
+    """[rows, W] uint32 -> [rows, h] keep bits (bit j&31 of word j>>5)."""
+    w = np.ascontiguousarray(np.asarray(words, dtype=np.uint32))
+    bits = np.unpackbits(w.view(np.uint8), bitorder="little")
+    return bits.reshape(w.shape[0], -1)[:, :h]
+
+
+def cfg_of(w):
+    return sp.make_cfg(w.s, w.b, w.h, w.t, dtype=w.dtype, norm=w.norm,
+                       eps=w.eps, p_drop=w.p_drop, seed=w.drop_seed,
+                       offset=w.drop_offset)
+
+
+def gpu_fwd(w, parts, bias, residual, gamma, beta, n_gathered=1,
+            with_mask=True, with_stats=True, inplace=False, offset_elems=0):
+    """Run the forward through the C ABI on device copies of the inputs.
+
+    offset_elems shifts every [s,b,h] buffer by that many elements from a
+    16-byte boundary (exercises the general kernel)."""
+    dev = "cuda"
+    dt = w.torch_dtype
+    N, h = w.rows, w.h
+    W = (h + 31) // 32
+
+    def dcopy(x):
+        if x is None:
+            return None, None
+        g = Guarded(tuple(x.shape), dt, dev, offset_elems)
+        g.t.copy_(x.to(dev))
+        return g, g.t
+
+    gp = [dcopy(p) for p in parts]
+    gres, res_t = dcopy(residual)
+    gb = dcopy(bias)[1]
+    gg = dcopy(gamma)[1]
+    gbe = dcopy(beta)[1]
+    if inplace:
+        rout_g, rout = gres, res_t
+    else:
+        rout_g = Guarded((N, h), dt, dev, offset_elems)
+        rout = rout_g.t
+    gath = [Guarded((N, h), dt, dev, offset_elems) for _ in range(n_gathered)]
+    mask_g = Guarded((N, W), torch.int32, dev) if with_mask else None
+    mean_g = Guarded((N,), torch.float32, dev) if with_stats else None
+    rstd_g = Guarded((N,), torch.float32, dev) if with_stats else None
+    sp.sp_rs_bias_dropout_add_norm_fwd(
+        cfg_of(w), [g.t for g, _ in gp], gb, res_t, gg, gbe, rout,
+        [g.t for g in gath],
+        mask_bits=mask_g.t if mask_g else None,
+        mean=mean_g.t if mean_g else None, rstd=rstd_g.t if rstd_g else None)
+    torch.cuda.synchronize()
+    assert sp.sp_device_error() == 0
+    for g in [rout_g, *gath, mask_g, mean_g, rstd_g]:
+        if g is not None:
+            assert g.intact(), "canary overwritten"
+    return dict(
+        residual_out=rout.cpu(), gathered=[g.t.cpu() for g in gath],
+        mask=(mask_g.t.cpu().numpy().view(np.uint32) if mask_g else None),
+        mean=mean_g.t.cpu().numpy() if mean_g else None,
+        rstd=rstd_g.t.cpu().numpy() if rstd_g else None)
+
+
+def gpu_bwd(w, dparts, drnext, x, gamma, mask, mean, rstd, with_dbeta=True,
+            with_dbias=True, offset_elems=0):
+    dev = "cuda"
+    dt = w.torch_dtype
+    N, h = w.rows, w.h
+
+    def dcopy(x_, dtype=dt, off=offset_elems):
+        if x_ is None:
+            return None
+        g = Guarded(tuple(x_.shape), dtype, dev, off)
+        g.t.copy_(torch.as_tensor(x_).to(dev))
+        return g.t
+
+    dp = [dcopy(p) for p in dparts]
+    drn = dcopy(drnext)
+    xt = dcopy(x)
+    gt = dcopy(gamma)
+    mt = (None if mask is None else
+          dcopy(torch.from_numpy(np.ascontiguousarray(mask).view(np.int32)),
+                torch.int32, 0))
+    mean_t = (None if mean is None else
+              dcopy(torch.from_numpy(np.asarray(mean, np.float32)),
+                    torch.float32, 0))
+    rstd_t = dcopy(torch.from_numpy(np.asarray(rstd, np.float32)),
+                   torch.float32, 0)
+    dres_g = Guarded((N, h), dt, dev, offset_elems)
+    dy_g = Guarded((N, h), dt, dev, offset_elems)
+    dgam_g = Guarded((h,), torch.float32, dev)
+    dbet_g = Guarded((h,), torch.float32, dev) if with_dbeta else None
+    dbia_g = Guarded((h,), torch.float32, dev) if with_dbias else None
+    cfg = cfg_of(w)
+    nws = sp.sp_bwd_workspace_bytes(cfg)
+    ws = torch.empty(nws // 4 + 4, dtype=torch.float32, device=dev)
+    ws.fill_(float("nan"))   # the kernel must not need zeroed scratch
+    sp.sp_rs_norm_dropout_bwd(
+        cfg, dp, drn, xt, gt, mt, mean_t, rstd_t, dres_g.t, dy_g.t, dgam_g.t,
+        dbet_g.t if dbet_g else None, dbia_g.t if dbia_g else None, ws)
+    torch.cuda.synchronize()
+    assert sp.sp_device_error() == 0
+    for g in [dres_g, dy_g, dgam_g, dbet_g, dbia_g]:
+        if g is not None:
+            assert g.intact(), "canary overwritten"
+    return dict(dresidual_in=dres_g.t.cpu(), dY=dy_g.t.cpu(),
+                dgamma=dgam_g.t.cpu().numpy(),
+                dbeta=dbet_g.t.cpu().numpy() if dbet_g else None,
+                dbias=dbia_g.t.cpu().numpy() if dbia_g else None)
+
+
+# ----------------------------------------------------------------------------
+# magnitudes for the tolerance bounds (float64, from inputs and oracle data)
+# ----------------------------------------------------------------------------
+
+def mag_residual_out(w, parts, bias, residual):
+    scale = 1.0 / (1.0 - float(np.float32(w.p_drop)))
+    m = sum(p.double().abs() for p in parts)
+    if bias is not None:
+        m = m + bias.double().abs()
+    return (residual.double().abs() + scale * m).numpy()
+
+
+def mag_norm_out(w, x, mean, rstd, gamma, beta):
+    x = x.double()
+    rs = torch.from_numpy(np.asarray(rstd, np.float64))[:, None]
+    if w.norm == "layernorm":
+        mu = torch.from_numpy(np.asarray(mean, np.float64))[:, None]
+        xh = (x - mu) * rs
+    else:
+        xh = x * rs
+    g = gamma.double().abs()
+    m = (xh.abs() * g + g)
+    if beta is not None and w.norm == "layernorm":
+        m = m + beta.double().abs()
+    return m.numpy()
+
+
+def mags_backward(w, dparts, drnext, x, gamma, mean, rstd):
+    """Magnitude bounds for dresidual_in and dY, and the |terms| of the
+    parameter-gradient sums."""
+    scale = 1.0 / (1.0 - float(np.float32(w.p_drop)))
+    x = x.double()
+    rs = torch.from_numpy(np.asarray(rstd, np.float64))[:, None]
+    if w.norm == "layernorm":
+        mu = torch.from_numpy(np.asarray(mean, np.float64))[:, None]
+        xh = (x - mu) * rs
+    else:
+        xh = x * rs
+    g = gamma.double()
+    absd = sum(d.double().abs() for d in dparts)
+    dn = sum(d.double() for d in dparts)
+    gg = (absd * g.abs())
+    m = rs * (gg + gg.mean(1, keepdim=True)
+              + xh.abs() * (gg * xh.abs()).mean(1, keepdim=True))
+    if drnext is not None:
+        m = m + drnext.double().abs()
+    return dict(dres=m.numpy(), dY=(scale * m).numpy(),
+                dgamma_terms=(dn.abs() * xh.abs()).sum(0).numpy(),
+                dbeta_terms=dn.abs().sum(0).numpy(),
+                dbias_terms=(scale * m).sum(0).numpy())

@@ -1,0 +1,158 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and its host-only logic (closed forms, status strings,
+argument validation before any device call) behaves as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sp_region.h")
+LIB = os.path.join(ROOT, "sp_region_b200", "libsp_region.so")
+
+
+def _header_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(sp_\w+)\s*\(", src,
+                       flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sp_region_b200 import build
+    build.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_boundary_calls():
+    names = _header_functions()
+    for required in ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
+                     "sp_rs_norm_dropout_bwd", "sp_activation_bytes"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol():
+    import sp_region_b200 as sp
+    assert sorted(sp.EXPORTS) == _header_functions()
+    for name in _header_functions():
+        assert callable(getattr(sp, name)), name
+
+
+def test_status_strings():
+    import sp_region_b200 as sp
+    assert sp.sp_status_string(0) == "ok"
+    assert "invalid" in sp.sp_status_string(1)
+    assert sp.sp_status_string(99) == "unknown status"
+
+
+def test_activation_bytes_matches_oracle(orc):
+    import sp_region_b200 as sp
+    for (s, b, h, a, t) in [(2048, 4, 12288, 96, 8), (32768, 1, 12288, 96, 16),
+                            (4096, 1, 8192, 64, 8), (4, 1, 4, 1, 2),
+                            (2048, 4, 6144, 48, 1)]:
+        for mode in (0, 1, 2):
+            for bpe in (1.0, 2.0):
+                got = sp.sp_activation_bytes(s, b, h, a, t, mode, bpe)
+                ref = orc.activation_bytes(s, b, h, a, t, mode, bpe)
+                assert got == pytest.approx(ref, rel=1e-15)
+
+
+def test_activation_bytes_rejects_bad_arguments():
+    import sp_region_b200 as sp
+    for args in [(0, 1, 1, 1, 1, 0, 2.0), (1, 1, 1, 1, 0, 0, 2.0),
+                 (1, 1, 1, 1, 1, 3, 2.0), (1, 1, 1, 1, 1, 0, 0.0)]:
+        with pytest.raises(sp.SPError) as e:
+            sp.sp_activation_bytes(*args)
+        assert e.value.status == sp.SP_ERR_INVALID_ARG
+
+
+def _fake_call_fwd(lib, cfg, t, n_gathered=1, ptr=0x1000):
+    """Call the forward with fake (never dereferenced) pointers; every case
+    here must be rejected by host validation before any CUDA call."""
+    import sp_region_b200 as sp
+    parts = (ctypes.c_void_p * max(t, 1))(*([ptr] * max(t, 1)))
+    outs = (ctypes.c_void_p * max(n_gathered, 1))(*([ptr] * max(n_gathered, 1)))
+    return lib.sp_rs_bias_dropout_add_norm_fwd(
+        ctypes.byref(cfg), parts, None, ctypes.c_void_p(ptr),
+        ctypes.c_void_p(ptr), None, ctypes.c_void_p(ptr), outs, n_gathered,
+        None, None, None, None)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(s=6, t=4),               # s % t != 0
+    dict(t=0), dict(t=65),        # t out of range
+    dict(h=0), dict(s=0), dict(b=0),
+    dict(p_drop=1.0), dict(p_drop=-0.1), dict(p_drop=float("nan")),
+    dict(eps=0.0), dict(eps=float("inf")),
+    dict(dtype=7), dict(norm=5),
+    dict(s=2 ** 33, t=1),         # token row beyond the 32-bit counter
+])
+def test_forward_validation_rejects_before_launch(lib, bad):
+    import sp_region_b200 as sp
+    kw = dict(s=8, b=2, h=64, t=4, dtype="bf16", norm="layernorm", eps=1e-5,
+              p_drop=0.1)
+    cfg = sp.make_cfg(**{k: v for k, v in kw.items()
+                         if k not in ("dtype", "norm")},
+                      dtype="bf16", norm="layernorm")
+    for k, v in bad.items():
+        setattr(cfg, k, v)
+    t = max(1, min(int(cfg.t), 64))
+    assert _fake_call_fwd(lib, cfg, t) == sp.SP_ERR_INVALID_ARG
+
+
+def test_forward_rejects_null_and_misaligned(lib):
+    import sp_region_b200 as sp
+    cfg = sp.make_cfg(8, 2, 64, 4, dtype="bf16", p_drop=0.1)
+    # n_gathered out of range
+    assert _fake_call_fwd(lib, cfg, 4, n_gathered=0) == sp.SP_ERR_INVALID_ARG
+    assert _fake_call_fwd(lib, cfg, 4, n_gathered=65) == sp.SP_ERR_INVALID_ARG
+    # a pointer not aligned to the element size
+    assert _fake_call_fwd(lib, cfg, 4, ptr=0x1001) == sp.SP_ERR_INVALID_ARG
+    # NULL residual
+    parts = (ctypes.c_void_p * 4)(*([0x1000] * 4))
+    outs = (ctypes.c_void_p * 1)(0x1000)
+    rc = lib.sp_rs_bias_dropout_add_norm_fwd(
+        ctypes.byref(cfg), parts, None, None, ctypes.c_void_p(0x1000), None,
+        ctypes.c_void_p(0x1000), outs, 1, None, None, None, None)
+    assert rc == sp.SP_ERR_INVALID_ARG
+
+
+def test_backward_validation(lib):
+    import sp_region_b200 as sp
+    cfg = sp.make_cfg(8, 2, 64, 4, dtype="bf16", p_drop=0.1)
+    P = ctypes.c_void_p(0x1000)
+    parts = (ctypes.c_void_p * 4)(*([0x1000] * 4))
+    # p > 0 needs the mask
+    rc = lib.sp_rs_norm_dropout_bwd(ctypes.byref(cfg), parts, None, P, P, None,
+                                    P, P, P, P, P, None, None, P, 1 << 20, None)
+    assert rc == sp.SP_ERR_INVALID_ARG
+    # LayerNorm needs mean
+    rc = lib.sp_rs_norm_dropout_bwd(ctypes.byref(cfg), parts, None, P, P, P,
+                                    None, P, P, P, P, None, None, P, 1 << 20,
+                                    None)
+    assert rc == sp.SP_ERR_INVALID_ARG
+    # workspace must be 16-byte aligned
+    rc = lib.sp_rs_norm_dropout_bwd(ctypes.byref(cfg), parts, None, P, P, P,
+                                    P, P, P, P, P, None, None,
+                                    ctypes.c_void_p(0x1008), 1 << 20, None)
+    assert rc == sp.SP_ERR_INVALID_ARG
+
+
+def test_all_gather_validation(lib):
+    import sp_region_b200 as sp
+    cfg = sp.make_cfg(8, 2, 64, 4, dtype="bf16")
+    sh = (ctypes.c_void_p * 4)(*([0x1000] * 4))
+    outs = (ctypes.c_void_p * 1)(0x1000)
+    assert lib.sp_all_gather(ctypes.byref(cfg), sh, outs, 0, None) == \
+        sp.SP_ERR_INVALID_ARG
+    cfg.s = 7
+    assert lib.sp_all_gather(ctypes.byref(cfg), sh, outs, 1, None) == \
+        sp.SP_ERR_INVALID_ARG
