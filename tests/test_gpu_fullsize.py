@@ -19,7 +19,8 @@ import torch
 import oracle
 import sp_synth
 from sp_synth import WORKLOADS
-from _parity import (assert_close, assert_sum_close, gpu_bwd, mag_norm_out,
+from _parity import (assert_close, assert_sum_close, check_forward,
+                     gpu_bwd, mag_norm_out,
                      mag_residual_out, mags_backward, cfg_of)
 
 import sp_region_b200 as sp
@@ -72,16 +73,10 @@ def _check_full_fwd(w, n_gathered=1):
         w, [p.cuda() for p in parts], d(bias), d(res), d(gamma), d(beta),
         n_gathered)
     ref = oracle.fwd(oracle.cfg_from(w), parts, bias, res, gamma, beta)
-    dt = w.torch_dtype
-    assert_close("residual_out", rout.cpu(), ref["residual_out"],
-                 mag_residual_out(w, parts, bias, res), dt)
-    mag = mag_norm_out(w, ref["residual_out"], ref["mean"], ref["rstd"],
-                       gamma, beta)
-    for q in range(n_gathered):
-        assert_close(f"gathered[{q}]", gath[q].cpu(), ref["gathered"][0], mag,
-                     dt)
-    assert np.array_equal(mask.cpu().numpy().view(np.uint32), ref["mask"])
-    assert np.allclose(rstd.cpu().numpy(), ref["rstd"], rtol=1e-5, atol=0)
+    got = dict(residual_out=rout.cpu(), gathered=[g.cpu() for g in gath],
+               mask=mask.cpu().numpy().view(np.uint32),
+               mean=mean.cpu().numpy(), rstd=rstd.cpu().numpy())
+    check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered)
     return parts, bias, res, gamma, beta, ref
 
 
@@ -182,14 +177,10 @@ def test_c5_long_sequence_forward_backward_sampled():
     rrow = res_d[idx].cpu()
     ref = oracle.fwd_rows(cfg, rows, prow, bias, rrow, gamma, beta)
     dt = w.torch_dtype
-    assert_close("residual_out rows", rout[idx].cpu(), ref["residual_out"],
-                 mag_residual_out(w, prow, bias, rrow), dt)
-    assert_close("gathered rows", gath[0][idx].cpu(), ref["norm_out"],
-                 mag_norm_out(w, ref["residual_out"], ref["mean"],
-                              ref["rstd"], gamma, beta), dt)
-    assert np.array_equal(mask[idx].cpu().numpy().view(np.uint32),
-                          ref["mask"])
-    assert np.allclose(rstd[idx].cpu().numpy(), ref["rstd"], rtol=1e-5)
+    got = dict(residual_out=rout[idx].cpu(), norm_out=gath[0][idx].cpu(),
+               mask=mask[idx].cpu().numpy().view(np.uint32),
+               mean=mean[idx].cpu().numpy(), rstd=rstd[idx].cpu().numpy())
+    check_forward(w, got, ref, prow, bias, rrow, gamma, beta)
     # keep rate over the whole mask, within 6 sigma of the binomial
     kept = int(torch.bitwise_count(mask.view(torch.int32)).sum().item()) \
         if hasattr(torch, "bitwise_count") else int(

@@ -15,7 +15,8 @@ import torch
 import oracle
 import sp_synth
 from sp_synth import WORKLOADS
-from _parity import (assert_close, assert_sum_close, gpu_bwd, gpu_fwd,
+from _parity import (assert_close, assert_sum_close, check_forward,
+                     gpu_bwd, gpu_fwd,
                      mag_norm_out, mag_residual_out, mags_backward,
                      unpack_mask, cfg_of, Guarded)
 
@@ -43,22 +44,7 @@ def _inputs(w, device="cpu"):
 
 
 def _check_fwd(w, got, ref, parts, bias, res, gamma, beta, n_gathered=1):
-    dt = w.torch_dtype
-    assert_close("residual_out", got["residual_out"], ref["residual_out"],
-                 mag_residual_out(w, parts, bias, res), dt)
-    mag = mag_norm_out(w, ref["residual_out"], ref["mean"], ref["rstd"],
-                       gamma, beta)
-    for q in range(n_gathered):
-        assert_close(f"gathered[{q}]", got["gathered"][q],
-                     ref["gathered"][0], mag, dt)
-    if got["mask"] is not None:
-        assert np.array_equal(got["mask"], ref["mask"]), "mask bits differ"
-    if got["rstd"] is not None:
-        assert np.allclose(got["rstd"], ref["rstd"], rtol=1e-5, atol=0)
-        if w.norm == "layernorm":
-            x = ref["residual_out"].double()
-            rms = x.pow(2).mean(1).sqrt().numpy()
-            assert (np.abs(got["mean"] - ref["mean"]) <= 1e-5 * rms).all()
+    check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered)
 
 
 FWD_CASES = {
@@ -78,7 +64,7 @@ FWD_CASES = {
     "bf16_t64_h64": dict(base="C2", s=128, b=1, h=64, t=64),
     "bf16_h8_one_vector": dict(base="C2", s=16, b=1, h=8, t=2),
     "bf16_single_row": dict(base="C2", s=1, b=1, h=6144, t=1),
-    "bf16_rms_no_bias_p01": dict(base="C3", s=64, b=2, h=1536, t=4,
+    "bf16_rms_bias_p01": dict(base="C3", s=64, b=2, h=1536, t=4,
                                  p_drop=0.1, has_bias=True),
     "bf16_seed_offset": dict(base="C2", s=32, b=1, h=768, t=2,
                              drop_seed=0xFEEDFACECAFEBEEF,
