@@ -201,7 +201,8 @@ def run_ours(args):
     N, h, t = w.rows, w.h, w.t
     dt = w.torch_dtype
     cfg = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm, eps=w.eps,
-                      p_drop=w.p_drop, seed=w.drop_seed, offset=w.drop_offset)
+                      p_drop=w.p_drop, seed=w.drop_seed, offset=w.drop_offset,
+                      fwd_plan=args.fwd_plan, bwd_plan=args.bwd_plan)
 
     parts = sp_synth.draw_partials(w, dev)
     bias, gamma, beta = sp_synth.draw_params(w, dev)
@@ -332,6 +333,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 3 * K,
+        "plan_hints": {"fwd": args.fwd_plan, "bwd": args.bwd_plan},
         "clocks": clocks.summary(h0, h1),
     }
     if world > 1:
@@ -527,6 +529,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=4)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-plan", type=int, default=0,
+                    help="forward kernel plan hint (0: library's choice)")
+    ap.add_argument("--bwd-plan", type=int, default=0,
+                    help="backward kernel plan hint (0: library's choice)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

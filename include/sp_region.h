@@ -88,7 +88,15 @@ typedef enum { SP_LAYERNORM = 0, SP_RMSNORM = 1 } sp_norm;
  *   eps      added to the variance (LayerNorm) or the mean square (RMSNorm)
  *            inside the square root
  *   p_drop   dropout probability in [0, 1)
- *   seed, offset   Philox4x32-10 key and counter offset of the dropout mask */
+ *   seed, offset   Philox4x32-10 key and counter offset of the dropout mask
+ *   fwd_plan, bwd_plan   kernel configuration hints, no counterpart on the
+ *            pages: 0 lets the library choose; k > 0 asks for fast-kernel
+ *            plan k-1 of the forward / backward plan tables (vectors per
+ *            thread, consumer groups per CTA, block size) when that plan
+ *            fits the shape, else the library chooses.  Results do not
+ *            depend on the plan except through the fp32 summation order of
+ *            the backward's parameter gradients.  Out-of-range values are
+ *            treated as 0. */
 typedef struct {
     int64_t s, b, h;
     int32_t t;
@@ -97,7 +105,12 @@ typedef struct {
     float eps;
     float p_drop;
     uint64_t seed, offset;
+    int32_t fwd_plan, bwd_plan;
 } sp_cfg;
+
+/* Number of fast-kernel plans of the forward and the backward (valid hint
+ * values are 1 .. count). */
+int sp_plan_count(int32_t* fwd_plans, int32_t* bwd_plans);
 
 /*
  * Forward of the boundary: reduce-scatter + bias + dropout + residual add +

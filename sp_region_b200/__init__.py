@@ -32,7 +32,7 @@ SP_MAX_T = 64
 EXPORTS = ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
            "sp_rs_norm_dropout_bwd", "sp_bwd_workspace_bytes",
            "sp_activation_bytes", "sp_status_string", "sp_device_error",
-           "sp_debug_wait_timeout")
+           "sp_debug_wait_timeout", "sp_plan_count")
 
 
 class SPError(RuntimeError):
@@ -46,14 +46,15 @@ class sp_cfg(ctypes.Structure):
                 ("h", ctypes.c_int64), ("t", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("norm", ctypes.c_int32),
                 ("eps", ctypes.c_float), ("p_drop", ctypes.c_float),
-                ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64),
+                ("fwd_plan", ctypes.c_int32), ("bwd_plan", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
             f"{LIB_PATH} is missing: build it with "
-            "`python -m sp_region_b200.build` (nvcc, sm_100a)")
+            "`python sp_region_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
     cfgp = ctypes.POINTER(sp_cfg)
@@ -72,6 +73,7 @@ def _load() -> ctypes.CDLL:
     lib.sp_status_string.restype = ctypes.c_char_p
     lib.sp_device_error.argtypes = [i32, ctypes.POINTER(i32), i32]
     lib.sp_debug_wait_timeout.argtypes = [i64, vp, vp]
+    lib.sp_plan_count.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(i32)]
     for f in EXPORTS:
         getattr(lib, f).restype = (ctypes.c_char_p if f == "sp_status_string"
                                    else ctypes.c_int)
@@ -92,12 +94,14 @@ def _check(fn: str, status: int) -> None:
 
 def make_cfg(s: int, b: int, h: int, t: int, dtype="bf16",
              norm="layernorm", eps: float = 1e-5, p_drop: float = 0.0,
-             seed: int = 0, offset: int = 0) -> sp_cfg:
+             seed: int = 0, offset: int = 0, fwd_plan: int = 0,
+             bwd_plan: int = 0) -> sp_cfg:
     dt = {"f32": SP_F32, "bf16": SP_BF16, torch.float32: SP_F32,
           torch.bfloat16: SP_BF16}[dtype]
     nm = {"layernorm": SP_LAYERNORM, "rmsnorm": SP_RMSNORM}[norm]
     return sp_cfg(s=s, b=b, h=h, t=t, dtype=dt, norm=nm, eps=eps,
-                  p_drop=p_drop, seed=seed, offset=offset)
+                  p_drop=p_drop, seed=seed, offset=offset, fwd_plan=fwd_plan,
+                  bwd_plan=bwd_plan)
 
 
 def _p(x: Optional[torch.Tensor]) -> Optional[int]:
@@ -191,3 +195,11 @@ def sp_debug_wait_timeout(limit_ns: int, status: torch.Tensor,
 
 def sp_status_string(status: int) -> str:
     return _status_string(status)
+
+
+def sp_plan_count():
+    """(forward plans, backward plans): valid hint values are 1..count."""
+    f, b = ctypes.c_int32(0), ctypes.c_int32(0)
+    _check("sp_plan_count", _lib.sp_plan_count(ctypes.byref(f),
+                                                ctypes.byref(b)))
+    return int(f.value), int(b.value)

@@ -1,6 +1,8 @@
 """Build step of the SP boundary library: nvcc -> libsp_region.so (in-tree).
 
-Run ``python -m sp_region_b200.build`` (``__graft_entry__.build()`` calls it).
+Run ``python sp_region_b200/build.py`` (``__graft_entry__.build()`` loads this
+file by path).  It is run as a file, not as ``sp_region_b200.build``, because
+importing the package loads the library that this script builds.
 The library is compiled for sm_100a only and links the CUDA runtime
 statically, so it loads next to any PyTorch build.
 """

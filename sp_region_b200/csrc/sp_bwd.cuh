@@ -16,7 +16,10 @@
 // vectors.  The x stage is held while the row is processed (it is read twice)
 // so the row never sits in registers.  ACC_SMEM keeps the per-CTA parameter
 // gradient partials in shared memory when 3 * 8V fp32 registers per thread
-// would not fit.
+// would not fit.  With several consumer groups sharing that one set, the
+// groups take turns in the CTA's row order (two turn barriers, one for each
+// accumulating pass), so the sums keep a fixed order and stay bitwise
+// deterministic while the groups' reduce-scatter phases overlap.
 #pragma once
 
 #include "sp_device.cuh"
@@ -52,81 +55,44 @@ struct BwdArgs {
     int want_dbias;
 };
 
-template <typename T, int V, bool LN, bool ACC_SMEM>
-__global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
-    k_bwd_tma(const __grid_constant__ BwdArgs a)
+template <typename T, int V, int G, int MAXT, bool LN, bool ACC_SMEM>
+__global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ BwdArgs a)
 {
     using Vec = typename IO<T>::Vec;
     extern __shared__ __align__(128) unsigned char smem[];
     RingTail* tail = reinterpret_cast<RingTail*>(smem + a.tail_off);
-    // gamma copy (thread-private slots) and, for ACC_SMEM, the per-CTA
-    // accumulators [3][2][hv][4] fp32, also thread-private
+    // gamma copy and, for ACC_SMEM, the per-CTA accumulators [3][2][hv][4]
+    // fp32; every slot is private to the thread that owns its vector
     unsigned char* sgam = smem + a.param_off;
     float4* accs = reinterpret_cast<float4*>(smem + a.acc_off);
     volatile int* abort = &tail->abort;
 
-    const int C = blockDim.x - 32;
+    const int C = (blockDim.x - 32) / G;
     const int tid = threadIdx.x;
     const int S = a.stages;
-    const int nsrc = a.t + 1 + (a.drnext ? 1 : 0);
+    const int nsrc = a.t + 1 + (a.drnext ? 1 : 0);   // dP_k..., x, [dR_next]
 
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&tail->full[s]), 1);
-            mbar_init(smem_addr(&tail->empty[s]), C / 32);
-        }
-        tail->abort = 0;
-        mbar_init_fence();
-    }
-    __syncthreads();
+    init_ring(tail, S, C / 32);
 
-    // ------------------------------------------------------------------ producer
-    if (tid >= C) {
-        if (tid != C) return;
-        const uint64_t pol = policy_evict_first();
-        uint32_t stage = 0, phase = 1;
-        long long issued = 0;
-        bool ok = true;
-        for (long long n = blockIdx.x; n < a.rows && ok; n += gridDim.x) {
-            for (int k = 0; k < nsrc; ++k) {
-                if (!mbar_wait(smem_addr(&tail->empty[stage]), phase, abort, ERR_WAIT_EMPTY)) {
-                    ok = false;
-                    break;
-                }
-                const void* base = k < a.t ? a.dparts[k] : (k == a.t ? a.x : a.drnext);
-                const unsigned char* src =
-                    static_cast<const unsigned char*>(base) + (size_t)n * a.seg_bytes;
-                const uint32_t bar = smem_addr(&tail->full[stage]);
-                mbar_arrive_expect_tx(bar, a.seg_bytes);
-                bulk_load(smem_addr(smem + (size_t)stage * a.stage_stride), src, a.seg_bytes,
-                          bar, pol);
-                ++issued;
-                if (++stage == (uint32_t)S) {
-                    stage = 0;
-                    phase ^= 1;
-                }
-            }
-        }
-        if (!ok) {
-            long long first = issued > S ? issued - S : 0;
-            for (long long i = first; i < issued; ++i) {
-                const uint32_t s = (uint32_t)(i % S);
-                const uint32_t par = (uint32_t)((i / S) & 1);
-                volatile int no_abort = 0;
-                if (!mbar_wait(smem_addr(&tail->full[s]), par, &no_abort, ERR_DRAIN)) break;
-            }
-        }
+    if (tid >= G * C) {
+        if (tid == G * C)
+            ring_produce<G>(smem, tail, abort, a.rows, nsrc, a.seg_bytes, a.stage_stride, S,
+                         [&](int k) {
+                             return k < a.t ? a.dparts[k] : (k == a.t ? a.x : a.drnext);
+                         });
         return;
     }
 
-    // ------------------------------------------------------------------ consumers
+    const int g = tid / C;
+    const int c = tid - g * C;
     const int lane = tid & 31;
+    const int bar_id = 1 + g;
     const int hv = a.hv;
     float ag[ACC_SMEM ? 1 : V][8], ab[ACC_SMEM ? 1 : V][8], ac[ACC_SMEM ? 1 : V][8];
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-        const int v = tid + i * C;
-        if (v < hv) store_vec<T>(sgam, v, load_vec<T>(a.gamma, v));
+        const int v = c + i * C;
+        if (g == 0 && v < hv) store_vec<T>(sgam, v, load_vec<T>(a.gamma, v));
         if (!ACC_SMEM) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) ag[i][e] = ab[i][e] = ac[i][e] = 0.f;
@@ -138,7 +104,8 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
             }
         }
     }
-    // thread-private read-modify-write of the shared accumulators
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
+
     auto acc_add = [&](int q, int v, const float d[8]) {
         float4* p0 = &accs[((size_t)q * 2 + 0) * hv + v];
         float4* p1 = &accs[((size_t)q * 2 + 1) * hv + v];
@@ -148,38 +115,49 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
         *p0 = x0;
         *p1 = x1;
     };
-
-    uint32_t stage = 0, phase = 0;
-    auto advance = [&]() {
-        if (++stage == (uint32_t)S) {
-            stage = 0;
-            phase ^= 1;
+    auto release_at = [&](uint32_t s_) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&tail->empty[s_]));
+    };
+    // turn q of CTA row j: phase j of turn[q] completes when row j's group has
+    // finished that pass; row j waits for phase j-1 (only one phase can be
+    // outstanding, since row j-2 is this group's own previous row)
+    constexpr bool kTurns = ACC_SMEM && (G > 1);
+    auto take_turn = [&](int q, long long j) {
+        if (kTurns && j > 0)
+            mbar_wait(smem_addr(&tail->turn[q]), (uint32_t)((j - 1) & 1), abort, ERR_WAIT_FULL);
+    };
+    auto pass_turn = [&](int q) {
+        if (kTurns) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->turn[q]));
         }
     };
-    auto release_at = [&](uint32_t s) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&tail->empty[s]));
-    };
 
-    for (long long n = blockIdx.x; n < a.rows; n += gridDim.x) {
+    const uint32_t Sg = (uint32_t)(S / G);
+    RingPos pos((uint32_t)g * Sg, 0, Sg);
+    int parity = 0;
+    for (long long j = g;; j += G, parity ^= 1) {
+        const long long n = blockIdx.x + j * (long long)gridDim.x;
+        if (n >= a.rows) break;
         // loads whose latency overlaps the reduction below
         const float rstd = a.rstd[n];
         const float mean = LN ? a.mean[n] : 0.f;
         uint32_t kb[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int v = tid + i * C;
+            const int v = c + i * C;
             kb[i] = (a.mask && v < hv) ? a.mask[(size_t)n * a.mask_row_bytes + v] : 0xFFu;
         }
 
         // reduce-scatter of the upstream gradient partials
         float dn[V][8];
         for (int k = 0; k < a.t; ++k) {
-            mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
-            const unsigned char* buf = smem + (size_t)stage * a.stage_stride;
+            mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
+            const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int v = tid + i * C;
+                const int v = c + i * C;
                 if (v < hv) {
                     float f[8];
                     IO<T>::unpack(load_vec<T>(buf, v), f);
@@ -187,27 +165,28 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                     for (int e = 0; e < 8; ++e) dn[i][e] = (k == 0) ? f[e] : dn[i][e] + f[e];
                 }
             }
-            release_at(stage);
-            advance();
+            release_at(pos.abs());
+            pos.next(Sg);
         }
 
         // pass 1 over x: row sums of g and g*xhat; parameter-gradient partials
-        mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
-        const uint32_t sx = stage;
+        mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
+        const uint32_t sx = pos.abs();
         const unsigned char* xb = smem + (size_t)sx * a.stage_stride;
-        advance();
+        pos.next(Sg);
+        take_turn(0, j);
         float sg = 0.f, sgx = 0.f;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int v = tid + i * C;
+            const int v = c + i * C;
             if (v < hv) {
-                float xv[8], g[8], dgm[8];
+                float xv[8], gm[8], dgm[8];
                 IO<T>::unpack(load_vec<T>(xb, v), xv);
-                IO<T>::unpack(load_vec<T>(sgam, v), g);
+                IO<T>::unpack(load_vec<T>(sgam, v), gm);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float xh = LN ? (xv[e] - mean) * rstd : xv[e] * rstd;
-                    const float gg = dn[i][e] * g[e];
+                    const float gg = dn[i][e] * gm[e];
                     sg += gg;
                     sgx += gg * xh;
                     dgm[e] = dn[i][e] * xh;
@@ -224,30 +203,40 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                 }
             }
         }
-        const float2 tot = consumer_sum2(make_float2(sg, sgx),
-                                         reinterpret_cast<float2*>(tail->red0), C);
+        pass_turn(0);
+        float2 tot = make_float2(warp_sum(sg), warp_sum(sgx));
+        {
+            float2* red = reinterpret_cast<float2*>(tail->red[parity][g]);
+            if (lane == 0) red[c >> 5] = tot;
+            asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
+            tot = make_float2(0.f, 0.f);
+            for (int w = 0; w < (C >> 5); ++w) {
+                tot.x += red[w].x;
+                tot.y += red[w].y;
+            }
+        }
         const float mg = tot.x / a.h_f, mgx = tot.y / a.h_f;
 
         const unsigned char* rb = nullptr;
         uint32_t sr = 0;
         if (a.drnext) {
-            mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
-            sr = stage;
+            mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
+            sr = pos.abs();
             rb = smem + (size_t)sr * a.stage_stride;
-            advance();
+            pos.next(Sg);
         }
 
         // pass 2: input gradient, residual gradient, dropout backward
+        take_turn(1, j);
         unsigned char* dres = static_cast<unsigned char*>(a.dres) + (size_t)n * a.seg_bytes;
         unsigned char* dy = static_cast<unsigned char*>(a.dY) + (size_t)n * a.seg_bytes;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int v = tid + i * C;
+            const int v = c + i * C;
             if (v < hv) {
-                float xv[8], g[8], dr[8], dz[8];
+                float xv[8], gm[8], dr[8], dz[8], rn[8];
                 IO<T>::unpack(load_vec<T>(xb, v), xv);
-                IO<T>::unpack(load_vec<T>(sgam, v), g);
-                float rn[8];
+                IO<T>::unpack(load_vec<T>(sgam, v), gm);
                 if (rb) {
                     IO<T>::unpack(load_vec<T>(rb, v), rn);
                 } else {
@@ -257,7 +246,7 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float xh = LN ? (xv[e] - mean) * rstd : xv[e] * rstd;
-                    const float gg = dn[i][e] * g[e];
+                    const float gg = dn[i][e] * gm[e];
                     const float dx = LN ? rstd * (gg - mg - xh * mgx) : rstd * (gg - xh * mgx);
                     dr[e] = dx + rn[e];
                     dz[e] = ((kb[i] >> e) & 1u) ? dr[e] * a.scale : 0.f;
@@ -274,15 +263,22 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                 }
             }
         }
+        pass_turn(1);
         release_at(sx);
         if (rb) release_at(sr);
     }
 
-    // this CTA's partial sums -> workspace [cta][q][h]
-    float* ws = a.ws + (size_t)blockIdx.x * 3 * a.h;
+    // partial sums -> workspace: register accumulators give one slice per
+    // group ([cta * G + g][q][h]); the shared set gives one slice per CTA
+    // ([cta][q][h]), written by group 0 once every group has finished
+    if (ACC_SMEM) {
+        if (G > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
+        if (g != 0) return;
+    }
+    float* ws = a.ws + (ACC_SMEM ? (size_t)blockIdx.x : (size_t)blockIdx.x * G + g) * 3 * a.h;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-        const int v = tid + i * C;
+        const int v = c + i * C;
         if (v < hv) {
             for (int q = 0; q < 3; ++q) {
                 float4 lo, hi;
@@ -290,11 +286,11 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                     lo = accs[((size_t)q * 2 + 0) * hv + v];
                     hi = accs[((size_t)q * 2 + 1) * hv + v];
                 } else {
-                    const float* s = q == 0 ? ag[ACC_SMEM ? 0 : i]
-                                            : (q == 1 ? ab[ACC_SMEM ? 0 : i]
-                                                      : ac[ACC_SMEM ? 0 : i]);
-                    lo = make_float4(s[0], s[1], s[2], s[3]);
-                    hi = make_float4(s[4], s[5], s[6], s[7]);
+                    const float* s_ = q == 0 ? ag[ACC_SMEM ? 0 : i]
+                                             : (q == 1 ? ab[ACC_SMEM ? 0 : i]
+                                                       : ac[ACC_SMEM ? 0 : i]);
+                    lo = make_float4(s_[0], s_[1], s_[2], s_[3]);
+                    hi = make_float4(s_[4], s_[5], s_[6], s_[7]);
                 }
                 float4* dst = reinterpret_cast<float4*>(ws + (size_t)q * a.h + 8 * (size_t)v);
                 dst[0] = lo;
@@ -355,29 +351,43 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
     }
 }
 
-// dgamma / dbeta / dbias: fixed-order sum of the per-CTA partials.
+// dgamma / dbeta / dbias: fixed-order sum of the per-CTA (per-group)
+// partials.  A block covers 32 consecutive columns of one quantity: lane =
+// column, warp w sums partials w, w+8, w+16, ... in order, then warp 0 adds
+// the 8 warp totals in order.  Deterministic for a given partial count.
 __global__ void __launch_bounds__(256)
     k_colreduce(const float* __restrict__ ws, int nparts, int h, float* dgamma, float* dbeta,
                 float* dbias)
 {
-    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= 3LL * h) return;
-    const int q = (int)(idx / h), j = (int)(idx % h);
+    __shared__ float part[8][33];
+    const int tiles = (h + 31) / 32;
+    const int q = blockIdx.x / tiles;
+    const int j = (blockIdx.x - q * tiles) * 32 + (threadIdx.x & 31);
+    const int w = threadIdx.x >> 5;
     float* out = q == 0 ? dgamma : (q == 1 ? dbeta : dbias);
-    if (!out) return;
-    const float* p = ws + (size_t)q * h + j;
-    const size_t stride = (size_t)3 * h;
+    if (!out) return;   // uniform over the block
     float s = 0.f;
-    int g = 0;
-    for (; g + 8 <= nparts; g += 8) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = p[(size_t)(g + u) * stride];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) s += v[u];
+    if (j < h) {
+        const float* p = ws + (size_t)q * h + j;
+        const size_t stride = (size_t)3 * h;
+        int k = w;
+        for (; k + 24 < nparts; k += 32) {
+            const float v0 = p[(size_t)k * stride], v1 = p[(size_t)(k + 8) * stride];
+            const float v2 = p[(size_t)(k + 16) * stride], v3 = p[(size_t)(k + 24) * stride];
+            s += v0;
+            s += v1;
+            s += v2;
+            s += v3;
+        }
+        for (; k < nparts; k += 8) s += p[(size_t)k * stride];
     }
-    for (; g < nparts; ++g) s += p[(size_t)g * stride];
-    out[j] = s;
+    part[w][threadIdx.x & 31] = s;
+    __syncthreads();
+    if (w == 0 && j < h) {
+        float t = 0.f;
+        for (int i = 0; i < 8; ++i) t += part[i][threadIdx.x];
+        out[j] = t;
+    }
 }
 
 }  // namespace spk

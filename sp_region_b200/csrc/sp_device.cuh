@@ -126,13 +126,6 @@ __device__ __forceinline__ uint64_t policy_evict_first()
     return p;
 }
 
-// Named barrier over the first `nthreads` threads of the CTA (the consumer
-// warps); the producer warp never takes part.
-__device__ __forceinline__ void consumer_sync(int nthreads)
-{
-    asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
 // Easy as 1, 2, 3", SC'11).  Each round multiplies counter words 0 and 2 by
@@ -296,35 +289,6 @@ __device__ __forceinline__ float warp_sum(float x)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
     return x;
-}
-
-// Sum over the C consumer threads; `red` holds >= C/32 floats and must not be
-// reused by the next call before every consumer has passed this one's barrier
-// (callers alternate two buffers).
-__device__ __forceinline__ float consumer_sum(float x, float* red, int C)
-{
-    x = warp_sum(x);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane == 0) red[warp] = x;
-    consumer_sync(C);
-    float s = 0.f;
-    for (int w = 0; w < (C >> 5); ++w) s += red[w];
-    return s;
-}
-
-__device__ __forceinline__ float2 consumer_sum2(float2 x, float2* red, int C)
-{
-    x.x = warp_sum(x.x);
-    x.y = warp_sum(x.y);
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (lane == 0) red[warp] = x;
-    consumer_sync(C);
-    float2 s = make_float2(0.f, 0.f);
-    for (int w = 0; w < (C >> 5); ++w) {
-        s.x += red[w].x;
-        s.y += red[w].y;
-    }
-    return s;
 }
 
 // Block-wide sum for the general kernels (all threads take part).

@@ -57,120 +57,196 @@ struct FwdArgs {
     int dropout;            // p > 0
 };
 
-// Shared-memory tail after the ring: barriers, reduction scratch, abort flag.
+// Shared-memory tail after the ring: barriers, per-group reduction scratch,
+// abort flag.
+constexpr int kMaxGroups = 4;
+// Reduction scratch: two buffers per group, used alternately by row parity
+// (or by the two reductions of one LayerNorm row), so a warp that runs ahead
+// to the next row never overwrites totals a slower warp is still reading.
 struct RingTail {
     uint64_t full[64];
     uint64_t empty[64];
-    float red0[32];
-    float red1[32];
+    uint64_t turn[2];   // backward: shared-accumulator turns, in row order
+    float red[2][kMaxGroups][64];
     int abort;
 };
 
-template <typename T, int V, bool LN>
-__global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
-    k_fwd_tma(const __grid_constant__ FwdArgs a)
+// Position in a sub-ring of Sg stages starting at stage `base`: the i-th
+// segment a consumer group receives lives in stage base + i % Sg and completes
+// phase i / Sg of that stage's barriers.  Each group consumes its own sub-ring
+// strictly in order, so a group never waits on a stage more than one phase
+// ahead of it (mbarrier parity waits only tell adjacent phases apart).
+struct RingPos {
+    uint32_t base, stage, phase;
+    __device__ __forceinline__ RingPos(uint32_t base_, uint32_t i, uint32_t Sg)
+        : base(base_), stage(i % Sg), phase((i / Sg) & 1u) {}
+    __device__ __forceinline__ uint32_t abs() const { return base + stage; }
+    __device__ __forceinline__ void next(uint32_t Sg)
+    {
+        if (++stage == Sg) {
+            stage = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
+// The producer lane: streams every segment of this CTA's rows, in row order.
+// Row j of the CTA belongs to consumer group j % G and goes to that group's
+// sub-ring (stages [g*Sg, (g+1)*Sg)).  nsrc sources per row; src(k) gives
+// source k's base pointer.
+template <int G, typename SrcFn>
+__device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail,
+                                             volatile int* abort, long long rows,
+                                             int nsrc, uint32_t seg_bytes,
+                                             uint32_t stage_stride, int S, SrcFn src)
+{
+    const uint64_t pol = policy_evict_first();
+    const int Sg = S / G;
+    uint32_t stage[G], phase[G];
+    long long issued[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        stage[g] = 0;
+        phase[g] = 1;   // a fresh "empty" barrier counts as released
+        issued[g] = 0;
+    }
+    bool ok = true;
+    for (long long jj = 0; ok; ++jj) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const long long n = blockIdx.x + (jj * G + g) * (long long)gridDim.x;
+            if (!ok || n >= rows) {
+                ok = false;
+                break;
+            }
+            for (int k = 0; k < nsrc; ++k) {
+                const uint32_t st = (uint32_t)(g * Sg) + stage[g];
+                if (!mbar_wait(smem_addr(&tail->empty[st]), phase[g], abort, ERR_WAIT_EMPTY)) {
+                    ok = false;
+                    break;
+                }
+                const unsigned char* p = static_cast<const unsigned char*>(src(k)) +
+                                         (size_t)n * seg_bytes;
+                const uint32_t bar = smem_addr(&tail->full[st]);
+                mbar_arrive_expect_tx(bar, seg_bytes);
+                bulk_load(smem_addr(smem + (size_t)st * stage_stride), p, seg_bytes, bar, pol);
+                ++issued[g];
+                if (++stage[g] == (uint32_t)Sg) {
+                    stage[g] = 0;
+                    phase[g] ^= 1;
+                }
+            }
+        }
+    }
+    if (*abort) {
+        // wind down: let every copy already issued land before the CTA exits
+        // (its shared memory must not be released under a copy)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const long long first = issued[g] > Sg ? issued[g] - Sg : 0;
+            for (long long i = first; i < issued[g]; ++i) {
+                volatile int no_abort = 0;
+                if (!mbar_wait(smem_addr(&tail->full[g * Sg + i % Sg]), (uint32_t)((i / Sg) & 1),
+                               &no_abort, ERR_DRAIN))
+                    break;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void init_ring(RingTail* tail, int S, int warps_per_group)
+{
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_addr(&tail->full[s]), 1);
+            mbar_init(smem_addr(&tail->empty[s]), warps_per_group);
+        }
+        mbar_init(smem_addr(&tail->turn[0]), warps_per_group);
+        mbar_init(smem_addr(&tail->turn[1]), warps_per_group);
+        tail->abort = 0;
+        mbar_init_fence();
+    }
+    __syncthreads();
+}
+
+// Fast-kernel instantiations are k_*_tma<T, V, G, MAXT, ...>: G consumer
+// groups of C threads (C <= (MAXT - 32) / G), each thread owning V vectors of
+// 8 features of a row, plus one producer warp; MAXT bounds the block size and
+// so sets the register budget.
+template <typename T, int V, int G, int MAXT, bool LN>
+__global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ FwdArgs a)
 {
     using Vec = typename IO<T>::Vec;
     extern __shared__ __align__(128) unsigned char smem[];
     RingTail* tail = reinterpret_cast<RingTail*>(smem + a.tail_off);
     volatile int* abort = &tail->abort;
-    // gamma, beta, bias copies: each consumer thread stores and later reads
-    // only its own vectors, so no barrier orders them
-    unsigned char* sg = smem + a.param_off;
+    unsigned char* sg = smem + a.param_off;   // gamma, beta, bias copies
     unsigned char* sb = sg + a.param_stride;
     unsigned char* sc = sb + a.param_stride;
 
-    const int C = blockDim.x - 32;   // consumer threads
+    const int C = (blockDim.x - 32) / G;      // consumer threads per group
     const int tid = threadIdx.x;
-    const int S = a.stages;
+    const int S = a.stages;                   // G sub-rings of S / G stages
+    const int nsrc = a.t + 1;                 // t partials, then the residual
 
-    if (tid == 0) {
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&tail->full[s]), 1);
-            mbar_init(smem_addr(&tail->empty[s]), C / 32);
-        }
-        tail->abort = 0;
-        mbar_init_fence();
-    }
-    __syncthreads();
+    init_ring(tail, S, C / 32);
 
-    const int nsrc = a.t + 1;   // t partials, then the residual row
-
-    // ------------------------------------------------------------------ producer
-    if (tid >= C) {
-        if (tid != C) return;
-        const uint64_t pol = policy_evict_first();
-        uint32_t stage = 0, phase = 1;   // a fresh "empty" barrier counts as released
-        long long issued = 0;
-        bool ok = true;
-        for (long long n = blockIdx.x; n < a.rows && ok; n += gridDim.x) {
-            for (int k = 0; k < nsrc; ++k) {
-                if (!mbar_wait(smem_addr(&tail->empty[stage]), phase, abort, ERR_WAIT_EMPTY)) {
-                    ok = false;
-                    break;
-                }
-                const unsigned char* src =
-                    static_cast<const unsigned char*>(k < a.t ? a.parts[k] : a.residual) +
-                    (size_t)n * a.seg_bytes;
-                const uint32_t bar = smem_addr(&tail->full[stage]);
-                mbar_arrive_expect_tx(bar, a.seg_bytes);
-                bulk_load(smem_addr(smem + (size_t)stage * a.stage_stride), src, a.seg_bytes,
-                          bar, pol);
-                ++issued;
-                if (++stage == (uint32_t)S) {
-                    stage = 0;
-                    phase ^= 1;
-                }
-            }
-        }
-        if (!ok) {
-            // wind down: let every copy already issued land before the CTA
-            // exits (its shared memory must not be released under a copy)
-            long long first = issued > S ? issued - S : 0;
-            for (long long i = first; i < issued; ++i) {
-                const uint32_t s = (uint32_t)(i % S);
-                const uint32_t par = (uint32_t)((i / S) & 1);
-                volatile int no_abort = 0;
-                if (!mbar_wait(smem_addr(&tail->full[s]), par, &no_abort, ERR_DRAIN)) break;
-            }
-        }
+    if (tid >= G * C) {
+        if (tid == G * C)
+            ring_produce<G>(smem, tail, abort, a.rows, nsrc, a.seg_bytes, a.stage_stride, S,
+                            [&](int k) { return k < a.t ? a.parts[k] : a.residual; });
         return;
     }
 
-    // ------------------------------------------------------------------ consumers
+    // consumers: group g handles every G-th row of this CTA; thread c of a
+    // group owns vectors v = c + i*C (8 features each)
+    const int g = tid / C;
+    const int c = tid - g * C;
     const int lane = tid & 31;
+    const int bar_id = 1 + g;
+    if (g == 0) {
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-        const int v = tid + i * C;
-        if (v < a.hv) {
-            store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
-            if (a.beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));
-            if (a.bias) store_vec<T>(sc, v, load_vec<T>(a.bias, v));
+        for (int i = 0; i < V; ++i) {
+            const int v = c + i * C;
+            if (v < a.hv) {
+                store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
+                if (a.beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));
+                if (a.bias) store_vec<T>(sc, v, load_vec<T>(a.bias, v));
+            }
         }
     }
+    // every group reads the copies group 0 wrote
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
 
-    uint32_t stage = 0, phase = 0;
-    auto advance = [&]() {
-        if (++stage == (uint32_t)S) {
-            stage = 0;
-            phase ^= 1;
-        }
+    auto group_sum = [&](float x, float* red) {
+        x = warp_sum(x);
+        if (lane == 0) red[c >> 5] = x;
+        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
+        float s_ = 0.f;
+        for (int w = 0; w < (C >> 5); ++w) s_ += red[w];
+        return s_;
     };
+
+    const uint32_t Sg = (uint32_t)(S / G);
+    RingPos pos((uint32_t)g * Sg, 0, Sg);
     auto release = [&]() {
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&tail->empty[stage]));
-        advance();
+        if (lane == 0) mbar_arrive(smem_addr(&tail->empty[pos.abs()]));
+        pos.next(Sg);
     };
+    int parity = 0;
+    for (long long j = g;; j += G, parity ^= 1) {
+        const long long n = blockIdx.x + j * (long long)gridDim.x;
+        if (n >= a.rows) break;
 
-    for (long long n = blockIdx.x; n < a.rows; n += gridDim.x) {
         float acc[V][8];
         // reduce-scatter: sum of the t partial rows, k ascending
         for (int k = 0; k < a.t; ++k) {
-            mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
-            const unsigned char* buf = smem + (size_t)stage * a.stage_stride;
+            mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
+            const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int v = tid + i * C;
+                const int v = c + i * C;
                 if (v < a.hv) {
                     float f[8];
                     IO<T>::unpack(load_vec<T>(buf, v), f);
@@ -185,7 +261,7 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
         uint8_t* mrow = a.mask ? a.mask + (size_t)n * a.mask_row_bytes : nullptr;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int v = tid + i * C;
+            const int v = c + i * C;
             if (v < a.hv) {
                 if (a.bias) {
                     float f[8];
@@ -204,19 +280,19 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                 if (mrow) mrow[v] = (uint8_t)kb;
             }
         }
-        if (mrow && tid == 0)
+        if (mrow && c == 0)
             for (int pbyte = a.hv; pbyte < a.mask_row_bytes; ++pbyte) mrow[pbyte] = 0;
 
         // residual add; the sum is stored in the I/O dtype and the norm reads
         // the stored (rounded) value
-        mbar_wait(smem_addr(&tail->full[stage]), phase, abort, ERR_WAIT_FULL);
+        mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
         {
-            const unsigned char* buf = smem + (size_t)stage * a.stage_stride;
-            unsigned char* rout = static_cast<unsigned char*>(a.residual_out) +
-                                  (size_t)n * a.seg_bytes;
+            const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
+            unsigned char* rout =
+                static_cast<unsigned char*>(a.residual_out) + (size_t)n * a.seg_bytes;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                const int v = tid + i * C;
+                const int v = c + i * C;
                 if (v < a.hv) {
                     float f[8];
                     IO<T>::unpack(load_vec<T>(buf, v), f);
@@ -233,41 +309,41 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
         // per-token norm, two passes over the row held in registers
         float mean = 0.f, rstd;
         if (LN) {
-            float s = 0.f;
+            float s_ = 0.f;
 #pragma unroll
             for (int i = 0; i < V; ++i)
-                if (tid + i * C < a.hv)
+                if (c + i * C < a.hv)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) s += acc[i][e];
-            mean = consumer_sum(s, tail->red0, C) / a.h_f;
+                    for (int e = 0; e < 8; ++e) s_ += acc[i][e];
+            mean = group_sum(s_, tail->red[0][g]) / a.h_f;
             float q = 0.f;
 #pragma unroll
             for (int i = 0; i < V; ++i)
-                if (tid + i * C < a.hv)
+                if (c + i * C < a.hv)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const float d = acc[i][e] - mean;
                         q += d * d;
                     }
-            const float var = consumer_sum(q, tail->red1, C) / a.h_f;
+            const float var = group_sum(q, tail->red[1][g]) / a.h_f;
             rstd = 1.0f / sqrtf(var + a.eps);
         } else {
             float q = 0.f;
 #pragma unroll
             for (int i = 0; i < V; ++i)
-                if (tid + i * C < a.hv)
+                if (c + i * C < a.hv)
 #pragma unroll
                     for (int e = 0; e < 8; ++e) q += acc[i][e] * acc[i][e];
-            const float ms = consumer_sum(q, tail->red0, C) / a.h_f;
+            const float ms = group_sum(q, tail->red[parity][g]) / a.h_f;
             rstd = 1.0f / sqrtf(ms + a.eps);
         }
 
 #pragma unroll
         for (int i = 0; i < V; ++i) {
-            const int v = tid + i * C;
+            const int v = c + i * C;
             if (v < a.hv) {
-                float g[8], b[8], o[8];
-                IO<T>::unpack(load_vec<T>(sg, v), g);
+                float gm[8], b[8], o[8];
+                IO<T>::unpack(load_vec<T>(sg, v), gm);
                 if (LN && a.beta) {
                     IO<T>::unpack(load_vec<T>(sb, v), b);
                 } else {
@@ -276,8 +352,8 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    o[e] = LN ? (acc[i][e] - mean) * rstd * g[e] + b[e]
-                              : acc[i][e] * rstd * g[e];
+                    o[e] = LN ? (acc[i][e] - mean) * rstd * gm[e] + b[e]
+                              : acc[i][e] * rstd * gm[e];
                 const Vec ov = IO<T>::pack(o);
                 for (int q = 0; q < a.n_gathered; ++q)
                     store_vec<T>(static_cast<unsigned char*>(a.gathered[q]) +
@@ -285,7 +361,7 @@ __global__ void __launch_bounds__(kFwdMaxConsumers + 32, 1)
                                  v, ov);
             }
         }
-        if (tid == 0) {
+        if (c == 0) {
             if (LN && a.mean) a.mean[n] = mean;
             if (a.rstd) a.rstd[n] = rstd;
         }

@@ -16,7 +16,6 @@ using namespace spk;
 namespace {
 
 constexpr int kGeneralThreads = 256;
-constexpr int kMaxV = 4;
 
 struct DevInfo {
     int id;
@@ -68,85 +67,222 @@ int elem_bytes(const sp_cfg* c) { return c->dtype == SP_F32 ? 4 : 2; }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
-uint32_t drop_threshold(float p)
-{
-    return (uint32_t)floor((double)p * 4294967296.0);
-}
-
-int launch_status()
-{
-    return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
-}
-
-// Fast-kernel shape for a row of hv 8-feature vectors: V vectors per
-// consumer thread, C consumer threads (multiple of 32, at most 512).
-bool fast_shape(int hv, int* V, int* C)
-{
-    int v = (hv + kFwdMaxConsumers - 1) / kFwdMaxConsumers;
-    if (v < 1) v = 1;
-    if (v > kMaxV) return false;
-    int c = (hv + v - 1) / v;
-    c = (c + 31) / 32 * 32;
-    *V = v;
-    *C = c;
-    return true;
-}
-
-template <typename T, bool LN>
-int launch_fwd_fast(const FwdArgs& a, int V, int C, int grid, size_t smem, cudaStream_t st)
-{
-    auto pick = [&](auto kern) -> int {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return SP_ERR_CUDA;
-        kern<<<grid, C + 32, smem, st>>>(a);
-        return launch_status();
-    };
-    switch (V) {
-    case 1: return pick(k_fwd_tma<T, 1, LN>);
-    case 2: return pick(k_fwd_tma<T, 2, LN>);
-    case 3: return pick(k_fwd_tma<T, 3, LN>);
-    default: return pick(k_fwd_tma<T, 4, LN>);
-    }
-}
-
-template <typename T, bool LN>
-int launch_bwd_fast(const BwdArgs& a, int V, int C, int grid, size_t smem, cudaStream_t st)
-{
-    auto pick = [&](auto kern) -> int {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return SP_ERR_CUDA;
-        kern<<<grid, C + 32, smem, st>>>(a);
-        return launch_status();
-    };
-    switch (V) {
-    case 1: return pick(k_bwd_tma<T, 1, LN, false>);
-    case 2: return pick(k_bwd_tma<T, 2, LN, true>);
-    case 3: return pick(k_bwd_tma<T, 3, LN, true>);
-    default: return pick(k_bwd_tma<T, 4, LN, true>);
-    }
-}
-
-size_t ring_tail_bytes() { return (sizeof(RingTail) + 127) & ~(size_t)127; }
+uint32_t drop_threshold(float p) { return (uint32_t)floor((double)p * 4294967296.0); }
 
 size_t round128(size_t x) { return (x + 127) & ~(size_t)127; }
 
-// accumulators in shared memory once a thread owns two or more vectors
-bool bwd_acc_in_smem(int V) { return V >= 2; }
+size_t ring_tail_bytes() { return round128(sizeof(RingTail)); }
 
-// Rows a general-kernel launch covers at once (grid), per device.
+// Rows covered at once by a general-kernel launch (its grid).
 long long general_grid(long long rows, int sms)
 {
     const long long g = (long long)sms * 4;
     return rows < g ? rows : g;
 }
 
-long long fast_grid(long long rows, int sms) { return rows < sms ? rows : sms; }
+// ---------------------------------------------------------------------------
+// Fast-kernel plans: V vectors of 8 features per consumer thread, G consumer
+// groups (each takes every G-th row of the CTA), at most maxT threads (which
+// sets the register budget), and for the backward the parameter-gradient
+// partials in registers or shared memory.  A group needs
+// C = 32 * ceil(ceil(hv / V) / 32) threads; a launch has G*C + 32.
+// ---------------------------------------------------------------------------
+struct Plan {
+    int V, G, maxT;
+    bool acc_smem;
+};
+
+constexpr Plan kFwdPlans[] = {
+    {1, 1, 1024, false},   // 0
+    {1, 2, 800, false},    // 1
+    {1, 4, 1024, false},   // 2
+    {2, 1, 544, false},    // 3
+    {2, 2, 800, false},    // 4
+    {3, 1, 544, false},    // 5
+    {3, 2, 800, false},    // 6
+    {4, 1, 544, false},    // 7
+    {4, 2, 800, false},    // 8
+};
+constexpr Plan kBwdPlans[] = {
+    {1, 1, 1024, false},   // 0
+    {1, 1, 800, false},    // 1
+    {1, 2, 800, false},    // 2
+    {2, 1, 544, true},     // 3
+    {2, 1, 800, false},    // 4
+    {3, 1, 544, true},     // 5
+    {4, 1, 544, true},     // 6
+    {2, 1, 544, false},    // 7
+    {2, 2, 800, true},     // 8
+    {3, 2, 800, true},     // 9
+    {4, 2, 800, true},     // 10
+};
+constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
+constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
+
+// Preference order when the caller gives no hint: the first feasible plan
+// wins.  A hinted plan is tried first.
+constexpr int kFwdOrder[] = {4, 1, 2, 6, 8, 0, 3, 5, 7};
+constexpr int kBwdOrder[] = {8, 9, 2, 3, 5, 10, 6, 1, 0, 4, 7};
+
+int group_threads(int hv, int V)
+{
+    const int per = (hv + V - 1) / V;
+    return (per + 31) / 32 * 32;
+}
+
+long long ring_stages(long long smem_optin, long long fixed, uint32_t stage_stride)
+{
+    if (smem_optin <= fixed) return 0;
+    long long S = (smem_optin - fixed) / stage_stride;
+    return S > 64 ? 64 : S;
+}
+
+#define SP_FWD_CASE(ID)                                                                 \
+    case ID:                                                                            \
+        return (const void*)k_fwd_tma<T, kFwdPlans[ID].V, kFwdPlans[ID].G,              \
+                                      kFwdPlans[ID].maxT, LN>;
+
+template <typename T, bool LN>
+const void* fwd_kernel(int id)
+{
+    switch (id) {
+        SP_FWD_CASE(0) SP_FWD_CASE(1) SP_FWD_CASE(2) SP_FWD_CASE(3) SP_FWD_CASE(4)
+        SP_FWD_CASE(5) SP_FWD_CASE(6) SP_FWD_CASE(7) SP_FWD_CASE(8)
+    }
+    return nullptr;
+}
+
+#define SP_BWD_CASE(ID)                                                                 \
+    case ID:                                                                            \
+        return (const void*)k_bwd_tma<T, kBwdPlans[ID].V, kBwdPlans[ID].G,              \
+                                      kBwdPlans[ID].maxT, LN, kBwdPlans[ID].acc_smem>;
+
+template <typename T, bool LN>
+const void* bwd_kernel(int id)
+{
+    switch (id) {
+        SP_BWD_CASE(0) SP_BWD_CASE(1) SP_BWD_CASE(2) SP_BWD_CASE(3) SP_BWD_CASE(4)
+        SP_BWD_CASE(5) SP_BWD_CASE(6) SP_BWD_CASE(7) SP_BWD_CASE(8) SP_BWD_CASE(9)
+        SP_BWD_CASE(10)
+    }
+    return nullptr;
+}
+
+template <bool LN>
+const void* fwd_kernel_dt(int dtype, int id)
+{
+    return dtype == SP_BF16 ? fwd_kernel<__nv_bfloat16, LN>(id) : fwd_kernel<float, LN>(id);
+}
+
+template <bool LN>
+const void* bwd_kernel_dt(int dtype, int id)
+{
+    return dtype == SP_BF16 ? bwd_kernel<__nv_bfloat16, LN>(id) : bwd_kernel<float, LN>(id);
+}
+
+int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream_t st,
+                  void* args)
+{
+    if (!kern) return SP_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    void* params[] = {args};
+    if (cudaLaunchKernel(kern, dim3(grid), dim3(block), params, smem, st) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
+}
+
+// A fast launch: the chosen plan, its block and grid, and its dynamic shared
+// memory (the layout offsets are written into the kernel arguments).
+struct FastLaunch {
+    int plan = -1;
+    int block = 0;
+    int grid = 0;
+    int groups = 1;
+    size_t smem = 0;
+};
+
+FastLaunch plan_fwd(FwdArgs& a, const DevInfo& dev, int E, int hint)
+{
+    FastLaunch L;
+    const size_t tailb = ring_tail_bytes();
+    const size_t pstride = round128((size_t)a.h * E);
+    int order[1 + kNumFwdPlans];
+    int no = 0;
+    if (hint >= 1 && hint <= kNumFwdPlans) order[no++] = hint - 1;
+    for (int id : kFwdOrder) order[no++] = id;
+    for (int oi = 0; oi < no; ++oi) {
+        const int id = order[oi];
+        const Plan& p = kFwdPlans[id];
+        const int C = group_threads(a.hv, p.V);
+        if (p.G * C + 32 > p.maxT) continue;
+        long long S = ring_stages(dev.smem_optin, (long long)(tailb + 3 * pstride),
+                                  a.stage_stride);
+        S -= S % p.G;                 // G sub-rings of S / G stages each
+        if (S < 2 * p.G) continue;
+        a.stages = (int)S;
+        a.param_off = (uint32_t)(S * a.stage_stride);
+        a.param_stride = (uint32_t)pstride;
+        a.tail_off = (uint32_t)(a.param_off + 3 * pstride);
+        L.plan = id;
+        L.block = p.G * C + 32;
+        L.grid = (int)(a.rows < dev.sms ? a.rows : dev.sms);
+        L.groups = p.G;
+        L.smem = (size_t)a.tail_off + tailb;
+        return L;
+    }
+    return L;
+}
+
+FastLaunch plan_bwd(BwdArgs& a, const DevInfo& dev, int E, int hint)
+{
+    FastLaunch L;
+    const size_t tailb = ring_tail_bytes();
+    const size_t pstride = round128((size_t)a.h * E);
+    int order[1 + kNumBwdPlans];
+    int no = 0;
+    if (hint >= 1 && hint <= kNumBwdPlans) order[no++] = hint - 1;
+    for (int id : kBwdOrder) order[no++] = id;
+    for (int oi = 0; oi < no; ++oi) {
+        const int id = order[oi];
+        const Plan& p = kBwdPlans[id];
+        const int C = group_threads(a.hv, p.V);
+        if (p.G * C + 32 > p.maxT) continue;
+        const size_t accb = p.acc_smem ? (size_t)3 * 2 * a.hv * sizeof(float4) : 0;
+        long long S = ring_stages(dev.smem_optin, (long long)(tailb + pstride + accb),
+                                  a.stage_stride);
+        S -= S % p.G;                 // G sub-rings of S / G stages each
+        if (S < 2 * p.G) continue;
+        a.stages = (int)S;
+        a.param_off = (uint32_t)(S * a.stage_stride);
+        a.acc_off = (uint32_t)(a.param_off + pstride);
+        a.tail_off = (uint32_t)(a.acc_off + accb);
+        L.plan = id;
+        L.block = p.G * C + 32;
+        L.grid = (int)(a.rows < dev.sms ? a.rows : dev.sms);
+        L.groups = p.G;
+        L.smem = (size_t)a.tail_off + tailb;
+        return L;
+    }
+    return L;
+}
 
 }  // namespace
 
 extern "C" {
+
+int sp_plan_count(int32_t* fwd_plans, int32_t* bwd_plans)
+{
+    if (!fwd_plans || !bwd_plans) return SP_ERR_INVALID_ARG;
+    *fwd_plans = kNumFwdPlans;
+    *bwd_plans = kNumBwdPlans;
+    return SP_OK;
+}
 
 const char* sp_status_string(int status)
 {
@@ -231,7 +367,7 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
     a.t = cfg->t;
     a.n_gathered = n_gathered;
     a.seg_bytes = (uint32_t)(h * E);
-    a.stage_stride = (a.seg_bytes + 127u) & ~127u;
+    a.stage_stride = (uint32_t)round128(a.seg_bytes);
     a.mask_row_bytes = 4 * ((h + 31) / 32);
     a.eps = cfg->eps;
     a.h_f = (float)h;
@@ -244,41 +380,26 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
     a.dropout = cfg->p_drop > 0.0f ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    int V = 0, C = 0;
-    if (h % 8 == 0 && all16 && fast_shape(h / 8, &V, &C)) {
-        const size_t tailb = ring_tail_bytes();
-        const size_t pstride = round128((size_t)h * E);
-        long long S = ((long long)dev.smem_optin - (long long)(tailb + 3 * pstride)) /
-                      a.stage_stride;
-        if (S > 64) S = 64;
-        if (S >= 2) {
-            a.stages = (int)S;
-            a.param_off = (uint32_t)(S * a.stage_stride);
-            a.param_stride = (uint32_t)pstride;
-            a.tail_off = (uint32_t)(a.param_off + 3 * pstride);
-            const size_t smem = (size_t)a.tail_off + tailb;
-            const int grid = (int)fast_grid(rows, dev.sms);
-            if (cfg->dtype == SP_BF16)
-                return ln ? launch_fwd_fast<__nv_bfloat16, true>(a, V, C, grid, smem, st)
-                          : launch_fwd_fast<__nv_bfloat16, false>(a, V, C, grid, smem, st);
-            return ln ? launch_fwd_fast<float, true>(a, V, C, grid, smem, st)
-                      : launch_fwd_fast<float, false>(a, V, C, grid, smem, st);
+    if (h % 8 == 0 && all16) {
+        const FastLaunch L = plan_fwd(a, dev, E, cfg->fwd_plan);
+        if (L.plan >= 0) {
+            const void* kern = ln ? fwd_kernel_dt<true>(cfg->dtype, L.plan)
+                                  : fwd_kernel_dt<false>(cfg->dtype, L.plan);
+            return launch_kernel(kern, L.grid, L.block, L.smem, st, &a);
         }
     }
-    // general kernel
+    // general kernel: any h, element-aligned pointers
     const size_t smem = (size_t)h * 4 + (size_t)a.mask_row_bytes;
     if (smem > (size_t)dev.smem_optin - 1024) return SP_ERR_UNSUPPORTED;
     const int grid = (int)general_grid(rows, dev.sms);
-    auto go = [&](auto kern) -> int {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess)
-            return SP_ERR_CUDA;
-        kern<<<grid, kGeneralThreads, smem, st>>>(a);
-        return launch_status();
-    };
+    const void* kern;
     if (cfg->dtype == SP_BF16)
-        return ln ? go(k_fwd_general<__nv_bfloat16, true>) : go(k_fwd_general<__nv_bfloat16, false>);
-    return ln ? go(k_fwd_general<float, true>) : go(k_fwd_general<float, false>);
+        kern = ln ? (const void*)k_fwd_general<__nv_bfloat16, true>
+                  : (const void*)k_fwd_general<__nv_bfloat16, false>;
+    else
+        kern = ln ? (const void*)k_fwd_general<float, true>
+                  : (const void*)k_fwd_general<float, false>;
+    return launch_kernel(kern, grid, kGeneralThreads, smem, st, &a);
 }
 
 int sp_all_gather(const sp_cfg* cfg, const void* const* shards, void* const* outs,
@@ -315,14 +436,10 @@ int sp_all_gather(const sp_cfg* cfg, const void* const* shards, void* const* out
     const long long cap = (long long)dev.sms * 4;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (vec)
-        k_all_gather<uint4><<<(int)grid, 512, 0, st>>>(a);
-    else if (E == 4)
-        k_all_gather<uint32_t><<<(int)grid, 512, 0, st>>>(a);
-    else
-        k_all_gather<uint16_t><<<(int)grid, 512, 0, st>>>(a);
-    return launch_status();
+    const void* kern = vec ? (const void*)k_all_gather<uint4>
+                           : (E == 4 ? (const void*)k_all_gather<uint32_t>
+                                     : (const void*)k_all_gather<uint16_t>);
+    return launch_kernel(kern, (int)grid, 512, 0, static_cast<cudaStream_t>(stream), &a);
 }
 
 int sp_bwd_workspace_bytes(const sp_cfg* cfg, int32_t device, size_t* bytes)
@@ -335,9 +452,13 @@ int sp_bwd_workspace_bytes(const sp_cfg* cfg, int32_t device, size_t* bytes)
         cudaGetLastError();
         return SP_ERR_CUDA;
     }
+    // partial sums of dgamma, dbeta, dbias, one slice per CTA (fast kernels:
+    // per consumer group, at most SMs x 4 groups; general kernel: its grid of
+    // at most 4 x SMs)
     const long long rows = cfg->s * cfg->b;
-    const long long g = general_grid(rows, sms);   // >= the fast kernel's grid
-    *bytes = (size_t)g * 3 * (size_t)cfg->h * sizeof(float);
+    const long long fast = (rows < sms ? rows : sms) * (long long)kMaxGroups;
+    const long long gen = general_grid(rows, sms);
+    *bytes = (size_t)(fast > gen ? fast : gen) * 3 * (size_t)cfg->h * sizeof(float);
     return SP_OK;
 }
 
@@ -393,7 +514,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     a.hv = h / 8;
     a.t = cfg->t;
     a.seg_bytes = (uint32_t)(h * E);
-    a.stage_stride = (a.seg_bytes + 127u) & ~127u;
+    a.stage_stride = (uint32_t)round128(a.seg_bytes);
     a.mask_row_bytes = 4 * ((h + 31) / 32);
     a.h_f = (float)h;
     a.scale = 1.0f / (1.0f - cfg->p_drop);
@@ -401,57 +522,39 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     a.want_dbias = dbias ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-    int grid = 0;
-    int V = 0, C = 0;
+    long long nparts = 0;
     bool launched = false;
-    if (h % 8 == 0 && all16 && fast_shape(h / 8, &V, &C)) {
-        const size_t tailb = ring_tail_bytes();
-        const size_t pstride = round128((size_t)h * E);
-        const size_t accb = bwd_acc_in_smem(V) ? (size_t)3 * 2 * a.hv * sizeof(float4) : 0;
-        long long S = ((long long)dev.smem_optin - (long long)(tailb + pstride + accb)) /
-                      a.stage_stride;
-        if (S > 64) S = 64;
-        if (S >= 2) {
-            a.stages = (int)S;
-            a.param_off = (uint32_t)(S * a.stage_stride);
-            a.acc_off = (uint32_t)(a.param_off + pstride);
-            a.tail_off = (uint32_t)(a.acc_off + accb);
-            grid = (int)fast_grid(rows, dev.sms);
-            if ((size_t)grid * 3 * h * sizeof(float) > workspace_bytes) return SP_ERR_INVALID_ARG;
-            const size_t smem = (size_t)a.tail_off + tailb;
-            if (cfg->dtype == SP_BF16)
-                rc = ln ? launch_bwd_fast<__nv_bfloat16, true>(a, V, C, grid, smem, st)
-                        : launch_bwd_fast<__nv_bfloat16, false>(a, V, C, grid, smem, st);
-            else
-                rc = ln ? launch_bwd_fast<float, true>(a, V, C, grid, smem, st)
-                        : launch_bwd_fast<float, false>(a, V, C, grid, smem, st);
-            if (rc) return rc;
+    if (h % 8 == 0 && all16) {
+        const FastLaunch L = plan_bwd(a, dev, E, cfg->bwd_plan);
+        if (L.plan >= 0) {
+            nparts = (long long)L.grid * (kBwdPlans[L.plan].acc_smem ? 1 : L.groups);
+            if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes)
+                return SP_ERR_INVALID_ARG;
+            const void* kern = ln ? bwd_kernel_dt<true>(cfg->dtype, L.plan)
+                                  : bwd_kernel_dt<false>(cfg->dtype, L.plan);
+            if ((rc = launch_kernel(kern, L.grid, L.block, L.smem, st, &a))) return rc;
             launched = true;
         }
     }
     if (!launched) {
         const size_t smem = (size_t)h * 4;
         if (smem > (size_t)dev.smem_optin - 1024) return SP_ERR_UNSUPPORTED;
-        grid = (int)general_grid(rows, dev.sms);
-        if ((size_t)grid * 3 * h * sizeof(float) > workspace_bytes) return SP_ERR_INVALID_ARG;
-        auto go = [&](auto kern) -> int {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)smem) != cudaSuccess)
-                return SP_ERR_CUDA;
-            kern<<<grid, kGeneralThreads, smem, st>>>(a);
-            return launch_status();
-        };
+        nparts = general_grid(rows, dev.sms);
+        if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes) return SP_ERR_INVALID_ARG;
+        const void* kern;
         if (cfg->dtype == SP_BF16)
-            rc = ln ? go(k_bwd_general<__nv_bfloat16, true>) : go(k_bwd_general<__nv_bfloat16, false>);
+            kern = ln ? (const void*)k_bwd_general<__nv_bfloat16, true>
+                      : (const void*)k_bwd_general<__nv_bfloat16, false>;
         else
-            rc = ln ? go(k_bwd_general<float, true>) : go(k_bwd_general<float, false>);
-        if (rc) return rc;
+            kern = ln ? (const void*)k_bwd_general<float, true>
+                      : (const void*)k_bwd_general<float, false>;
+        if ((rc = launch_kernel(kern, (int)nparts, kGeneralThreads, smem, st, &a))) return rc;
     }
-    const long long n = 3LL * h;
-    k_colreduce<<<(int)((n + 255) / 256), 256, 0, st>>>(a.ws, grid, h, dgamma,
-                                                        a.want_dbeta ? dbeta : nullptr,
-                                                        a.want_dbias ? dbias : nullptr);
-    return launch_status();
+    const int tiles = (h + 31) / 32;
+    k_colreduce<<<3 * tiles, 256, 0, st>>>(a.ws, (int)nparts, h, dgamma,
+                                           a.want_dbeta ? dbeta : nullptr,
+                                           a.want_dbias ? dbias : nullptr);
+    return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
 
 int sp_device_error(int32_t device, int32_t* code, int32_t clear)
@@ -477,9 +580,15 @@ int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream)
     DevInfo dev;
     int rc = use_device_of(status, &dev);
     if (rc) return rc;
-    k_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
-        (unsigned long long)limit_ns, reinterpret_cast<int*>(status));
-    return launch_status();
+    unsigned long long lim = (unsigned long long)limit_ns;
+    int* st = reinterpret_cast<int*>(status);
+    void* params[] = {&lim, &st};
+    if (cudaLaunchKernel((const void*)k_wait_selftest, dim3(1), dim3(32), params, 0,
+                         static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
 }
 
 }  // extern "C"

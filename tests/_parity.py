@@ -114,14 +114,16 @@ def unpack_mask(words, h):
     return bits.reshape(w.shape[0], -1)[:, :h]
 
 
-def cfg_of(w):
+def cfg_of(w, fwd_plan=0, bwd_plan=0):
     return sp.make_cfg(w.s, w.b, w.h, w.t, dtype=w.dtype, norm=w.norm,
                        eps=w.eps, p_drop=w.p_drop, seed=w.drop_seed,
-                       offset=w.drop_offset)
+                       offset=w.drop_offset, fwd_plan=fwd_plan,
+                       bwd_plan=bwd_plan)
 
 
 def gpu_fwd(w, parts, bias, residual, gamma, beta, n_gathered=1,
-            with_mask=True, with_stats=True, inplace=False, offset_elems=0):
+            with_mask=True, with_stats=True, inplace=False, offset_elems=0,
+            plan=0):
     """Run the forward through the C ABI on device copies of the inputs.
 
     offset_elems shifts every [s,b,h] buffer by that many elements from a
@@ -153,7 +155,8 @@ def gpu_fwd(w, parts, bias, residual, gamma, beta, n_gathered=1,
     mean_g = Guarded((N,), torch.float32, dev) if with_stats else None
     rstd_g = Guarded((N,), torch.float32, dev) if with_stats else None
     sp.sp_rs_bias_dropout_add_norm_fwd(
-        cfg_of(w), [g.t for g, _ in gp], gb, res_t, gg, gbe, rout,
+        cfg_of(w, fwd_plan=plan), [g.t for g, _ in gp], gb, res_t, gg, gbe,
+        rout,
         [g.t for g in gath],
         mask_bits=mask_g.t if mask_g else None,
         mean=mean_g.t if mean_g else None, rstd=rstd_g.t if rstd_g else None)
@@ -170,7 +173,7 @@ def gpu_fwd(w, parts, bias, residual, gamma, beta, n_gathered=1,
 
 
 def gpu_bwd(w, dparts, drnext, x, gamma, mask, mean, rstd, with_dbeta=True,
-            with_dbias=True, offset_elems=0):
+            with_dbias=True, offset_elems=0, plan=0):
     dev = "cuda"
     dt = w.torch_dtype
     N, h = w.rows, w.h
@@ -199,7 +202,7 @@ def gpu_bwd(w, dparts, drnext, x, gamma, mask, mean, rstd, with_dbeta=True,
     dgam_g = Guarded((h,), torch.float32, dev)
     dbet_g = Guarded((h,), torch.float32, dev) if with_dbeta else None
     dbia_g = Guarded((h,), torch.float32, dev) if with_dbias else None
-    cfg = cfg_of(w)
+    cfg = cfg_of(w, bwd_plan=plan)
     nws = sp.sp_bwd_workspace_bytes(cfg)
     ws = torch.empty(nws // 4 + 4, dtype=torch.float32, device=dev)
     ws.fill_(float("nan"))   # the kernel must not need zeroed scratch

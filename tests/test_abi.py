@@ -22,8 +22,12 @@ def _header_functions():
 
 @pytest.fixture(scope="module")
 def lib():
-    from sp_region_b200 import build
-    build.build()
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "sp_region_build", os.path.join(ROOT, "sp_region_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
     return ctypes.CDLL(LIB)
 
 
