@@ -266,6 +266,42 @@ int sp_device_error(int32_t device, int32_t* code, int32_t clear);
  * = 0 would mean the wait completed. */
 int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream);
 
+/*
+ * Backward without caller-provided scratch: sp_rs_norm_dropout_bwd with the
+ * workspace taken from a fixed array inside the library.  The pages have no
+ * counterpart; this exists for callers that cannot allocate device memory
+ * where they run the backward (a memory-capped arena that owns every byte, an
+ * allocator that must not be re-entered from here, or a loop that may not
+ * synchronise, since cudaMalloc and cudaFree can).
+ *
+ * Arguments, layout and results are those of sp_rs_norm_dropout_bwd without
+ * `workspace` / `workspace_bytes`.  The call allocates nothing: the scratch
+ * is a 64 MiB array of this library's device image, reserved on every GPU
+ * that loads the library and held until the process exits.
+ *
+ * Limit   a configuration whose sp_bwd_workspace_bytes() exceeds 64 MiB is
+ *         rejected with SP_ERR_UNSUPPORTED before any launch (on a 148-SM
+ *         B200 that is h > 9447).
+ * Set-up  the first call on a device looks up the array's device address
+ *         (cudaGetSymbolAddress) and caches it; make that first call before
+ *         any stream capture.
+ * Sharing every call on a device uses the same array and leaves its
+ *         contents behind; the kernels write every part of it they read, so
+ *         nothing needs clearing, but calls that overlap on the GPU (other
+ *         streams, other host threads) race on it and must be serialised by
+ *         the caller.
+ */
+int sp_rs_norm_dropout_bwd_noalloc(const sp_cfg* cfg,
+                                   const void* const* dn_partials,
+                                   const void* dR_next,
+                                   const void* residual_out,
+                                   const void* gamma,
+                                   const uint32_t* mask_bits,
+                                   const float* mean, const float* rstd,
+                                   void* dresidual_in, void* dY,
+                                   float* dgamma, float* dbeta, float* dbias,
+                                   void* stream);
+
 #ifdef __cplusplus
 }
 #endif

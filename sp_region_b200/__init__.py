@@ -32,7 +32,8 @@ SP_MAX_T = 64
 EXPORTS = ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
            "sp_rs_norm_dropout_bwd", "sp_bwd_workspace_bytes",
            "sp_activation_bytes", "sp_status_string", "sp_device_error",
-           "sp_debug_wait_timeout", "sp_plan_count")
+           "sp_debug_wait_timeout", "sp_plan_count",
+           "sp_rs_norm_dropout_bwd_noalloc")
 
 
 class SPError(RuntimeError):
@@ -74,6 +75,8 @@ def _load() -> ctypes.CDLL:
     lib.sp_device_error.argtypes = [i32, ctypes.POINTER(i32), i32]
     lib.sp_debug_wait_timeout.argtypes = [i64, vp, vp]
     lib.sp_plan_count.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(i32)]
+    lib.sp_rs_norm_dropout_bwd_noalloc.argtypes = [
+        cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     for f in EXPORTS:
         getattr(lib, f).restype = (ctypes.c_char_p if f == "sp_status_string"
                                    else ctypes.c_int)
@@ -165,6 +168,23 @@ def sp_rs_norm_dropout_bwd(cfg: sp_cfg, dn_partials, dR_next, residual_out,
                _p(residual_out), _p(gamma), _p(mask_bits), _p(mean), _p(rstd),
                _p(dresidual_in), _p(dY), _p(dgamma), _p(dbeta), _p(dbias),
                _p(workspace), workspace.numel() * workspace.element_size(),
+               _stream(stream, residual_out)))
+
+
+def sp_rs_norm_dropout_bwd_noalloc(cfg: sp_cfg, dn_partials, dR_next,
+                                   residual_out, gamma, mask_bits, mean, rstd,
+                                   dresidual_in, dY, dgamma, dbeta, dbias,
+                                   stream=None) -> None:
+    """The backward with its scratch in the library's fixed 64 MiB device
+    array instead of a caller buffer, for callers that cannot allocate device
+    memory at this point.  Calls that overlap on the GPU share that array and
+    must be serialised; the first call on a device looks up the array's
+    address and should come before any stream capture."""
+    _check("sp_rs_norm_dropout_bwd_noalloc",
+           _lib.sp_rs_norm_dropout_bwd_noalloc(
+               ctypes.byref(cfg), _ptrs(dn_partials), _p(dR_next),
+               _p(residual_out), _p(gamma), _p(mask_bits), _p(mean), _p(rstd),
+               _p(dresidual_in), _p(dY), _p(dgamma), _p(dbeta), _p(dbias),
                _stream(stream, residual_out)))
 
 

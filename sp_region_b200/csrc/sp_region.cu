@@ -5,6 +5,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "sp_region.h"
 #include "sp_bwd.cuh"
 #include "sp_device.cuh"
@@ -592,3 +594,72 @@ int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without caller-provided scratch.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// backward: code inside a memory-capped arena that owns every byte, a
+// runtime whose allocator must not be re-entered from this call, or a host
+// loop that may not synchronise (cudaMalloc and cudaFree can synchronise the
+// device).  For them the scratch of the parameter-gradient partial sums lives
+// in one fixed array in this library's device image instead of a buffer they
+// pass in.  The array is reserved on every GPU that loads the library and is
+// held until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;   // 64 MiB per GPU
+constexpr int kNoAllocMaxDevices = 64;
+
+}  // namespace
+
+// Host code must not use this name as a device address: it is the host-side
+// stand-in of the symbol.  Its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on device `dev`, which must be the
+// current device.  Looked up on the first call per device, then cached.
+int noalloc_scratch(int dev, void** out)
+{
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return SP_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return SP_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SP_OK;
+}
+
+}  // namespace
+
+extern "C" int sp_rs_norm_dropout_bwd_noalloc(
+    const sp_cfg* cfg, const void* const* dn_partials, const void* dR_next,
+    const void* residual_out, const void* gamma, const uint32_t* mask_bits, const float* mean,
+    const float* rstd, void* dresidual_in, void* dY, float* dgamma, float* dbeta, float* dbias,
+    void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (!residual_out) return SP_ERR_INVALID_ARG;
+    DevInfo dev;
+    if ((rc = use_device_of(residual_out, &dev))) return rc;   // makes it current
+    size_t need = 0;
+    if ((rc = sp_bwd_workspace_bytes(cfg, dev.id, &need))) return rc;
+    if (need > kNoAllocScratchBytes) return SP_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    if ((rc = noalloc_scratch(dev.id, &scratch))) return rc;
+    return sp_rs_norm_dropout_bwd(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits,
+                                  mean, rstd, dresidual_in, dY, dgamma, dbeta, dbias, scratch,
+                                  kNoAllocScratchBytes, stream);
+}
