@@ -119,18 +119,23 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(&tail->empty[s_]));
     };
-    // turn q of CTA row j: phase j of turn[q] completes when row j's group has
-    // finished that pass; row j waits for phase j-1 (only one phase can be
-    // outstanding, since row j-2 is this group's own previous row)
+    // Turns of the shared accumulators, passed around the groups in CTA row
+    // order: when row j finishes pass q it arrives on turn[q][next group],
+    // and row j waits on turn[q][its own group] for the completion that row
+    // j-1 made.  Group g's k-th row (j = g + k*G) waits for completion k of
+    // its barrier (k-1 for group 0, whose first row has no predecessor).  A
+    // barrier's next completion needs this group's own turn first, so no
+    // barrier ever runs two phases ahead of its waiter.
     constexpr bool kTurns = ACC_SMEM && (G > 1);
     auto take_turn = [&](int q, long long j) {
-        if (kTurns && j > 0)
-            mbar_wait(smem_addr(&tail->turn[q]), (uint32_t)((j - 1) & 1), abort, ERR_WAIT_FULL);
+        if (!kTurns || j == 0) return;
+        const long long k = (j - g) / G - (g == 0 ? 1 : 0);
+        mbar_wait(smem_addr(&tail->turn[q][g]), (uint32_t)(k & 1), abort, ERR_WAIT_FULL);
     };
     auto pass_turn = [&](int q) {
         if (kTurns) {
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&tail->turn[q]));
+            if (lane == 0) mbar_arrive(smem_addr(&tail->turn[q][g + 1 == G ? 0 : g + 1]));
         }
     };
 
@@ -150,8 +155,12 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             kb[i] = (a.mask && v < hv) ? a.mask[(size_t)n * a.mask_row_bytes + v] : 0xFFu;
         }
 
-        // reduce-scatter of the upstream gradient partials
+        // reduce-scatter of the upstream gradient partials, k ascending, from +0
         float dn[V][8];
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dn[i][e] = 0.f;
         for (int k = 0; k < a.t; ++k) {
             mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
             const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
@@ -162,7 +171,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
                     float f[8];
                     IO<T>::unpack(load_vec<T>(buf, v), f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) dn[i][e] = (k == 0) ? f[e] : dn[i][e] + f[e];
+                    for (int e = 0; e < 8; ++e) dn[i][e] += f[e];
                 }
             }
             release_at(pos.abs());
@@ -209,11 +218,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             float2* red = reinterpret_cast<float2*>(tail->red[parity][g]);
             if (lane == 0) red[c >> 5] = tot;
             asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
-            tot = make_float2(0.f, 0.f);
-            for (int w = 0; w < (C >> 5); ++w) {
-                tot.x += red[w].x;
-                tot.y += red[w].y;
-            }
+            tot = warps_total2(red, C >> 5);
         }
         const float mg = tot.x / a.h_f, mgx = tot.y / a.h_f;
 

@@ -71,15 +71,20 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// A thread whose phase has not completed is suspended in hardware until the
+// phase completes or about kSuspendHintNs pass, so waiting warps do not spin
+// on the issue slots the working warps need.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -289,6 +294,23 @@ __device__ __forceinline__ float warp_sum(float x)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
     return x;
+}
+
+// Second level of a group reduction: lane l adds the total of warp l (warps
+// have stored theirs in red[0 .. nwarps)); every lane of every warp ends with
+// the same bits (an xor butterfly combines the same two partials on both
+// sides of each exchange).
+__device__ __forceinline__ float warps_total(const float* red, int nwarps)
+{
+    const int lane = threadIdx.x & 31;
+    return warp_sum(lane < nwarps ? red[lane] : 0.f);
+}
+
+__device__ __forceinline__ float2 warps_total2(const float2* red, int nwarps)
+{
+    const int lane = threadIdx.x & 31;
+    const float2 v = lane < nwarps ? red[lane] : make_float2(0.f, 0.f);
+    return make_float2(warp_sum(v.x), warp_sum(v.y));
 }
 
 // Block-wide sum for the general kernels (all threads take part).

@@ -59,14 +59,14 @@ struct FwdArgs {
 
 // Shared-memory tail after the ring: barriers, per-group reduction scratch,
 // abort flag.
-constexpr int kMaxGroups = 4;
+constexpr int kMaxGroups = 6;
 // Reduction scratch: two buffers per group, used alternately by row parity
 // (or by the two reductions of one LayerNorm row), so a warp that runs ahead
 // to the next row never overwrites totals a slower warp is still reading.
 struct RingTail {
     uint64_t full[64];
     uint64_t empty[64];
-    uint64_t turn[2];   // backward: shared-accumulator turns, in row order
+    uint64_t turn[2][kMaxGroups];   // backward: shared-accumulator turns
     float red[2][kMaxGroups][64];
     int abort;
 };
@@ -161,8 +161,10 @@ __device__ __forceinline__ void init_ring(RingTail* tail, int S, int warps_per_g
             mbar_init(smem_addr(&tail->full[s]), 1);
             mbar_init(smem_addr(&tail->empty[s]), warps_per_group);
         }
-        mbar_init(smem_addr(&tail->turn[0]), warps_per_group);
-        mbar_init(smem_addr(&tail->turn[1]), warps_per_group);
+        for (int g = 0; g < kMaxGroups; ++g) {
+            mbar_init(smem_addr(&tail->turn[0][g]), warps_per_group);
+            mbar_init(smem_addr(&tail->turn[1][g]), warps_per_group);
+        }
         tail->abort = 0;
         mbar_init_fence();
     }
@@ -222,9 +224,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
         x = warp_sum(x);
         if (lane == 0) red[c >> 5] = x;
         asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
-        float s_ = 0.f;
-        for (int w = 0; w < (C >> 5); ++w) s_ += red[w];
-        return s_;
+        return warps_total(red, C >> 5);
     };
 
     const uint32_t Sg = (uint32_t)(S / G);
@@ -239,8 +239,12 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
         const long long n = blockIdx.x + j * (long long)gridDim.x;
         if (n >= a.rows) break;
 
+        // reduce-scatter: sum of the t partial rows, k ascending, from +0
         float acc[V][8];
-        // reduce-scatter: sum of the t partial rows, k ascending
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
         for (int k = 0; k < a.t; ++k) {
             mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
             const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
@@ -251,7 +255,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                     float f[8];
                     IO<T>::unpack(load_vec<T>(buf, v), f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[i][e] = (k == 0) ? f[e] : acc[i][e] + f[e];
+                    for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
                 }
             }
             release();

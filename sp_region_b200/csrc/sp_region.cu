@@ -104,6 +104,9 @@ constexpr Plan kFwdPlans[] = {
     {3, 2, 800, false},    // 6
     {4, 1, 544, false},    // 7
     {4, 2, 800, false},    // 8
+    {2, 3, 800, false},    // 9
+    {4, 4, 544, false},    // 10
+    {4, 6, 800, false},    // 11
 };
 constexpr Plan kBwdPlans[] = {
     {1, 1, 1024, false},   // 0
@@ -117,14 +120,18 @@ constexpr Plan kBwdPlans[] = {
     {2, 2, 800, true},     // 8
     {3, 2, 800, true},     // 9
     {4, 2, 800, true},     // 10
+    {2, 3, 800, true},     // 11
+    {4, 4, 544, true},     // 12
 };
 constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
 constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
 
 // Preference order when the caller gives no hint: the first feasible plan
 // wins.  A hinted plan is tried first.
-constexpr int kFwdOrder[] = {4, 1, 2, 6, 8, 0, 3, 5, 7};
-constexpr int kBwdOrder[] = {8, 9, 2, 3, 5, 10, 6, 1, 0, 4, 7};
+// (measured on B200 for h = 4096 ... 12288: more rows in flight per SM wins
+// while the registers and the ring's stages allow it)
+constexpr int kFwdOrder[] = {10, 4, 9, 6, 8, 1, 2, 11, 0, 3, 5, 7};
+constexpr int kBwdOrder[] = {11, 8, 9, 12, 2, 3, 5, 10, 6, 1, 0, 4, 7};
 
 int group_threads(int hv, int V)
 {
@@ -149,7 +156,8 @@ const void* fwd_kernel(int id)
 {
     switch (id) {
         SP_FWD_CASE(0) SP_FWD_CASE(1) SP_FWD_CASE(2) SP_FWD_CASE(3) SP_FWD_CASE(4)
-        SP_FWD_CASE(5) SP_FWD_CASE(6) SP_FWD_CASE(7) SP_FWD_CASE(8)
+        SP_FWD_CASE(5) SP_FWD_CASE(6) SP_FWD_CASE(7) SP_FWD_CASE(8) SP_FWD_CASE(9)
+        SP_FWD_CASE(10) SP_FWD_CASE(11)
     }
     return nullptr;
 }
@@ -165,7 +173,7 @@ const void* bwd_kernel(int id)
     switch (id) {
         SP_BWD_CASE(0) SP_BWD_CASE(1) SP_BWD_CASE(2) SP_BWD_CASE(3) SP_BWD_CASE(4)
         SP_BWD_CASE(5) SP_BWD_CASE(6) SP_BWD_CASE(7) SP_BWD_CASE(8) SP_BWD_CASE(9)
-        SP_BWD_CASE(10)
+        SP_BWD_CASE(10) SP_BWD_CASE(11) SP_BWD_CASE(12)
     }
     return nullptr;
 }
