@@ -344,9 +344,15 @@ def run_ours(args):
 
 
 def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
-    """Same metric through the public API with host buffers: every step copies
-    its inputs from pinned host memory, runs forward and backward, and reads
-    every output back to pinned host memory, inside the timed region."""
+    """Same metric through the public API with host buffers: every step
+    copies its inputs from pinned host memory, runs forward and backward, and
+    reads every output back to pinned host memory, inside the timed region.
+
+    Steps are pipelined the way a caller with host buffers would run them:
+    inputs are double-buffered on the device, uploads run on one copy stream,
+    the boundary on the compute stream and downloads on another copy stream,
+    so step i+1's upload overlaps step i's compute and download (PCIe carries
+    both directions at once)."""
     import sp_synth
     N, h = w.rows, w.h
     dt = w.torch_dtype
@@ -362,12 +368,12 @@ def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
     hd = [pin(p) for p in sp_synth.draw_grad_partials(w, dev)]
     ins = [*hp, hb, hg, hbe, hr, *hd]
     h2d = sum(x.numel() * x.element_size() for x in ins if x is not None)
-    dev_in = [None if x is None else torch.empty_like(x, device=dev)
-              for x in ins]
     t = w.t
-    d_parts, d_b, d_g, d_be, d_r = (dev_in[:t], dev_in[t], dev_in[t + 1],
-                                    dev_in[t + 2], dev_in[t + 3])
-    d_dp = dev_in[t + 4:]
+    bufs = []
+    for _ in range(2):
+        dev_in = [None if x is None else torch.empty_like(x, device=dev)
+                  for x in ins]
+        bufs.append(dev_in)
     outs_d = dict(rout=torch.empty((N, h), dtype=dt, device=dev),
                   out=torch.empty((N, h), dtype=dt, device=dev),
                   mask=torch.empty((N, (h + 31) // 32), dtype=torch.int32,
@@ -390,33 +396,73 @@ def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
               if v is not None)
     ws = torch.empty(sp.sp_bwd_workspace_bytes(cfg, dev.index) // 4,
                      dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    comp = torch.cuda.current_stream(dev)
+    up = torch.cuda.Stream(dev)
+    down = torch.cuda.Stream(dev)
 
-    def step():
-        for d_, h_ in zip(dev_in, ins):
-            if h_ is not None:
-                d_.copy_(h_, non_blocking=True)
+    def upload(i):
+        """enqueue step i's input copies; returns the event that marks them"""
+        dev_in = bufs[i % 2]
+        with torch.cuda.stream(up):
+            # the buffer set was last read by step i-2's compute
+            if i >= 2:
+                up.wait_event(done_compute[i - 2])
+            for d_, h_ in zip(dev_in, ins):
+                if h_ is not None:
+                    d_.copy_(h_, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(up)
+        return ev
+
+    def compute(i, uploaded):
+        dev_in = bufs[i % 2]
+        d_parts, d_b, d_g, d_be, d_r = (dev_in[:t], dev_in[t], dev_in[t + 1],
+                                        dev_in[t + 2], dev_in[t + 3])
+        d_dp = dev_in[t + 4:]
+        comp.wait_event(uploaded)
+        if i >= 1:
+            comp.wait_event(done_download[i - 1])   # outputs are reused
         o = outs_d
         sp.sp_rs_bias_dropout_add_norm_fwd(cfg, d_parts, d_b, d_r, d_g, d_be,
                                            o["rout"], [o["out"]], o["mask"],
-                                           o["mean"], o["rstd"], stream=stream)
+                                           o["mean"], o["rstd"], stream=comp)
         sp.sp_rs_norm_dropout_bwd(cfg, d_dp, None, o["rout"], d_g, o["mask"],
                                   o["mean"], o["rstd"], o["dres"], o["dY"],
-                                  o["dg"], o["db"], o["dc"], ws, stream=stream)
-        for k, v in o.items():
-            if v is not None:
-                outs_h[k].copy_(v, non_blocking=True)
+                                  o["dg"], o["db"], o["dc"], ws, stream=comp)
+        ev = torch.cuda.Event()
+        ev.record(comp)
+        done_compute[i] = ev
 
-    for _ in range(2):
-        step()
+    def download(i):
+        with torch.cuda.stream(down):
+            down.wait_event(done_compute[i])
+            for k, v in outs_d.items():
+                if v is not None:
+                    outs_h[k].copy_(v, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(down)
+            done_download[i] = ev
+
+    def run(nsteps):
+        uploaded = upload(0)
+        for i in range(nsteps):
+            nxt = upload(i + 1) if i + 1 < nsteps else None
+            compute(i, uploaded)
+            download(i)
+            uploaded = nxt
+
+    done_compute, done_download = {}, {}
+    run(2)
     torch.cuda.synchronize(dev)
     K = args.e2e_steps
+    done_compute, done_download = {}, {}
+    torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(K):
-        step()
-    e1.record(stream)
+    e0.record(up)
+    run(K)
+    down.wait_event(done_download[K - 1])
+    e1.record(down)
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1)
     if world > 1:
@@ -427,8 +473,10 @@ def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
     return {"value": round(step_bytes * world * K / (ms * 1e-3) / 1e9, 2),
             "unit": "GB/s", "ms_per_step": round(ms / K, 3), "steps": K,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "path": "pinned host -> device copies, fwd + bwd through the C "
-                    "ABI, every output copied back to pinned host"}
+            "path": "every step: pinned host -> device copies of all inputs, "
+                    "fwd + bwd through the C ABI, every output copied back "
+                    "to pinned host; uploads, compute and downloads on three "
+                    "streams, inputs double-buffered"}
 
 
 # ----------------------------------------------------------------------------
@@ -526,7 +574,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="C2")
-    ap.add_argument("--e2e-steps", type=int, default=4)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--fwd-plan", type=int, default=0,

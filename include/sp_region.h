@@ -96,7 +96,18 @@ typedef enum { SP_LAYERNORM = 0, SP_RMSNORM = 1 } sp_norm;
  *            fits the shape, else the library chooses.  Results do not
  *            depend on the plan except through the fp32 summation order of
  *            the backward's parameter gradients.  Out-of-range values are
- *            treated as 0. */
+ *            treated as 0.
+ *   row_begin, row_end   the global token rows [row_begin, row_end) this
+ *            call processes; 0, 0 means all N rows.  With t GPUs as t real
+ *            ranks, rank r passes its own shard [r*N/t, (r+1)*N/t) (its
+ *            residual, stored outputs, mask and statistics hold only those
+ *            rows, indexed from 0) while partials, gathered outputs and dY
+ *            are full [s,b,h] tensors indexed by global row -- on a real
+ *            system, peers' buffers reached through peer pointers.  The
+ *            dropout counter uses the global row, so a split into ranges
+ *            gives exactly the rows of the whole call.  Parameter gradients
+ *            of a range cover its rows only; summing them over the ranges
+ *            (the all-reduce of replicated parameters) gives the total. */
 typedef struct {
     int64_t s, b, h;
     int32_t t;
@@ -106,6 +117,7 @@ typedef struct {
     float p_drop;
     uint64_t seed, offset;
     int32_t fwd_plan, bwd_plan;
+    int64_t row_begin, row_end;
 } sp_cfg;
 
 /* Number of fast-kernel plans of the forward and the backward (valid hint

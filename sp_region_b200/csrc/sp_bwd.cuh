@@ -38,7 +38,8 @@ struct BwdArgs {
     void* dres;
     void* dY;
     float* ws;               // [gridDim.x][3][h] per-CTA partial sums
-    long long rows;
+    long long rows;          // token rows of this call (local index i)
+    long long row0;          // global index of local row 0: n = row0 + i
     int h;
     int hv;
     int t;
@@ -77,9 +78,16 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
     if (tid >= G * C) {
         if (tid == G * C)
             ring_produce<G>(smem, tail, abort, a.rows, nsrc, a.seg_bytes, a.stage_stride, S,
-                         [&](int k) {
-                             return k < a.t ? a.dparts[k] : (k == a.t ? a.x : a.drnext);
-                         });
+                            [&](int k, long long i) -> const void* {
+                                // upstream partials by global row; x and dR_next
+                                // are this call's shard, by local row
+                                if (k < a.t)
+                                    return static_cast<const unsigned char*>(a.dparts[k]) +
+                                           (size_t)(a.row0 + i) * a.seg_bytes;
+                                return static_cast<const unsigned char*>(k == a.t ? a.x
+                                                                                  : a.drnext) +
+                                       (size_t)i * a.seg_bytes;
+                            });
         return;
     }
 
@@ -143,16 +151,17 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
     RingPos pos((uint32_t)g * Sg, 0, Sg);
     int parity = 0;
     for (long long j = g;; j += G, parity ^= 1) {
-        const long long n = blockIdx.x + j * (long long)gridDim.x;
-        if (n >= a.rows) break;
+        const long long i_row = blockIdx.x + j * (long long)gridDim.x;   // local row
+        if (i_row >= a.rows) break;
+        const long long n = a.row0 + i_row;                                // global row
         // loads whose latency overlaps the reduction below
-        const float rstd = a.rstd[n];
-        const float mean = LN ? a.mean[n] : 0.f;
+        const float rstd = a.rstd[i_row];
+        const float mean = LN ? a.mean[i_row] : 0.f;
         uint32_t kb[V];
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
-            kb[i] = (a.mask && v < hv) ? a.mask[(size_t)n * a.mask_row_bytes + v] : 0xFFu;
+            kb[i] = (a.mask && v < hv) ? a.mask[(size_t)i_row * a.mask_row_bytes + v] : 0xFFu;
         }
 
         // reduce-scatter of the upstream gradient partials, k ascending, from +0
@@ -233,8 +242,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 
         // pass 2: input gradient, residual gradient, dropout backward
         take_turn(1, j);
-        unsigned char* dres = static_cast<unsigned char*>(a.dres) + (size_t)n * a.seg_bytes;
-        unsigned char* dy = static_cast<unsigned char*>(a.dY) + (size_t)n * a.seg_bytes;
+        unsigned char* dres =
+            static_cast<unsigned char*>(a.dres) + (size_t)i_row * a.seg_bytes;   // shard
+        unsigned char* dy =
+            static_cast<unsigned char*>(a.dY) + (size_t)n * a.seg_bytes;       // gathered
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
@@ -318,17 +329,19 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
     float* ws = a.ws + (size_t)blockIdx.x * 3 * h;
     for (int j = threadIdx.x; j < 3 * h; j += blockDim.x) ws[j] = 0.f;
 
-    for (long long n = blockIdx.x; n < a.rows; n += gridDim.x) {
-        const long long base = n * (long long)h;
-        const float rstd = a.rstd[n];
-        const float mean = LN ? a.mean[n] : 0.f;
+    for (long long i_row = blockIdx.x; i_row < a.rows; i_row += gridDim.x) {
+        const long long n = a.row0 + i_row;              // global row
+        const long long base = n * (long long)h;         // upstream partials, dY
+        const long long lbase = i_row * (long long)h;    // this call's shard
+        const float rstd = a.rstd[i_row];
+        const float mean = LN ? a.mean[i_row] : 0.f;
         float sg = 0.f, sgx = 0.f;
         for (int j = threadIdx.x; j < h; j += blockDim.x) {
             float d = 0.f;
             for (int k = 0; k < a.t; ++k) d = (k == 0) ? IO<T>::load1(a.dparts[k], base + j)
                                                        : d + IO<T>::load1(a.dparts[k], base + j);
             dns[j] = d;
-            const float xv = IO<T>::load1(a.x, base + j);
+            const float xv = IO<T>::load1(a.x, lbase + j);
             const float xh = LN ? (xv - mean) * rstd : xv * rstd;
             const float gg = d * IO<T>::load1(a.gamma, j);
             sg += gg;
@@ -340,14 +353,14 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
         const float mgx = block_sum(sgx, red) / a.h_f;
         for (int j = threadIdx.x; j < h; j += blockDim.x) {
             const float d = dns[j];
-            const float xv = IO<T>::load1(a.x, base + j);
+            const float xv = IO<T>::load1(a.x, lbase + j);
             const float xh = LN ? (xv - mean) * rstd : xv * rstd;
             const float gg = d * IO<T>::load1(a.gamma, j);
             const float dx = LN ? rstd * (gg - mg - xh * mgx) : rstd * (gg - xh * mgx);
-            const float dr = dx + (a.drnext ? IO<T>::load1(a.drnext, base + j) : 0.f);
-            IO<T>::store1(a.dres, base + j, dr);
+            const float dr = dx + (a.drnext ? IO<T>::load1(a.drnext, lbase + j) : 0.f);
+            IO<T>::store1(a.dres, lbase + j, dr);
             uint32_t keep = 1u;
-            if (a.mask) keep = (a.mask[(size_t)n * a.mask_row_bytes + (j >> 3)] >> (j & 7)) & 1u;
+            if (a.mask) keep = (a.mask[(size_t)i_row * a.mask_row_bytes + (j >> 3)] >> (j & 7)) & 1u;
             const float dz = keep ? dr * a.scale : 0.f;
             IO<T>::store1(a.dY, base + j, dz);
             if (a.want_dbias) ws[2 * h + j] += dz;

@@ -37,7 +37,8 @@ struct FwdArgs {
     uint8_t* mask;          // bytes: [rows][mask_row_bytes]
     float* mean;
     float* rstd;
-    long long rows;
+    long long rows;         // token rows of this call (local index i)
+    long long row0;         // global index of local row 0: n = row0 + i
     int h;
     int hv;                 // h / 8 (fast kernel)
     int t;
@@ -92,8 +93,8 @@ struct RingPos {
 
 // The producer lane: streams every segment of this CTA's rows, in row order.
 // Row j of the CTA belongs to consumer group j % G and goes to that group's
-// sub-ring (stages [g*Sg, (g+1)*Sg)).  nsrc sources per row; src(k) gives
-// source k's base pointer.
+// sub-ring (stages [g*Sg, (g+1)*Sg)).  nsrc sources per row; src(k, i) gives
+// the address of source k's segment for local row i.
 template <int G, typename SrcFn>
 __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail,
                                              volatile int* abort, long long rows,
@@ -114,8 +115,8 @@ __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail
     for (long long jj = 0; ok; ++jj) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const long long n = blockIdx.x + (jj * G + g) * (long long)gridDim.x;
-            if (!ok || n >= rows) {
+            const long long i = blockIdx.x + (jj * G + g) * (long long)gridDim.x;
+            if (!ok || i >= rows) {
                 ok = false;
                 break;
             }
@@ -125,8 +126,7 @@ __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail
                     ok = false;
                     break;
                 }
-                const unsigned char* p = static_cast<const unsigned char*>(src(k)) +
-                                         (size_t)n * seg_bytes;
+                const void* p = src(k, i);
                 const uint32_t bar = smem_addr(&tail->full[st]);
                 mbar_arrive_expect_tx(bar, seg_bytes);
                 bulk_load(smem_addr(smem + (size_t)st * stage_stride), p, seg_bytes, bar, pol);
@@ -196,7 +196,14 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
     if (tid >= G * C) {
         if (tid == G * C)
             ring_produce<G>(smem, tail, abort, a.rows, nsrc, a.seg_bytes, a.stage_stride, S,
-                            [&](int k) { return k < a.t ? a.parts[k] : a.residual; });
+                            [&](int k, long long i) -> const void* {
+                                // partial sums are indexed by global row, the
+                                // residual shard by local row
+                                return k < a.t ? static_cast<const unsigned char*>(a.parts[k]) +
+                                                     (size_t)(a.row0 + i) * a.seg_bytes
+                                               : static_cast<const unsigned char*>(a.residual) +
+                                                     (size_t)i * a.seg_bytes;
+                            });
         return;
     }
 
@@ -236,8 +243,9 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
     };
     int parity = 0;
     for (long long j = g;; j += G, parity ^= 1) {
-        const long long n = blockIdx.x + j * (long long)gridDim.x;
-        if (n >= a.rows) break;
+        const long long i_row = blockIdx.x + j * (long long)gridDim.x;   // local row
+        if (i_row >= a.rows) break;
+        const long long n = a.row0 + i_row;                                // global row
 
         // reduce-scatter: sum of the t partial rows, k ascending, from +0
         float acc[V][8];
@@ -262,7 +270,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
         }
 
         // bias once, then inverted dropout with the packed keep bits
-        uint8_t* mrow = a.mask ? a.mask + (size_t)n * a.mask_row_bytes : nullptr;
+        uint8_t* mrow = a.mask ? a.mask + (size_t)i_row * a.mask_row_bytes : nullptr;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
@@ -293,7 +301,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
         {
             const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
             unsigned char* rout =
-                static_cast<unsigned char*>(a.residual_out) + (size_t)n * a.seg_bytes;
+                static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.seg_bytes;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
@@ -366,8 +374,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
             }
         }
         if (c == 0) {
-            if (LN && a.mean) a.mean[n] = mean;
-            if (a.rstd) a.rstd[n] = rstd;
+            if (LN && a.mean) a.mean[i_row] = mean;
+            if (a.rstd) a.rstd[i_row] = rstd;
         }
     }
 }
@@ -384,10 +392,12 @@ __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ Fwd
     __shared__ float red[32];
     const int h = a.h;
 
-    for (long long n = blockIdx.x; n < a.rows; n += gridDim.x) {
+    for (long long i_row = blockIdx.x; i_row < a.rows; i_row += gridDim.x) {
+        const long long n = a.row0 + i_row;      // global row
         for (int w = threadIdx.x; w < W; w += blockDim.x) mw[w] = 0u;
         __syncthreads();
-        const long long base = n * (long long)h;
+        const long long base = n * (long long)h;         // partials, gathered
+        const long long lbase = i_row * (long long)h;    // this call's shard
         for (int j = threadIdx.x; j < h; j += blockDim.x) {
             float y = 0.f;
             for (int k = 0; k < a.t; ++k) y = (k == 0) ? IO<T>::load1(a.parts[k], base + j)
@@ -400,13 +410,14 @@ __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ Fwd
                 y = keep ? y * a.scale : 0.f;
             }
             if (keep) atomicOr(&mw[j >> 5], 1u << (j & 31));
-            const float r = IO<T>::round1(IO<T>::load1(a.residual, base + j) + y);
-            IO<T>::store1(a.residual_out, base + j, r);
+            const float r = IO<T>::round1(IO<T>::load1(a.residual, lbase + j) + y);
+            IO<T>::store1(a.residual_out, lbase + j, r);
             xs[j] = r;
         }
         __syncthreads();
         if (a.mask) {
-            uint32_t* mrow = reinterpret_cast<uint32_t*>(a.mask + (size_t)n * a.mask_row_bytes);
+            uint32_t* mrow =
+                reinterpret_cast<uint32_t*>(a.mask + (size_t)i_row * a.mask_row_bytes);
             for (int w = threadIdx.x; w < W; w += blockDim.x) mrow[w] = mw[w];
         }
         float mean = 0.f, rstd;
@@ -437,8 +448,8 @@ __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ Fwd
             for (int q = 0; q < a.n_gathered; ++q) IO<T>::store1(a.gathered[q], base + j, o);
         }
         if (threadIdx.x == 0) {
-            if (LN && a.mean) a.mean[n] = mean;
-            if (a.rstd) a.rstd[n] = rstd;
+            if (LN && a.mean) a.mean[i_row] = mean;
+            if (a.rstd) a.rstd[i_row] = rstd;
         }
         __syncthreads();   // xs / mw are reused by the next row
     }

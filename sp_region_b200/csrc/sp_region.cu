@@ -62,7 +62,22 @@ int check_cfg(const sp_cfg* c)
     if (c->s > (1LL << 32) || c->b > (1LL << 32)) return SP_ERR_INVALID_ARG;
     if (c->s * c->b > 0xFFFFFFFFLL) return SP_ERR_INVALID_ARG;
     if (c->h > (1LL << 24)) return SP_ERR_INVALID_ARG;
+    if (!(c->row_begin == 0 && c->row_end == 0) &&
+        !(c->row_begin >= 0 && c->row_begin < c->row_end && c->row_end <= c->s * c->b))
+        return SP_ERR_INVALID_ARG;
     return SP_OK;
+}
+
+// The token rows [*r0, *r0 + *nrows) a call processes.
+void call_rows(const sp_cfg* c, long long* r0, long long* nrows)
+{
+    if (c->row_begin == 0 && c->row_end == 0) {
+        *r0 = 0;
+        *nrows = c->s * c->b;
+    } else {
+        *r0 = c->row_begin;
+        *nrows = c->row_end - c->row_begin;
+    }
 }
 
 int elem_bytes(const sp_cfg* c) { return c->dtype == SP_F32 ? 4 : 2; }
@@ -357,7 +372,8 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
     DevInfo dev;
     if ((rc = use_device_of(residual, &dev))) return rc;
 
-    const long long rows = cfg->s * cfg->b;
+    long long row0 = 0, rows = 0;
+    call_rows(cfg, &row0, &rows);
     const int h = (int)cfg->h;
     FwdArgs a;
     memset(&a, 0, sizeof(a));
@@ -372,6 +388,7 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
     a.mean = ln ? mean : nullptr;
     a.rstd = rstd;
     a.rows = rows;
+    a.row0 = row0;
     a.h = h;
     a.hv = h / 8;
     a.t = cfg->t;
@@ -465,7 +482,8 @@ int sp_bwd_workspace_bytes(const sp_cfg* cfg, int32_t device, size_t* bytes)
     // partial sums of dgamma, dbeta, dbias, one slice per CTA (fast kernels:
     // per consumer group, at most SMs x 4 groups; general kernel: its grid of
     // at most 4 x SMs)
-    const long long rows = cfg->s * cfg->b;
+    long long row0 = 0, rows = 0;
+    call_rows(cfg, &row0, &rows);
     const long long fast = (rows < sms ? rows : sms) * (long long)kMaxGroups;
     const long long gen = general_grid(rows, sms);
     *bytes = (size_t)(fast > gen ? fast : gen) * 3 * (size_t)cfg->h * sizeof(float);
@@ -505,7 +523,8 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     DevInfo dev;
     if ((rc = use_device_of(residual_out, &dev))) return rc;
 
-    const long long rows = cfg->s * cfg->b;
+    long long row0 = 0, rows = 0;
+    call_rows(cfg, &row0, &rows);
     const int h = (int)cfg->h;
     BwdArgs a;
     memset(&a, 0, sizeof(a));
@@ -520,6 +539,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     a.dY = dY;
     a.ws = static_cast<float*>(workspace);
     a.rows = rows;
+    a.row0 = row0;
     a.h = h;
     a.hv = h / 8;
     a.t = cfg->t;
