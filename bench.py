@@ -71,6 +71,23 @@ def bwd_bytes(w, with_drnext=False):
     return rd + wr
 
 
+def entry_fwd_bytes(w, n_gathered=1):
+    """Entry into a TP region: read x, write the gathered norm output."""
+    E, N, h = w.elem_bytes, w.rows, w.h
+    params = h * E * (1 + (1 if w.norm == "layernorm" else 0))
+    stats = (8 if w.norm == "layernorm" else 4) * N
+    return E * N * h + params + n_gathered * E * N * h + stats
+
+
+def entry_bwd_bytes(w):
+    """Its backward: reduce-scatter of t upstream partials, norm backward from
+    x and the statistics, the residual-stream gradient written."""
+    E, N, h = w.elem_bytes, w.rows, w.h
+    stats = (8 if w.norm == "layernorm" else 4) * N
+    ngrad = 1 + (1 if w.norm == "layernorm" else 0)
+    return (w.t + 1) * E * N * h + stats + h * E + E * N * h + 4 * h * ngrad
+
+
 def measured_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -238,6 +255,22 @@ def run_ours(args):
                                   rstd, dres, dY, dg, db, dc, ws,
                                   stream=stream)
 
+    if args.op == "entry":
+        # the entry into a TP region: norm of the shard then all-gather; its
+        # backward: reduce-scatter of the upstream partials, norm backward
+        cfg0 = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm,
+                           eps=w.eps, p_drop=0.0, fwd_plan=args.fwd_plan,
+                           bwd_plan=args.bwd_plan)
+
+        def fwd():
+            sp.sp_norm_all_gather_fwd(cfg0, res, gamma, beta, [out], mean,
+                                      rstd, stream=stream)
+
+        def bwd():
+            sp.sp_rs_norm_dropout_bwd(cfg0, dparts, None, res, gamma, None,
+                                      mean, rstd, dres, None, dg, db, None,
+                                      ws, stream=stream)
+
     for _ in range(args.warmup):
         fwd()
         bwd()
@@ -280,7 +313,10 @@ def run_ours(args):
         dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
     total_ms = float(tmax.item())
 
-    fb, bb = fwd_bytes(w), bwd_bytes(w)
+    if args.op == "entry":
+        fb, bb = entry_fwd_bytes(w), entry_bwd_bytes(w)
+    else:
+        fb, bb = fwd_bytes(w), bwd_bytes(w)
     step_bytes = fb + bb
     value = step_bytes * world * K / (total_ms * 1e-3) / 1e9
     ms_step = total_ms / K
@@ -288,7 +324,9 @@ def run_ours(args):
     f_avg = statistics.mean(fwd_ms)
     b_avg = statistics.mean(bwd_ms)
     kern = {
-        "fwd": {"kernel": "k_fwd_tma", "bytes_per_launch": fb,
+        "fwd": {"kernel": "k_fwd_tma" + (" (entry: no partials)"
+                                         if args.op == "entry" else ""),
+                "bytes_per_launch": fb,
                 "avg_ms": f_avg, "gbs": fb / (f_avg * 1e-3) / 1e9},
         "bwd": {"kernel": "k_bwd_tma + k_colreduce", "bytes_per_launch": bb,
                 "avg_ms": b_avg, "gbs": bb / (b_avg * 1e-3) / 1e9},
@@ -303,11 +341,12 @@ def run_ours(args):
                 "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": dk["bytes_per_launch"]}
 
-    e2e = run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world)
-
+    e2e = None
     cpu = None
-    if rank == 0 and world == 1 and not args.skip_cpu_baseline:
-        cpu = cpu_baseline(w, fb, bb, budget_s=args.cpu_seconds)
+    if args.op == "boundary":
+        e2e = run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world)
+        if rank == 0 and world == 1 and not args.skip_cpu_baseline:
+            cpu = cpu_baseline(w, fb, bb, budget_s=args.cpu_seconds)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s",
@@ -318,7 +357,11 @@ def run_ours(args):
         "config": {
             "workload": (f"{w.name}: SP boundary fwd+bwd, s={w.s} b={w.b} "
                          f"h={h} t={t} emulated ranks, {w.dtype} I/O, "
-                         f"{w.norm}, p={w.p_drop}, bias"),
+                         f"{w.norm}, p={w.p_drop}, bias"
+                         if args.op == "boundary" else
+                         f"{w.name} shape: entry into a TP region (norm + "
+                         f"all-gather) fwd+bwd, s={w.s} b={w.b} h={h} t={t}, "
+                         f"{w.dtype} I/O, {w.norm}"),
             "s": w.s, "b": w.b, "h": h, "t": t,
             "global_batch": w.b * world, "seq_len": w.s,
             "parallelism": f"{world} independent replicas (t={t} ranks "
@@ -574,6 +617,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="C2")
+    ap.add_argument("--op", default="boundary", choices=["boundary", "entry"],
+                    help="boundary: the exit of a TP region (reduce-scatter "
+                         "+ epilogue + all-gather); entry: norm + all-gather")
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")

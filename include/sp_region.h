@@ -179,6 +179,37 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg,
                                     float* rstd, void* stream);
 
 /*
+ * Entry into a tensor-parallel region: per-token norm of the caller's shard,
+ * then the all-gather into the full [s,b,h] input of the column-parallel
+ * linear.
+ *
+ * Defined by: "SP: Partition Activations Alongside TP", section "Connect SP
+ * and TP across a layer" (in a pre-norm layer each GPU first normalizes its
+ * own tokens, then the all-gather combines the inputs of the QKV / first FFN
+ * projection); "TP and SP explained with pictures", section "Add Sequence
+ * parallelism" (apply LayerNorm locally, then all-gather).
+ *
+ * For every token row n of the call (cfg->row_begin/row_end, default all):
+ *   LN:  o = (x - mean) * rstd * gamma + beta   RMS: o = x * rstd * gamma
+ *   gathered[q][n, :] = round(o) for every q < n_gathered
+ * cfg->p_drop is ignored (no dropout here); nothing is reduced.
+ *
+ * Arguments (device unless stated):
+ *   x          [s,b,h] (the caller's shard when a row range is given)
+ *   gamma      [h];  beta [h] or NULL (ignored for RMSNorm)
+ *   gathered   HOST array of n_gathered device pointers, each [s,b,h],
+ *              indexed by global row
+ *   mean, rstd [rows of the call] fp32 or NULL (mean not written for RMS)
+ * Its backward is sp_rs_norm_dropout_bwd with p_drop = 0, mask_bits = NULL,
+ * dY = NULL and dbias = NULL: the reduce-scatter of the upstream gradient
+ * partials, then the norm backward (plus dR_next) into dresidual_in.
+ */
+int sp_norm_all_gather_fwd(const sp_cfg* cfg, const void* x, const void* gamma,
+                           const void* beta, void* const* gathered,
+                           int32_t n_gathered, float* mean, float* rstd,
+                           void* stream);
+
+/*
  * All-gather of t sequence shards into n_out full [s,b,h] tensors.
  *
  * Defined by: "SP: Partition Activations Alongside TP", section "Change
@@ -222,7 +253,8 @@ int sp_all_gather(const sp_cfg* cfg, const void* const* shards,
  *   residual_out, mask_bits, mean, rstd   the forward's outputs (mask_bits
  *                may be NULL only when p_drop == 0; mean unused for RMS)
  *   gamma        [h]
- *   dresidual_in [s,b,h]; dY [s,b,h]
+ *   dresidual_in [s,b,h]; dY [s,b,h] or NULL (not written; the backward of
+ *                the entry into a TP region has no dropout input)
  *   dgamma [h] fp32; dbeta [h] fp32 or NULL; dbias [h] fp32 or NULL
  *   workspace    device scratch of at least sp_bwd_workspace_bytes() bytes,
  *                16-byte aligned; no initial contents needed

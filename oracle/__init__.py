@@ -86,6 +86,8 @@ def _lib():
         L.orc_fwd_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp, vp,
                                    vp, dp, dp]
         L.orc_fwd_rows.restype = ctypes.c_int
+        L.orc_norm_ag_fwd.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int, dp, dp]
+        L.orc_norm_ag_fwd.restype = ctypes.c_int
         L.orc_bwd.argtypes = [vp, vp, vp, vp, vp, vp, dp, dp, vp, vp, dp, dp,
                               dp]
         L.orc_bwd.restype = ctypes.c_int
@@ -273,6 +275,24 @@ def fwd_rows(cfg: Cfg, row_ids, part_rows, bias, residual_rows, gamma,
     if rc != 0:
         raise ValueError(f"oracle forward rejected the configuration ({rc})")
     return dict(residual_out=rout, norm_out=out, mask=mask,
+                mean=mean if cfg.norm == LAYERNORM else None, rstd=rstd)
+
+
+def norm_ag_fwd(cfg: Cfg, x, gamma, beta, n_out: int = 1) -> dict:
+    """Entry into a TP region: per-rank norm of x's shard, then all-gather."""
+    dt = cfg.dtype
+    tdt = _torch_dtype(dt)
+    x, gamma, beta = (_cpu(v, dt) for v in (x, gamma, beta))
+    N, h = cfg.s * cfg.b, cfg.h
+    gathered = [torch.empty((N, h), dtype=tdt) for _ in range(n_out)]
+    mean = np.zeros(N)
+    rstd = np.zeros(N)
+    rc = _lib().orc_norm_ag_fwd(ctypes.byref(cfg), _ptr(x), _ptr(gamma),
+                                _ptr(beta), _ptr_array(gathered), n_out,
+                                mean.ctypes.data, rstd.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle entry forward rejected the configuration ({rc})")
+    return dict(gathered=gathered,
                 mean=mean if cfg.norm == LAYERNORM else None, rstd=rstd)
 
 

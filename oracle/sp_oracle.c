@@ -359,6 +359,70 @@ int orc_fwd_rows(const orc_cfg* c, int64_t nrows, const int64_t* row_ids,
     return 0;
 }
 
+/*
+ * Entry into a tensor-parallel region ("SP: Partition Activations Alongside
+ * TP", section "Connect SP and TP across a layer": each GPU first normalizes
+ * its own tokens, then the all-gather combines the inputs of the QKV /
+ * first FFN linear).  Rank r normalises its rows of x; every requested
+ * replica receives all ranks' shards in order.  No reduction, bias, dropout
+ * or residual add: the SP region's sum was formed by the previous exit.
+ *   x         [s,b,h] in the I/O dtype, rank r's shard is its rows
+ *   gathered  n_out buffers [s,b,h];  mean/rstd [s*b] (mean NULL for RMS)
+ */
+int orc_norm_ag_fwd(const orc_cfg* c, const void* x, const void* gamma,
+                    const void* beta, void* const* gathered, int n_out,
+                    double* mean, double* rstd)
+{
+    if (!cfg_ok(c)) return -1;
+    const int64_t N = c->s * c->b, h = c->h, per = N / c->t;
+    double* full = (double*)malloc(sizeof(double) * (size_t)(N * h));
+    double** shards = (double**)malloc(sizeof(double*) * (size_t)c->t);
+    double* xr = (double*)malloc(sizeof(double) * (size_t)h);
+    if (!full || !shards || !xr) {
+        free(full); free(shards); free(xr);
+        return -2;
+    }
+    for (int r = 0; r < c->t; ++r) {
+        shards[r] = full + (int64_t)r * per * h;
+        for (int64_t i = 0; i < per; ++i) {
+            const int64_t n = (int64_t)r * per + i;
+            double* o = shards[r] + i * h;
+            for (int64_t j = 0; j < h; ++j) xr[j] = ld(x, n * h + j, c->dtype);
+            double mu = 0.0, var = 0.0, rs;
+            if (c->norm == ORC_LAYERNORM) {
+                for (int64_t j = 0; j < h; ++j) mu += xr[j];
+                mu /= (double)h;
+                for (int64_t j = 0; j < h; ++j) var += (xr[j] - mu) * (xr[j] - mu);
+                var /= (double)h;
+                rs = 1.0 / sqrt(var + (double)c->eps);
+                for (int64_t j = 0; j < h; ++j) {
+                    double b = beta ? ld(beta, j, c->dtype) : 0.0;
+                    o[j] = (xr[j] - mu) * rs * ld(gamma, j, c->dtype) + b;
+                }
+            } else {
+                double ms = 0.0;
+                for (int64_t j = 0; j < h; ++j) ms += xr[j] * xr[j];
+                ms /= (double)h;
+                rs = 1.0 / sqrt(ms + (double)c->eps);
+                for (int64_t j = 0; j < h; ++j)
+                    o[j] = xr[j] * rs * ld(gamma, j, c->dtype);
+            }
+            if (mean) mean[n] = mu;
+            if (rstd) rstd[n] = rs;
+        }
+    }
+    double* g = (double*)malloc(sizeof(double) * (size_t)(N * h));
+    if (!g) {
+        free(full); free(shards); free(xr);
+        return -2;
+    }
+    orc_all_gather(c->t, per, h, (const double* const*)shards, g);
+    for (int q = 0; q < n_out; ++q)
+        for (int64_t i = 0; i < N * h; ++i) st(gathered[q], i, c->dtype, g[i]);
+    free(g); free(full); free(shards); free(xr);
+    return 0;
+}
+
 /* ------------------------------------------------------------------------- */
 /* Backward                                                                   */
 /* ------------------------------------------------------------------------- */

@@ -33,7 +33,7 @@ EXPORTS = ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
            "sp_rs_norm_dropout_bwd", "sp_bwd_workspace_bytes",
            "sp_activation_bytes", "sp_status_string", "sp_device_error",
            "sp_debug_wait_timeout", "sp_plan_count",
-           "sp_rs_norm_dropout_bwd_noalloc")
+           "sp_rs_norm_dropout_bwd_noalloc", "sp_norm_all_gather_fwd")
 
 
 class SPError(RuntimeError):
@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
     lib.sp_rs_bias_dropout_add_norm_fwd.argtypes = [
         cfgp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
     lib.sp_all_gather.argtypes = [cfgp, vp, vp, i32, vp]
+    lib.sp_norm_all_gather_fwd.argtypes = [cfgp, vp, vp, vp, vp, i32, vp, vp,
+                                           vp]
     lib.sp_rs_norm_dropout_bwd.argtypes = [
         cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp,
         ctypes.c_size_t, vp]
@@ -139,6 +141,17 @@ def sp_rs_bias_dropout_add_norm_fwd(cfg: sp_cfg, partials, bias, residual,
                _p(gamma), _p(beta), _p(residual_out), _ptrs(gathered),
                len(gathered), _p(mask_bits), _p(mean), _p(rstd),
                _stream(stream, residual)))
+
+
+def sp_norm_all_gather_fwd(cfg: sp_cfg, x, gamma, beta, gathered, mean=None,
+                           rstd=None, stream=None) -> None:
+    """Entry into a TP region: per-token norm of x, all-gathered into every
+    tensor in ``gathered``."""
+    gathered = list(gathered)
+    _check("sp_norm_all_gather_fwd",
+           _lib.sp_norm_all_gather_fwd(
+               ctypes.byref(cfg), _p(x), _p(gamma), _p(beta), _ptrs(gathered),
+               len(gathered), _p(mean), _p(rstd), _stream(stream, x)))
 
 
 def sp_all_gather(cfg: sp_cfg, shards, outs, stream=None) -> None:

@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
                     dz[e] = ((kb[i] >> e) & 1u) ? dr[e] * a.scale : 0.f;
                 }
                 store_vec<T>(dres, v, IO<T>::pack(dr));
-                store_vec<T>(dy, v, IO<T>::pack(dz));
+                if (a.dY) store_vec<T>(dy, v, IO<T>::pack(dz));
                 if (a.want_dbias) {
                     if (ACC_SMEM) {
                         acc_add(2, v, dz);
@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
             uint32_t keep = 1u;
             if (a.mask) keep = (a.mask[(size_t)i_row * a.mask_row_bytes + (j >> 3)] >> (j & 7)) & 1u;
             const float dz = keep ? dr * a.scale : 0.f;
-            IO<T>::store1(a.dY, base + j, dz);
+            if (a.dY) IO<T>::store1(a.dY, base + j, dz);
             if (a.want_dbias) ws[2 * h + j] += dz;
         }
         __syncthreads();   // dns is rewritten by the next row

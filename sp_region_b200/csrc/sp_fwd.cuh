@@ -311,14 +311,15 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] += acc[i][e];
                     const Vec r = IO<T>::pack(f);
-                    store_vec<T>(rout, v, r);
+                    if (a.residual_out) store_vec<T>(rout, v, r);
                     IO<T>::unpack(r, acc[i]);
                 }
             }
         }
         release();
 
-        // per-token norm, two passes over the row held in registers
+        // per-token norm, two passes over the row held in registers (the
+        // two reductions use the group's two scratch buffers)
         float mean = 0.f, rstd;
         if (LN) {
             float s_ = 0.f;
@@ -411,7 +412,7 @@ __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ Fwd
             }
             if (keep) atomicOr(&mw[j >> 5], 1u << (j & 31));
             const float r = IO<T>::round1(IO<T>::load1(a.residual, lbase + j) + y);
-            IO<T>::store1(a.residual_out, lbase + j, r);
+            if (a.residual_out) IO<T>::store1(a.residual_out, lbase + j, r);
             xs[j] = r;
         }
         __syncthreads();

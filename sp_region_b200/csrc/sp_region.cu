@@ -122,6 +122,8 @@ constexpr Plan kFwdPlans[] = {
     {2, 3, 800, false},    // 9
     {4, 4, 544, false},    // 10
     {4, 6, 800, false},    // 11
+    {3, 3, 800, false},    // 12
+    {4, 4, 800, false},    // 13
 };
 constexpr Plan kBwdPlans[] = {
     {1, 1, 1024, false},   // 0
@@ -137,6 +139,8 @@ constexpr Plan kBwdPlans[] = {
     {4, 2, 800, true},     // 10
     {2, 3, 800, true},     // 11
     {4, 4, 544, true},     // 12
+    {3, 3, 800, true},     // 13
+    {4, 4, 800, true},     // 14
 };
 constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
 constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
@@ -145,8 +149,11 @@ constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
 // wins.  A hinted plan is tried first.
 // (measured on B200 for h = 4096 ... 12288: more rows in flight per SM wins
 // while the registers and the ring's stages allow it)
-constexpr int kFwdOrder[] = {10, 4, 9, 6, 8, 1, 2, 11, 0, 3, 5, 7};
-constexpr int kBwdOrder[] = {11, 8, 9, 12, 2, 3, 5, 10, 6, 1, 0, 4, 7};
+constexpr int kFwdOrder[] = {10, 4, 9, 6, 8, 1, 2, 11, 0, 3, 5, 7, 12, 13};
+// the entry into a TP region streams one segment per row, so its per-row
+// reductions dominate and more rows in flight per SM pay off first
+constexpr int kFwdEntryOrder[] = {13, 12, 11, 10, 4, 9, 6, 8, 1, 2, 0, 3, 5, 7};
+constexpr int kBwdOrder[] = {11, 8, 9, 12, 2, 3, 5, 10, 6, 1, 0, 4, 7, 13, 14};
 
 int group_threads(int hv, int V)
 {
@@ -172,7 +179,7 @@ const void* fwd_kernel(int id)
     switch (id) {
         SP_FWD_CASE(0) SP_FWD_CASE(1) SP_FWD_CASE(2) SP_FWD_CASE(3) SP_FWD_CASE(4)
         SP_FWD_CASE(5) SP_FWD_CASE(6) SP_FWD_CASE(7) SP_FWD_CASE(8) SP_FWD_CASE(9)
-        SP_FWD_CASE(10) SP_FWD_CASE(11)
+        SP_FWD_CASE(10) SP_FWD_CASE(11) SP_FWD_CASE(12) SP_FWD_CASE(13)
     }
     return nullptr;
 }
@@ -188,7 +195,7 @@ const void* bwd_kernel(int id)
     switch (id) {
         SP_BWD_CASE(0) SP_BWD_CASE(1) SP_BWD_CASE(2) SP_BWD_CASE(3) SP_BWD_CASE(4)
         SP_BWD_CASE(5) SP_BWD_CASE(6) SP_BWD_CASE(7) SP_BWD_CASE(8) SP_BWD_CASE(9)
-        SP_BWD_CASE(10) SP_BWD_CASE(11) SP_BWD_CASE(12)
+        SP_BWD_CASE(10) SP_BWD_CASE(11) SP_BWD_CASE(12) SP_BWD_CASE(13) SP_BWD_CASE(14)
     }
     return nullptr;
 }
@@ -240,7 +247,10 @@ FastLaunch plan_fwd(FwdArgs& a, const DevInfo& dev, int E, int hint)
     int order[1 + kNumFwdPlans];
     int no = 0;
     if (hint >= 1 && hint <= kNumFwdPlans) order[no++] = hint - 1;
-    for (int id : kFwdOrder) order[no++] = id;
+    if (a.t == 0)
+        for (int id : kFwdEntryOrder) order[no++] = id;
+    else
+        for (int id : kFwdOrder) order[no++] = id;
     for (int oi = 0; oi < no; ++oi) {
         const int id = order[oi];
         const Plan& p = kFwdPlans[id];
@@ -339,20 +349,27 @@ int sp_activation_bytes(int64_t s, int64_t b, int64_t h, int64_t a, int32_t t, i
     return SP_OK;
 }
 
-int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partials,
-                                    const void* bias, const void* residual, const void* gamma,
-                                    const void* beta, void* residual_out, void* const* gathered,
-                                    int32_t n_gathered, uint32_t* mask_bits, float* mean,
-                                    float* rstd, void* stream)
+}  // extern "C"
+
+namespace {
+
+// The forward with an explicit number of partial sums: cfg->t for the exit
+// of a tensor-parallel region, 0 for the entry into one (norm, then
+// all-gather; residual_out is then NULL and there is no dropout).
+int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const void* bias,
+             const void* residual, const void* gamma, const void* beta, void* residual_out,
+             void* const* gathered, int32_t n_gathered, uint32_t* mask_bits, float* mean,
+             float* rstd, void* stream)
 {
     int rc = check_cfg(cfg);
     if (rc) return rc;
-    if (!partials || !residual || !gamma || !residual_out || !gathered) return SP_ERR_INVALID_ARG;
+    if ((nparts > 0 && (!partials || !residual_out)) || !residual || !gamma || !gathered)
+        return SP_ERR_INVALID_ARG;
     if (n_gathered < 1 || n_gathered > SP_MAX_T) return SP_ERR_INVALID_ARG;
     const int E = elem_bytes(cfg);
     const bool ln = cfg->norm == SP_LAYERNORM;
     bool all16 = true;
-    for (int k = 0; k < cfg->t; ++k) {
+    for (int k = 0; k < nparts; ++k) {
         if (!partials[k] || !aligned(partials[k], E)) return SP_ERR_INVALID_ARG;
         all16 = all16 && aligned(partials[k], 16);
     }
@@ -377,7 +394,7 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
     const int h = (int)cfg->h;
     FwdArgs a;
     memset(&a, 0, sizeof(a));
-    for (int k = 0; k < cfg->t; ++k) a.parts[k] = partials[k];
+    for (int k = 0; k < nparts; ++k) a.parts[k] = partials[k];
     for (int q = 0; q < n_gathered; ++q) a.gathered[q] = gathered[q];
     a.bias = bias;
     a.residual = residual;
@@ -391,7 +408,7 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
     a.row0 = row0;
     a.h = h;
     a.hv = h / 8;
-    a.t = cfg->t;
+    a.t = nparts;
     a.n_gathered = n_gathered;
     a.seg_bytes = (uint32_t)(h * E);
     a.stage_stride = (uint32_t)round128(a.seg_bytes);
@@ -427,6 +444,32 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partia
         kern = ln ? (const void*)k_fwd_general<float, true>
                   : (const void*)k_fwd_general<float, false>;
     return launch_kernel(kern, grid, kGeneralThreads, smem, st, &a);
+}
+
+}  // namespace
+
+extern "C" {
+
+int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partials,
+                                    const void* bias, const void* residual, const void* gamma,
+                                    const void* beta, void* residual_out, void* const* gathered,
+                                    int32_t n_gathered, uint32_t* mask_bits, float* mean,
+                                    float* rstd, void* stream)
+{
+    if (!cfg) return SP_ERR_INVALID_ARG;
+    return fwd_impl(cfg, cfg->t, partials, bias, residual, gamma, beta, residual_out, gathered,
+                    n_gathered, mask_bits, mean, rstd, stream);
+}
+
+int sp_norm_all_gather_fwd(const sp_cfg* cfg, const void* x, const void* gamma,
+                           const void* beta, void* const* gathered, int32_t n_gathered,
+                           float* mean, float* rstd, void* stream)
+{
+    if (!cfg) return SP_ERR_INVALID_ARG;
+    sp_cfg c = *cfg;
+    c.p_drop = 0.0f;   // the entry has no dropout
+    return fwd_impl(&c, 0, nullptr, nullptr, x, gamma, beta, nullptr, gathered, n_gathered,
+                    nullptr, mean, rstd, stream);
 }
 
 int sp_all_gather(const sp_cfg* cfg, const void* const* shards, void* const* outs,
@@ -499,7 +542,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     int rc = check_cfg(cfg);
     if (rc) return rc;
     const bool ln = cfg->norm == SP_LAYERNORM;
-    if (!dn_partials || !residual_out || !gamma || !rstd || !dresidual_in || !dY || !dgamma ||
+    if (!dn_partials || !residual_out || !gamma || !rstd || !dresidual_in || !dgamma ||
         !workspace)
         return SP_ERR_INVALID_ARG;
     if (ln && !mean) return SP_ERR_INVALID_ARG;

@@ -32,7 +32,8 @@ MUTANTS = {
     "rounding ties away from zero": (
         "double r = nearbyint(scaled);", "double r = round(scaled);"),
     "unbiased variance": (
-        "var /= (double)h;", "var /= (double)(h - 1);"),
+        "var += (x[j] - mean) * (x[j] - mean);\n        var /= (double)h;",
+        "var += (x[j] - mean) * (x[j] - mean);\n        var /= (double)(h - 1);"),
     "eps outside the square root": (
         "rstd = 1.0 / sqrt(var + (double)c->eps);",
         "rstd = 1.0 / (sqrt(var) + (double)c->eps);"),
@@ -68,6 +69,12 @@ MUTANTS = {
     "norm reads the unrounded residual sum": (
         "        x[j] = r;\n",
         "        x[j] = ld(resid, rrow * h + j, c->dtype) + v;\n"),
+    "entry norm drops beta": (
+        "o[j] = (xr[j] - mu) * rs * ld(gamma, j, c->dtype) + b;",
+        "o[j] = (xr[j] - mu) * rs * ld(gamma, j, c->dtype) + 0 * b;"),
+    "entry norm uses the unbiased variance": (
+        "var += (xr[j] - mu) * (xr[j] - mu);\n                var /= (double)h;",
+        "var += (xr[j] - mu) * (xr[j] - mu);\n                var /= (double)(h - 1);"),
     "ring volume without (t-1)/t": (
         "double phase = (double)(t - 1) / (double)t * V;",
         "double phase = V;"),

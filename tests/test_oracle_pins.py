@@ -599,3 +599,34 @@ def test_activation_long_sequence_coefficients(orc):
     assert orc.activation_bytes(s, b, h, a, t, 0, 1.0) == 1314 * sbh
     assert orc.activation_bytes(s, b, h, a, t, 1, 1.0) == 91.5 * sbh
     assert orc.activation_bytes(s, b, h, a, t, 2, 1.0) == 82.125 * sbh
+
+
+# ----------------------------------------------------------------------------
+# entry into a TP region: norm of the shard, then all-gather
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+def test_entry_norm_matches_torch_and_gathers_in_rank_order(orc, norm):
+    """Each rank normalises its own tokens, then the shards are gathered in
+    rank order: the gathered tensor is the library norm of the whole x."""
+    w = sp_synth.WORKLOADS["C2"].replace(s=16, b=2, h=64, t=4, norm=norm,
+                                          dtype="f32")
+    cfg = orc.cfg_from(w)
+    x = sp_synth.draw_residual(w)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    beta = beta if norm == "layernorm" else None
+    out = orc.norm_ag_fwd(cfg, x, gamma, beta, n_out=2)
+    eps = float(np.float32(w.eps))
+    if norm == "layernorm":
+        ref = F.layer_norm(x.double(), (w.h,), gamma.double(), beta.double(),
+                           eps)
+    else:
+        ref = F.rms_norm(x.double(), (w.h,), gamma.double(), eps)
+    for q in range(2):
+        assert np.allclose(out["gathered"][q].double().numpy(), ref.numpy(),
+                           rtol=2 ** -23, atol=1e-30)
+    # the same as the exit's norm with nothing to reduce: zero partials, no
+    # bias, p = 0, the residual is x
+    fo = orc.fwd(orc.cfg_from(w, p_drop=0.0), [torch.zeros_like(x)] * w.t, None, x,
+                 gamma, beta)
+    assert torch.equal(fo["gathered"][0], out["gathered"][0])
