@@ -20,6 +20,7 @@ enum : unsigned {
     ERR_WAIT_FULL = 1,      // a consumer waited too long for a staged row
     ERR_WAIT_EMPTY = 2,     // the producer waited too long for a free stage
     ERR_DRAIN = 3,          // an aborted CTA could not drain its copies
+    ERR_WAIT_PEER = 4,      // a CTA waited too long for its cluster peer's sums
     ERR_SELFTEST = 9,       // the diagnostic wait of sp_debug_wait_timeout
 };
 
@@ -104,6 +105,96 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) {
+            *abort = 1;
+            record_error(code);
+            return false;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: a token row split across the CTAs of a cluster
+// exchanges its per-row partial sums through distributed shared memory.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_index()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_count()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+
+// Every thread of every CTA of the cluster (release / acquire at cluster
+// scope): orders the barrier initialisation before any remote access, and
+// keeps a CTA from exiting while a peer may still touch its shared memory.
+__device__ __forceinline__ void cluster_sync_all()
+{
+    asm volatile(
+        "barrier.cluster.arrive.release.aligned;\n\t"
+        "barrier.cluster.wait.acquire.aligned;" ::
+            : "memory");
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t local, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ void st_peer_f32x2(uint32_t addr, float x, float y)
+{
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y)
+                 : "memory");
+}
+
+// Arrive on an mbarrier in a peer CTA, releasing this thread's prior writes
+// (the value just stored there) at cluster scope.
+__device__ __forceinline__ void mbar_arrive_peer(uint32_t peer_bar)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(peer_bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire (for values a peer CTA released).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity,
+                                                  volatile int* abort, unsigned code)
+{
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (;;) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
             *abort = 1;
             record_error(code);
             return false;

@@ -68,6 +68,8 @@ struct RingTail {
     uint64_t full[64];
     uint64_t empty[64];
     uint64_t turn[2][kMaxGroups];   // backward: shared-accumulator turns
+    uint64_t xbar[2][kMaxGroups][2];   // cluster split: the peer's sums landed
+    float2 xslot[2][kMaxGroups][2];    // cluster split: the peer's sums
     float red[2][kMaxGroups][64];
     int abort;
 };
@@ -99,8 +101,16 @@ template <int G, typename SrcFn>
 __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail,
                                              volatile int* abort, long long rows,
                                              int nsrc, uint32_t seg_bytes,
-                                             uint32_t stage_stride, int S, SrcFn src)
+                                             uint32_t stage_stride, int S, SrcFn src,
+                                             long long first = -1, long long stride = 0,
+                                             uint32_t slice_off = 0)
 {
+    // rows first, first + stride, ... (default: this CTA's blockIdx rows);
+    // each copy moves seg_bytes starting slice_off bytes into the segment
+    if (first < 0) {
+        first = blockIdx.x;
+        stride = gridDim.x;
+    }
     const uint64_t pol = policy_evict_first();
     const int Sg = S / G;
     uint32_t stage[G], phase[G];
@@ -115,7 +125,7 @@ __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail
     for (long long jj = 0; ok; ++jj) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-            const long long i = blockIdx.x + (jj * G + g) * (long long)gridDim.x;
+            const long long i = first + (jj * G + g) * stride;
             if (!ok || i >= rows) {
                 ok = false;
                 break;
@@ -126,7 +136,7 @@ __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail
                     ok = false;
                     break;
                 }
-                const void* p = src(k, i);
+                const void* p = static_cast<const unsigned char*>(src(k, i)) + slice_off;
                 const uint32_t bar = smem_addr(&tail->full[st]);
                 mbar_arrive_expect_tx(bar, seg_bytes);
                 bulk_load(smem_addr(smem + (size_t)st * stage_stride), p, seg_bytes, bar, pol);
@@ -164,6 +174,7 @@ __device__ __forceinline__ void init_ring(RingTail* tail, int S, int warps_per_g
         for (int g = 0; g < kMaxGroups; ++g) {
             mbar_init(smem_addr(&tail->turn[0][g]), warps_per_group);
             mbar_init(smem_addr(&tail->turn[1][g]), warps_per_group);
+            for (int q = 0; q < 4; ++q) mbar_init(smem_addr(&tail->xbar[q >> 1][g][q & 1]), 1);
         }
         tail->abort = 0;
         mbar_init_fence();
@@ -175,14 +186,19 @@ __device__ __forceinline__ void init_ring(RingTail* tail, int S, int warps_per_g
 // groups of C threads (C <= (MAXT - 32) / G), each thread owning V vectors of
 // 8 features of a row, plus one producer warp; MAXT bounds the block size and
 // so sets the register budget.
-template <typename T, int V, int G, int MAXT, bool LN>
+// CS = 1: one CTA per token row.  CS = 2: each token row is split across the
+// two CTAs of a thread-block cluster (CTA rank r owns vectors
+// [r*hv/2, (r+1)*hv/2) of every row); the row's partial sums for mean and
+// variance are exchanged through distributed shared memory and added in rank
+// order, so both CTAs normalise with the same bits.
+template <typename T, int V, int G, int MAXT, bool LN, int CS = 1>
 __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ FwdArgs a)
 {
     using Vec = typename IO<T>::Vec;
     extern __shared__ __align__(128) unsigned char smem[];
     RingTail* tail = reinterpret_cast<RingTail*>(smem + a.tail_off);
     volatile int* abort = &tail->abort;
-    unsigned char* sg = smem + a.param_off;   // gamma, beta, bias copies
+    unsigned char* sg = smem + a.param_off;   // gamma, beta, bias copies (this slice)
     unsigned char* sb = sg + a.param_stride;
     unsigned char* sc = sb + a.param_stride;
 
@@ -190,12 +206,19 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
     const int tid = threadIdx.x;
     const int S = a.stages;                   // G sub-rings of S / G stages
     const int nsrc = a.t + 1;                 // t partials, then the residual
+    const uint32_t rank = CS > 1 ? cluster_rank() : 0u;
+    const long long cid = CS > 1 ? (long long)cluster_index() : (long long)blockIdx.x;
+    const long long ncl = CS > 1 ? (long long)cluster_count() : (long long)gridDim.x;
+    const int hvc = a.hv / CS;                // vectors of this CTA's slice
+    const int vg0 = (int)rank * hvc;          // first global vector of the slice
+    const uint32_t slice_bytes = a.seg_bytes / CS;
 
     init_ring(tail, S, C / 32);
+    if (CS > 1) cluster_sync_all();   // the peer's barriers exist before any remote arrive
 
     if (tid >= G * C) {
         if (tid == G * C)
-            ring_produce<G>(smem, tail, abort, a.rows, nsrc, a.seg_bytes, a.stage_stride, S,
+            ring_produce<G>(smem, tail, abort, a.rows, nsrc, slice_bytes, a.stage_stride, S,
                             [&](int k, long long i) -> const void* {
                                 // partial sums are indexed by global row, the
                                 // residual shard by local row
@@ -203,181 +226,196 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                                                      (size_t)(a.row0 + i) * a.seg_bytes
                                                : static_cast<const unsigned char*>(a.residual) +
                                                      (size_t)i * a.seg_bytes;
-                            });
-        return;
-    }
-
-    // consumers: group g handles every G-th row of this CTA; thread c of a
-    // group owns vectors v = c + i*C (8 features each)
-    const int g = tid / C;
-    const int c = tid - g * C;
-    const int lane = tid & 31;
-    const int bar_id = 1 + g;
-    if (g == 0) {
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int v = c + i * C;
-            if (v < a.hv) {
-                store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
-                if (a.beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));
-                if (a.bias) store_vec<T>(sc, v, load_vec<T>(a.bias, v));
-            }
-        }
-    }
-    // every group reads the copies group 0 wrote
-    asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
-
-    auto group_sum = [&](float x, float* red) {
-        x = warp_sum(x);
-        if (lane == 0) red[c >> 5] = x;
-        asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
-        return warps_total(red, C >> 5);
-    };
-
-    const uint32_t Sg = (uint32_t)(S / G);
-    RingPos pos((uint32_t)g * Sg, 0, Sg);
-    auto release = [&]() {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&tail->empty[pos.abs()]));
-        pos.next(Sg);
-    };
-    int parity = 0;
-    for (long long j = g;; j += G, parity ^= 1) {
-        const long long i_row = blockIdx.x + j * (long long)gridDim.x;   // local row
-        if (i_row >= a.rows) break;
-        const long long n = a.row0 + i_row;                                // global row
-
-        // reduce-scatter: sum of the t partial rows, k ascending, from +0
-        float acc[V][8];
-#pragma unroll
-        for (int i = 0; i < V; ++i)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
-        for (int k = 0; k < a.t; ++k) {
-            mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
-            const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
+                            },
+                            cid, ncl, rank * slice_bytes);
+    } else {
+        // consumers: group g handles every G-th row of this CTA (cluster);
+        // thread c of a group owns slice vectors v = c + i*C (8 features each)
+        const int g = tid / C;
+        const int c = tid - g * C;
+        const int lane = tid & 31;
+        const int bar_id = 1 + g;
+        if (g == 0) {
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
-                if (v < a.hv) {
-                    float f[8];
-                    IO<T>::unpack(load_vec<T>(buf, v), f);
+                if (v < hvc) {
+                    store_vec<T>(sg, v, load_vec<T>(a.gamma, vg0 + v));
+                    if (a.beta) store_vec<T>(sb, v, load_vec<T>(a.beta, vg0 + v));
+                    if (a.bias) store_vec<T>(sc, v, load_vec<T>(a.bias, vg0 + v));
+                }
+            }
+        }
+        // every group reads the copies group 0 wrote
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
+
+        int parity = 0, rcount = 0;
+        // sum over the row: this group's warps, then (CS = 2) the peer CTA
+        auto row_sum = [&](float x, float* red, int idx) {
+            x = warp_sum(x);
+            if (lane == 0) red[c >> 5] = x;
+            asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
+            const float local = warps_total(red, C >> 5);
+            if (CS == 1) return local;
+            const uint32_t slot = smem_addr(&tail->xslot[parity][g][idx]);
+            const uint32_t xb = smem_addr(&tail->xbar[parity][g][idx]);
+            if (c == 0) {
+                st_peer_f32x2(peer_addr(slot, rank ^ 1u), local, 0.f);
+                mbar_arrive_peer(peer_addr(xb, rank ^ 1u));
+            }
+            mbar_wait_cluster(xb, (uint32_t)((rcount >> 1) & 1), abort, ERR_WAIT_PEER);
+            const float other = tail->xslot[parity][g][idx].x;
+            return rank == 0 ? local + other : other + local;
+        };
+
+        const uint32_t Sg = (uint32_t)(S / G);
+        RingPos pos((uint32_t)g * Sg, 0, Sg);
+        auto release = [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->empty[pos.abs()]));
+            pos.next(Sg);
+        };
+        for (long long j = g;; j += G, parity ^= 1, ++rcount) {
+            const long long i_row = cid + j * ncl;              // local row
+            if (i_row >= a.rows) break;
+            const long long n = a.row0 + i_row;                  // global row
+
+            // reduce-scatter: sum of the t partial rows, k ascending, from +0
+            float acc[V][8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
+            for (int i = 0; i < V; ++i)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+            for (int k = 0; k < a.t; ++k) {
+                mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
+                const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int v = c + i * C;
+                    if (v < hvc) {
+                        float f[8];
+                        IO<T>::unpack(load_vec<T>(buf, v), f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
+                    }
+                }
+                release();
+            }
+
+            // bias once, then inverted dropout with the packed keep bits
+            uint8_t* mrow = a.mask ? a.mask + (size_t)i_row * a.mask_row_bytes : nullptr;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int v = c + i * C;
+                if (v < hvc) {
+                    if (a.bias) {
+                        float f[8];
+                        IO<T>::unpack(load_vec<T>(sc, v), f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
+                    }
+                    uint32_t kb = 0xFFu;
+                    if (a.dropout) {
+                        kb = keep_bits8((uint32_t)(vg0 + v), (uint32_t)n, a.off_lo, a.off_hi,
+                                        a.seed_lo, a.seed_hi, a.thr);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            acc[i][e] = ((kb >> e) & 1u) ? acc[i][e] * a.scale : 0.f;
+                    }
+                    if (mrow) mrow[vg0 + v] = (uint8_t)kb;
+                }
+            }
+            if (mrow && c == 0 && rank == 0)
+                for (int pbyte = a.hv; pbyte < a.mask_row_bytes; ++pbyte) mrow[pbyte] = 0;
+
+            // residual add; the sum is stored in the I/O dtype and the norm
+            // reads the stored (rounded) value
+            mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
+            {
+                const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
+                unsigned char* rout =
+                    static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.seg_bytes;
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int v = c + i * C;
+                    if (v < hvc) {
+                        float f[8];
+                        IO<T>::unpack(load_vec<T>(buf, v), f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] += acc[i][e];
+                        const Vec r = IO<T>::pack(f);
+                        if (a.residual_out) store_vec<T>(rout, vg0 + v, r);
+                        IO<T>::unpack(r, acc[i]);
+                    }
                 }
             }
             release();
-        }
 
-        // bias once, then inverted dropout with the packed keep bits
-        uint8_t* mrow = a.mask ? a.mask + (size_t)i_row * a.mask_row_bytes : nullptr;
+            // per-token norm, two passes over the row held in registers (the
+            // two reductions use the group's two scratch buffers)
+            float mean = 0.f, rstd;
+            if (LN) {
+                float s_ = 0.f;
 #pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int v = c + i * C;
-            if (v < a.hv) {
-                if (a.bias) {
-                    float f[8];
-                    IO<T>::unpack(load_vec<T>(sc, v), f);
+                for (int i = 0; i < V; ++i)
+                    if (c + i * C < hvc)
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
-                }
-                uint32_t kb = 0xFFu;
-                if (a.dropout) {
-                    kb = keep_bits8((uint32_t)v, (uint32_t)n, a.off_lo, a.off_hi, a.seed_lo,
-                                    a.seed_hi, a.thr);
+                        for (int e = 0; e < 8; ++e) s_ += acc[i][e];
+                mean = row_sum(s_, tail->red[0][g], 0) / a.h_f;
+                float q = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        acc[i][e] = ((kb >> e) & 1u) ? acc[i][e] * a.scale : 0.f;
-                }
-                if (mrow) mrow[v] = (uint8_t)kb;
+                for (int i = 0; i < V; ++i)
+                    if (c + i * C < hvc)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float d = acc[i][e] - mean;
+                            q += d * d;
+                        }
+                const float var = row_sum(q, tail->red[1][g], 1) / a.h_f;
+                rstd = 1.0f / sqrtf(var + a.eps);
+            } else {
+                float q = 0.f;
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    if (c + i * C < hvc)
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) q += acc[i][e] * acc[i][e];
+                const float ms = row_sum(q, tail->red[parity][g], 0) / a.h_f;
+                rstd = 1.0f / sqrtf(ms + a.eps);
             }
-        }
-        if (mrow && c == 0)
-            for (int pbyte = a.hv; pbyte < a.mask_row_bytes; ++pbyte) mrow[pbyte] = 0;
 
-        // residual add; the sum is stored in the I/O dtype and the norm reads
-        // the stored (rounded) value
-        mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
-        {
-            const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
-            unsigned char* rout =
-                static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.seg_bytes;
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
-                if (v < a.hv) {
-                    float f[8];
-                    IO<T>::unpack(load_vec<T>(buf, v), f);
+                if (v < hvc) {
+                    float gm[8], b[8], o[8];
+                    IO<T>::unpack(load_vec<T>(sg, v), gm);
+                    if (LN && a.beta) {
+                        IO<T>::unpack(load_vec<T>(sb, v), b);
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] += acc[i][e];
-                    const Vec r = IO<T>::pack(f);
-                    if (a.residual_out) store_vec<T>(rout, v, r);
-                    IO<T>::unpack(r, acc[i]);
-                }
-            }
-        }
-        release();
-
-        // per-token norm, two passes over the row held in registers (the
-        // two reductions use the group's two scratch buffers)
-        float mean = 0.f, rstd;
-        if (LN) {
-            float s_ = 0.f;
-#pragma unroll
-            for (int i = 0; i < V; ++i)
-                if (c + i * C < a.hv)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) s_ += acc[i][e];
-            mean = group_sum(s_, tail->red[0][g]) / a.h_f;
-            float q = 0.f;
-#pragma unroll
-            for (int i = 0; i < V; ++i)
-                if (c + i * C < a.hv)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float d = acc[i][e] - mean;
-                        q += d * d;
+                        for (int e = 0; e < 8; ++e) b[e] = 0.f;
                     }
-            const float var = group_sum(q, tail->red[1][g]) / a.h_f;
-            rstd = 1.0f / sqrtf(var + a.eps);
-        } else {
-            float q = 0.f;
 #pragma unroll
-            for (int i = 0; i < V; ++i)
-                if (c + i * C < a.hv)
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) q += acc[i][e] * acc[i][e];
-            const float ms = group_sum(q, tail->red[parity][g]) / a.h_f;
-            rstd = 1.0f / sqrtf(ms + a.eps);
-        }
-
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            const int v = c + i * C;
-            if (v < a.hv) {
-                float gm[8], b[8], o[8];
-                IO<T>::unpack(load_vec<T>(sg, v), gm);
-                if (LN && a.beta) {
-                    IO<T>::unpack(load_vec<T>(sb, v), b);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) b[e] = 0.f;
+                    for (int e = 0; e < 8; ++e)
+                        o[e] = LN ? (acc[i][e] - mean) * rstd * gm[e] + b[e]
+                                  : acc[i][e] * rstd * gm[e];
+                    const Vec ov = IO<T>::pack(o);
+                    for (int q = 0; q < a.n_gathered; ++q)
+                        store_vec<T>(static_cast<unsigned char*>(a.gathered[q]) +
+                                         (size_t)n * a.seg_bytes,
+                                     vg0 + v, ov);
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    o[e] = LN ? (acc[i][e] - mean) * rstd * gm[e] + b[e]
-                              : acc[i][e] * rstd * gm[e];
-                const Vec ov = IO<T>::pack(o);
-                for (int q = 0; q < a.n_gathered; ++q)
-                    store_vec<T>(static_cast<unsigned char*>(a.gathered[q]) +
-                                     (size_t)n * a.seg_bytes,
-                                 v, ov);
+            }
+            if (c == 0 && rank == 0) {
+                if (LN && a.mean) a.mean[i_row] = mean;
+                if (a.rstd) a.rstd[i_row] = rstd;
             }
         }
-        if (c == 0) {
-            if (LN && a.mean) a.mean[i_row] = mean;
-            if (a.rstd) a.rstd[i_row] = rstd;
-        }
+    }
+    if (CS > 1) {
+        __syncwarp();
+        cluster_sync_all();   // no CTA leaves while its peer may still write here
     }
 }
 

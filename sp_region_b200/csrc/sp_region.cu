@@ -107,52 +107,62 @@ long long general_grid(long long rows, int sms)
 struct Plan {
     int V, G, maxT;
     bool acc_smem;
+    int CS;   // CTAs per token row (a thread-block cluster when 2)
 };
 
 constexpr Plan kFwdPlans[] = {
-    {1, 1, 1024, false},   // 0
-    {1, 2, 800, false},    // 1
-    {1, 4, 1024, false},   // 2
-    {2, 1, 544, false},    // 3
-    {2, 2, 800, false},    // 4
-    {3, 1, 544, false},    // 5
-    {3, 2, 800, false},    // 6
-    {4, 1, 544, false},    // 7
-    {4, 2, 800, false},    // 8
-    {2, 3, 800, false},    // 9
-    {4, 4, 544, false},    // 10
-    {4, 6, 800, false},    // 11
-    {3, 3, 800, false},    // 12
-    {4, 4, 800, false},    // 13
+    {1, 1, 1024, false, 1},   // 0
+    {1, 2, 800, false, 1},    // 1
+    {1, 4, 1024, false, 1},   // 2
+    {2, 1, 544, false, 1},    // 3
+    {2, 2, 800, false, 1},    // 4
+    {3, 1, 544, false, 1},    // 5
+    {3, 2, 800, false, 1},    // 6
+    {4, 1, 544, false, 1},    // 7
+    {4, 2, 800, false, 1},    // 8
+    {2, 3, 800, false, 1},    // 9
+    {4, 4, 544, false, 1},    // 10
+    {4, 6, 800, false, 1},    // 11
+    {3, 3, 800, false, 1},    // 12
+    {4, 4, 800, false, 1},    // 13
+    {1, 2, 800, false, 2},    // 14
+    {2, 2, 800, false, 2},    // 15
+    {2, 1, 544, false, 2},    // 16
+    {1, 1, 1024, false, 2},   // 17
+    {4, 1, 544, false, 2},    // 18
 };
 constexpr Plan kBwdPlans[] = {
-    {1, 1, 1024, false},   // 0
-    {1, 1, 800, false},    // 1
-    {1, 2, 800, false},    // 2
-    {2, 1, 544, true},     // 3
-    {2, 1, 800, false},    // 4
-    {3, 1, 544, true},     // 5
-    {4, 1, 544, true},     // 6
-    {2, 1, 544, false},    // 7
-    {2, 2, 800, true},     // 8
-    {3, 2, 800, true},     // 9
-    {4, 2, 800, true},     // 10
-    {2, 3, 800, true},     // 11
-    {4, 4, 544, true},     // 12
-    {3, 3, 800, true},     // 13
-    {4, 4, 800, true},     // 14
+    {1, 1, 1024, false, 1},   // 0
+    {1, 1, 800, false, 1},    // 1
+    {1, 2, 800, false, 1},    // 2
+    {2, 1, 544, true, 1},     // 3
+    {2, 1, 800, false, 1},    // 4
+    {3, 1, 544, true, 1},     // 5
+    {4, 1, 544, true, 1},     // 6
+    {2, 1, 544, false, 1},    // 7
+    {2, 2, 800, true, 1},     // 8
+    {3, 2, 800, true, 1},     // 9
+    {4, 2, 800, true, 1},     // 10
+    {2, 3, 800, true, 1},     // 11
+    {4, 4, 544, true, 1},     // 12
+    {3, 3, 800, true, 1},     // 13
+    {4, 4, 800, true, 1},     // 14
 };
 constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
 constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
 
 // Preference order when the caller gives no hint: the first feasible plan
-// wins.  A hinted plan is tried first.
+// wins.  A hinted plan is tried first.  Plans that split a row across a
+// 2-CTA cluster come last: their per-row exchange of partial sums between
+// SMs costs more than it saves wherever a one-CTA plan fits, so they serve
+// rows too wide for one CTA (h > 16384 in bf16).
 // (measured on B200 for h = 4096 ... 12288: more rows in flight per SM wins
 // while the registers and the ring's stages allow it)
-constexpr int kFwdOrder[] = {10, 4, 9, 6, 8, 1, 2, 11, 0, 3, 5, 7, 12, 13};
+constexpr int kFwdOrder[] = {10, 4, 9, 6, 8, 1, 2, 11, 0, 3, 5, 7, 12, 13, 15, 14, 16, 17, 18};
 // the entry into a TP region streams one segment per row, so its per-row
 // reductions dominate and more rows in flight per SM pay off first
-constexpr int kFwdEntryOrder[] = {13, 12, 11, 10, 4, 9, 6, 8, 1, 2, 0, 3, 5, 7};
+constexpr int kFwdEntryOrder[] = {13, 12, 11, 10, 4, 9, 6, 8, 1, 2, 0, 3, 5, 7, 15, 14, 16,
+                                  17, 18};
 constexpr int kBwdOrder[] = {11, 8, 9, 12, 2, 3, 5, 10, 6, 1, 0, 4, 7, 13, 14};
 
 int group_threads(int hv, int V)
@@ -171,7 +181,7 @@ long long ring_stages(long long smem_optin, long long fixed, uint32_t stage_stri
 #define SP_FWD_CASE(ID)                                                                 \
     case ID:                                                                            \
         return (const void*)k_fwd_tma<T, kFwdPlans[ID].V, kFwdPlans[ID].G,              \
-                                      kFwdPlans[ID].maxT, LN>;
+                                      kFwdPlans[ID].maxT, LN, kFwdPlans[ID].CS>;
 
 template <typename T, bool LN>
 const void* fwd_kernel(int id)
@@ -179,7 +189,8 @@ const void* fwd_kernel(int id)
     switch (id) {
         SP_FWD_CASE(0) SP_FWD_CASE(1) SP_FWD_CASE(2) SP_FWD_CASE(3) SP_FWD_CASE(4)
         SP_FWD_CASE(5) SP_FWD_CASE(6) SP_FWD_CASE(7) SP_FWD_CASE(8) SP_FWD_CASE(9)
-        SP_FWD_CASE(10) SP_FWD_CASE(11) SP_FWD_CASE(12) SP_FWD_CASE(13)
+        SP_FWD_CASE(10) SP_FWD_CASE(11) SP_FWD_CASE(12) SP_FWD_CASE(13) SP_FWD_CASE(14)
+        SP_FWD_CASE(15) SP_FWD_CASE(16) SP_FWD_CASE(17) SP_FWD_CASE(18)
     }
     return nullptr;
 }
@@ -229,6 +240,47 @@ int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream
     return SP_OK;
 }
 
+// A persistent launch of clusters of `cs` CTAs: as many clusters as fit on
+// the device at once (at most `rows`), each CTA one SM.  *grid returns the
+// CTA count.
+int launch_clusters(const void* kern, long long rows, int cs, int block, size_t smem,
+                    cudaStream_t st, void* args, int* grid)
+{
+    if (!kern) return SP_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cfg.gridDim = dim3(cs);
+    int max_clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess ||
+        max_clusters < 1) {
+        cudaGetLastError();
+        return SP_ERR_UNSUPPORTED;
+    }
+    const long long ncl = rows < max_clusters ? rows : max_clusters;
+    cfg.gridDim = dim3((unsigned)(ncl * cs));
+    *grid = (int)(ncl * cs);
+    void* params[] = {args};
+    if (cudaLaunchKernelExC(&cfg, kern, params) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
+}
+
 // A fast launch: the chosen plan, its block and grid, and its dynamic shared
 // memory (the layout offsets are written into the kernel arguments).
 struct FastLaunch {
@@ -236,6 +288,7 @@ struct FastLaunch {
     int block = 0;
     int grid = 0;
     int groups = 1;
+    int cs = 1;
     size_t smem = 0;
 };
 
@@ -254,23 +307,29 @@ FastLaunch plan_fwd(FwdArgs& a, const DevInfo& dev, int E, int hint)
     for (int oi = 0; oi < no; ++oi) {
         const int id = order[oi];
         const Plan& p = kFwdPlans[id];
-        const int C = group_threads(a.hv, p.V);
+        if (a.hv % p.CS) continue;
+        const int C = group_threads(a.hv / p.CS, p.V);
         if (p.G * C + 32 > p.maxT) continue;
-        long long S = ring_stages(dev.smem_optin, (long long)(tailb + 3 * pstride),
-                                  a.stage_stride);
+        // each CTA stages and keeps parameters for its 1/CS of the row
+        const uint32_t stride = (uint32_t)round128(a.seg_bytes / p.CS);
+        const size_t pstride_c = round128((size_t)a.h * E / p.CS);
+        long long S = ring_stages(dev.smem_optin, (long long)(tailb + 3 * pstride_c), stride);
         S -= S % p.G;                 // G sub-rings of S / G stages each
         if (S < 2 * p.G) continue;
+        a.stage_stride = stride;
         a.stages = (int)S;
         a.param_off = (uint32_t)(S * a.stage_stride);
-        a.param_stride = (uint32_t)pstride;
-        a.tail_off = (uint32_t)(a.param_off + 3 * pstride);
+        a.param_stride = (uint32_t)pstride_c;
+        a.tail_off = (uint32_t)(a.param_off + 3 * pstride_c);
         L.plan = id;
         L.block = p.G * C + 32;
         L.grid = (int)(a.rows < dev.sms ? a.rows : dev.sms);
         L.groups = p.G;
+        L.cs = p.CS;
         L.smem = (size_t)a.tail_off + tailb;
         return L;
     }
+    (void)pstride;
     return L;
 }
 
@@ -286,6 +345,7 @@ FastLaunch plan_bwd(BwdArgs& a, const DevInfo& dev, int E, int hint)
     for (int oi = 0; oi < no; ++oi) {
         const int id = order[oi];
         const Plan& p = kBwdPlans[id];
+        if (p.CS != 1) continue;
         const int C = group_threads(a.hv, p.V);
         if (p.G * C + 32 > p.maxT) continue;
         const size_t accb = p.acc_smem ? (size_t)3 * 2 * a.hv * sizeof(float4) : 0;
@@ -429,6 +489,10 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
         if (L.plan >= 0) {
             const void* kern = ln ? fwd_kernel_dt<true>(cfg->dtype, L.plan)
                                   : fwd_kernel_dt<false>(cfg->dtype, L.plan);
+            if (L.cs > 1) {
+                int grid = 0;
+                return launch_clusters(kern, rows, L.cs, L.block, L.smem, st, &a, &grid);
+            }
             return launch_kernel(kern, L.grid, L.block, L.smem, st, &a);
         }
     }

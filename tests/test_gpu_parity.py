@@ -55,6 +55,7 @@ FWD_CASES = {
     "bf16_rms_h8192_t8_p0": dict(base="C3", s=304, b=1),
     "bf16_ln_h12288_t16_outliers": dict(base="C5", s=160, b=1),
     "bf16_ln_h16384_t2": dict(base="C2", s=64, b=1, h=16384, t=2),
+    "bf16_ln_h32768_cluster": dict(base="C2", s=80, b=2, h=32768, t=2),
     "bf16_ln_h4096_t4": dict(base="C4", s=300, b=2),
     "f32_ln_h512_t2": dict(base="C2", s=64, b=3, h=512, t=2, dtype="f32"),
     "f32_rms_h2048_t4": dict(base="C3", s=96, b=1, h=2048, t=4, dtype="f32"),
@@ -195,6 +196,7 @@ BWD_CASES = {
     "bf16_ln_no_dbias_dbeta": dict(base="C4", s=64, b=1, h=2048,
                                    no_param_grads=True),
     "bf16_ln_h16384_t2": dict(base="C2", s=64, b=1, h=16384, t=2),
+    "bf16_ln_h32768_cluster": dict(base="C2", s=80, b=2, h=32768, t=2),
     "bf16_t64_h64": dict(base="C2", s=128, b=1, h=64, t=64),
 }
 

@@ -26,6 +26,8 @@ SHAPES = {
     "h12288_t16": dict(base="C5", s=608, b=1, h=12288, t=16),
     "h8192_rms_t8": dict(base="C3", s=640, b=1, h=8192, t=8, p_drop=0.1,
                          has_bias=True),
+    # wider than any one-CTA plan: the forward splits rows across a cluster
+    "h24576_t2": dict(base="C2", s=320, b=1, h=24576, t=2),
 }
 
 
