@@ -124,6 +124,28 @@ def recorded_traffic(kernel_key):
 
 
 # ----------------------------------------------------------------------------
+# aggregation over ranks (N independent replicas)
+# ----------------------------------------------------------------------------
+
+def max_over_ranks(local_ms, device=None):
+    """The job's time is the slowest rank's: all-reduce MAX of the local
+    device-timed milliseconds (a no-op without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or \
+            dist.get_world_size() == 1:
+        return float(local_ms)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step, steps, world, max_ms):
+    """Whole-job GB/s: the bytes every rank processed over the job's time."""
+    return bytes_per_step * world * steps / (max_ms * 1e-3) / 1e9
+
+
+# ----------------------------------------------------------------------------
 # clocks during the timed region
 # ----------------------------------------------------------------------------
 
@@ -305,20 +327,16 @@ def run_ours(args):
     clocks.stop()
     assert sp.sp_device_error(local) == 0, "device-side wait timed out"
 
-    total_ms = e0.elapsed_time(e1)
     fwd_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
     bwd_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
-    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    total_ms = float(tmax.item())
+    total_ms = max_over_ranks(e0.elapsed_time(e1), dev)
 
     if args.op == "entry":
         fb, bb = entry_fwd_bytes(w), entry_bwd_bytes(w)
     else:
         fb, bb = fwd_bytes(w), bwd_bytes(w)
     step_bytes = fb + bb
-    value = step_bytes * world * K / (total_ms * 1e-3) / 1e9
+    value = job_throughput(step_bytes, K, world, total_ms)
     ms_step = total_ms / K
     peak, peak_src = measured_peak()
     f_avg = statistics.mean(fwd_ms)
@@ -507,13 +525,8 @@ def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
     down.wait_event(done_download[K - 1])
     e1.record(down)
     torch.cuda.synchronize(dev)
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        tm = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        ms = float(tm.item())
-    return {"value": round(step_bytes * world * K / (ms * 1e-3) / 1e9, 2),
+    ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    return {"value": round(job_throughput(step_bytes, K, world, ms), 2),
             "unit": "GB/s", "ms_per_step": round(ms / K, 3), "steps": K,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "path": "every step: pinned host -> device copies of all inputs, "
