@@ -14,12 +14,15 @@
 // partial rows, the x row and (optionally) the dR_next row into a ring of
 // shared-memory stages with cp.async.bulk; consumer threads own 8-feature
 // vectors.  The x stage is held while the row is processed (it is read twice)
-// so the row never sits in registers.  ACC_SMEM keeps the per-CTA parameter
-// gradient partials in shared memory when 3 * 8V fp32 registers per thread
-// would not fit.  With several consumer groups sharing that one set, the
-// groups take turns in the CTA's row order (two turn barriers, one for each
-// accumulating pass), so the sums keep a fixed order and stay bitwise
-// deterministic while the groups' reduce-scatter phases overlap.
+// so the row never sits in registers.  The per-thread parameter-gradient
+// partials (3 * 8V fp32) live in registers, in shared memory, or in tensor
+// memory.  Tensor memory (256 KB per SM, outside both the register file and
+// shared memory) is the default: it costs neither registers nor ring stages,
+// and each thread keeps its own set, so the sums have a fixed order per
+// consumer group.  With the shared-memory set, several consumer groups share
+// one set and take turns in the CTA's row order (two turn barriers, one for
+// each accumulating pass), so the sums stay bitwise deterministic while the
+// groups' reduce-scatter phases overlap.
 #pragma once
 
 #include "sp_device.cuh"
@@ -54,18 +57,27 @@ struct BwdArgs {
     float scale;
     int want_dbeta;
     int want_dbias;
+    uint32_t tmem_cols;      // tensor-memory columns allocated (ACC = 2)
 };
 
-template <typename T, int V, int G, int MAXT, bool LN, bool ACC_SMEM>
+// ACC: where the per-CTA parameter-gradient partials live.  0: registers,
+// one set per consumer group.  1: shared memory, one set per CTA that the
+// groups update by turns.  2: tensor memory, one private set per thread:
+// warp w uses the columns [(w / 4) * 24V, (w / 4 + 1) * 24V) of its lane
+// quarter, 24 columns per vector i (dgamma, dbeta, dbias; 8 each).
+template <typename T, int V, int G, int MAXT, bool LN, int ACC>
 __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ BwdArgs a)
 {
+    constexpr bool ACC_SMEM = ACC == 1;
+    constexpr bool ACC_TMEM = ACC == 2;
+    constexpr bool ACC_REGS = ACC == 0;
     using Vec = typename IO<T>::Vec;
     extern __shared__ __align__(128) unsigned char smem[];
     RingTail* tail = reinterpret_cast<RingTail*>(smem + a.tail_off);
     // gamma copy and, for ACC_SMEM, the per-CTA accumulators [3][2][hv][4]
     // fp32; every slot is private to the thread that owns its vector
     unsigned char* sgam = smem + a.param_off;
-    float4* accs = reinterpret_cast<float4*>(smem + a.acc_off);
+    ulonglong2* accs = reinterpret_cast<ulonglong2*>(smem + a.acc_off);
     volatile int* abort = &tail->abort;
 
     const int C = (blockDim.x - 32) / G;
@@ -73,6 +85,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
     const int S = a.stages;
     const int nsrc = a.t + 1 + (a.drnext ? 1 : 0);   // dP_k..., x, [dR_next]
 
+    if (ACC_TMEM && tid < 32) {
+        tmem_alloc(smem_addr(&tail->tmem_base), a.tmem_cols);
+        tmem_fence_before_sync();
+    }
     init_ring(tail, S, C / 32);
 
     if (tid >= G * C) {
@@ -96,32 +112,74 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
     const int lane = tid & 31;
     const int bar_id = 1 + g;
     const int hv = a.hv;
-    float ag[ACC_SMEM ? 1 : V][8], ab[ACC_SMEM ? 1 : V][8], ac[ACC_SMEM ? 1 : V][8];
+    // fp32 pairs throughout (features 2p, 2p+1 of a vector in pair p)
+    F2 ag[ACC_REGS ? V : 1][4], ab[ACC_REGS ? V : 1][4], ac[ACC_REGS ? V : 1][4];
+    uint32_t tacc = 0;   // this thread's first tensor-memory accumulator
+    if (ACC_TMEM) {
+        tmem_fence_after_sync();
+        const int w = tid >> 5;
+        tacc = tail->tmem_base + ((uint32_t)(32 * (w & 3)) << 16) + (uint32_t)((w >> 2) * 24 * V);
+        const uint32_t z[16] = {};
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            tmem_st16(tacc + 24 * i, z);
+            tmem_st8(tacc + 24 * i + 16, z);
+        }
+    }
 #pragma unroll
     for (int i = 0; i < V; ++i) {
         const int v = c + i * C;
         if (g == 0 && v < hv) store_vec<T>(sgam, v, load_vec<T>(a.gamma, v));
-        if (!ACC_SMEM) {
+        if (ACC_REGS) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ag[i][e] = ab[i][e] = ac[i][e] = 0.f;
-        } else if (v < hv) {
+            for (int p = 0; p < 4; ++p) ag[i][p] = ab[i][p] = ac[i][p] = f2(0.f);
+        } else if (ACC_SMEM && v < hv) {
 #pragma unroll
             for (int q = 0; q < 3; ++q) {
-                accs[((size_t)q * 2 + 0) * hv + v] = make_float4(0.f, 0.f, 0.f, 0.f);
-                accs[((size_t)q * 2 + 1) * hv + v] = make_float4(0.f, 0.f, 0.f, 0.f);
+                accs[((size_t)q * 2 + 0) * hv + v] = make_ulonglong2(0ull, 0ull);
+                accs[((size_t)q * 2 + 1) * hv + v] = make_ulonglong2(0ull, 0ull);
             }
         }
     }
     asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
 
-    auto acc_add = [&](int q, int v, const float d[8]) {
-        float4* p0 = &accs[((size_t)q * 2 + 0) * hv + v];
-        float4* p1 = &accs[((size_t)q * 2 + 1) * hv + v];
-        float4 x0 = *p0, x1 = *p1;
-        x0.x += d[0]; x0.y += d[1]; x0.z += d[2]; x0.w += d[3];
-        x1.x += d[4]; x1.y += d[5]; x1.z += d[6]; x1.w += d[7];
+    // accumulator q of vector v: pairs 0, 1 in the first 16 bytes, 2, 3 in
+    // the second ([3][2][hv] slots of 16 bytes)
+    auto acc_add = [&](int q, int v, const F2 d[4]) {
+        ulonglong2* p0 = &accs[((size_t)q * 2 + 0) * hv + v];
+        ulonglong2* p1 = &accs[((size_t)q * 2 + 1) * hv + v];
+        ulonglong2 x0 = *p0, x1 = *p1;
+        x0.x = add2(F2{x0.x}, d[0]).r;
+        x0.y = add2(F2{x0.y}, d[1]).r;
+        x1.x = add2(F2{x1.x}, d[2]).r;
+        x1.y = add2(F2{x1.y}, d[3]).r;
         *p0 = x0;
         *p1 = x1;
+    };
+    // add d0 (and d1) to the 8 (16) tensor-memory cells at column offset col
+    auto tmem_add8 = [&](uint32_t col, const F2 (&d0)[4]) {
+        uint32_t r[8];
+        tmem_ld8(tacc + col, r);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+            const float2 x =
+                halves(add2(f2(__uint_as_float(r[2 * p]), __uint_as_float(r[2 * p + 1])), d0[p]));
+            r[2 * p] = __float_as_uint(x.x);
+            r[2 * p + 1] = __float_as_uint(x.y);
+        }
+        tmem_st8(tacc + col, r);
+    };
+    auto tmem_add16 = [&](uint32_t col, const F2 (&d0)[4], const F2 (&d1)[4]) {
+        uint32_t r[16];
+        tmem_ld16(tacc + col, r);
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {
+            const float2 x = halves(add2(f2(__uint_as_float(r[2 * p]), __uint_as_float(r[2 * p + 1])),
+                                         p < 4 ? d0[p] : d1[p - 4]));
+            r[2 * p] = __float_as_uint(x.x);
+            r[2 * p + 1] = __float_as_uint(x.y);
+        }
+        tmem_st16(tacc + col, r);
     };
     auto release_at = [&](uint32_t s_) {
         __syncwarp();
@@ -147,6 +205,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         }
     };
 
+    const F2 scale2 = f2(a.scale);
     const uint32_t Sg = (uint32_t)(S / G);
     RingPos pos((uint32_t)g * Sg, 0, Sg);
     int parity = 0;
@@ -165,11 +224,11 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         }
 
         // reduce-scatter of the upstream gradient partials, k ascending, from +0
-        float dn[V][8];
+        F2 dn[V][4];
 #pragma unroll
         for (int i = 0; i < V; ++i)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) dn[i][e] = 0.f;
+            for (int p = 0; p < 4; ++p) dn[i][p] = f2(0.f);
         for (int k = 0; k < a.t; ++k) {
             mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
             const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
@@ -177,10 +236,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
                 if (v < hv) {
-                    float f[8];
-                    IO<T>::unpack(load_vec<T>(buf, v), f);
+                    F2 f[4];
+                    IO<T>::unpack2(load_vec<T>(buf, v), f);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) dn[i][e] += f[e];
+                    for (int p = 0; p < 4; ++p) dn[i][p] = add2(dn[i][p], f[p]);
                 }
             }
             release_at(pos.abs());
@@ -193,36 +252,52 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         const unsigned char* xb = smem + (size_t)sx * a.stage_stride;
         pos.next(Sg);
         take_turn(0, j);
-        float sg = 0.f, sgx = 0.f;
+        const F2 mean2 = f2(mean), rstd2 = f2(rstd);
+        auto xhat = [&](F2 xv) { return LN ? mul2(sub2(xv, mean2), rstd2) : mul2(xv, rstd2); };
+        F2 sg2 = f2(0.f), sgx2 = f2(0.f);
+        if (ACC_TMEM) {
+            __syncwarp();
+            tmem_wait_st();   // the previous row's updates have landed
+        }
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
+            F2 dgm[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
             if (v < hv) {
-                float xv[8], gm[8], dgm[8];
-                IO<T>::unpack(load_vec<T>(xb, v), xv);
-                IO<T>::unpack(load_vec<T>(sgam, v), gm);
+                F2 xv[4], gm[4];
+                IO<T>::unpack2(load_vec<T>(xb, v), xv);
+                IO<T>::unpack2(load_vec<T>(sgam, v), gm);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float xh = LN ? (xv[e] - mean) * rstd : xv[e] * rstd;
-                    const float gg = dn[i][e] * gm[e];
-                    sg += gg;
-                    sgx += gg * xh;
-                    dgm[e] = dn[i][e] * xh;
+                for (int p = 0; p < 4; ++p) {
+                    const F2 xh = xhat(xv[p]);
+                    const F2 gg = mul2(dn[i][p], gm[p]);
+                    sg2 = add2(sg2, gg);
+                    sgx2 = fma2(gg, xh, sgx2);
+                    dgm[p] = mul2(dn[i][p], xh);
                 }
                 if (ACC_SMEM) {
                     acc_add(0, v, dgm);
                     if (a.want_dbeta) acc_add(1, v, dn[i]);
-                } else {
+                } else if (ACC_REGS) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        ag[ACC_SMEM ? 0 : i][e] += dgm[e];
-                        ab[ACC_SMEM ? 0 : i][e] += dn[i][e];
+                    for (int p = 0; p < 4; ++p) {
+                        ag[ACC_REGS ? i : 0][p] = add2(ag[ACC_REGS ? i : 0][p], dgm[p]);
+                        ab[ACC_REGS ? i : 0][p] = add2(ab[ACC_REGS ? i : 0][p], dn[i][p]);
                     }
                 }
             }
+            // warp-wide, outside the per-thread branch; vectors past the row
+            // add zeros
+            if (ACC_TMEM) {
+                __syncwarp();
+                if (a.want_dbeta)
+                    tmem_add16(24 * i, dgm, dn[i]);
+                else
+                    tmem_add8(24 * i, dgm);
+            }
         }
         pass_turn(0);
-        float2 tot = make_float2(warp_sum(sg), warp_sum(sgx));
+        float2 tot = make_float2(warp_sum(hsum(sg2)), warp_sum(hsum(sgx2)));
         {
             float2* red = reinterpret_cast<float2*>(tail->red[parity][g]);
             if (lane == 0) red[c >> 5] = tot;
@@ -230,6 +305,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             tot = warps_total2(red, C >> 5);
         }
         const float mg = tot.x / a.h_f, mgx = tot.y / a.h_f;
+        const F2 mg2 = f2(mg), nmgx2 = f2(-mgx);
 
         const unsigned char* rb = nullptr;
         uint32_t sr = 0;
@@ -249,34 +325,44 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
+            F2 dz[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
             if (v < hv) {
-                float xv[8], gm[8], dr[8], dz[8], rn[8];
-                IO<T>::unpack(load_vec<T>(xb, v), xv);
-                IO<T>::unpack(load_vec<T>(sgam, v), gm);
+                F2 xv[4], gm[4], dr[4];
+                IO<T>::unpack2(load_vec<T>(xb, v), xv);
+                IO<T>::unpack2(load_vec<T>(sgam, v), gm);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const F2 xh = xhat(xv[p]);
+                    const F2 gg = mul2(dn[i][p], gm[p]);
+                    // rstd * (g - mean(g) - xhat * mean(g * xhat))
+                    const F2 u = fma2(xh, nmgx2, LN ? sub2(gg, mg2) : gg);
+                    dr[p] = mul2(rstd2, u);
+                }
                 if (rb) {
-                    IO<T>::unpack(load_vec<T>(rb, v), rn);
-                } else {
+                    F2 rn[4];
+                    IO<T>::unpack2(load_vec<T>(rb, v), rn);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) rn[e] = 0.f;
+                    for (int p = 0; p < 4; ++p) dr[p] = add2(dr[p], rn[p]);
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float xh = LN ? (xv[e] - mean) * rstd : xv[e] * rstd;
-                    const float gg = dn[i][e] * gm[e];
-                    const float dx = LN ? rstd * (gg - mg - xh * mgx) : rstd * (gg - xh * mgx);
-                    dr[e] = dx + rn[e];
-                    dz[e] = ((kb[i] >> e) & 1u) ? dr[e] * a.scale : 0.f;
-                }
-                store_vec<T>(dres, v, IO<T>::pack(dr));
-                if (a.dY) store_vec<T>(dy, v, IO<T>::pack(dz));
+                for (int p = 0; p < 4; ++p)
+                    dz[p] = keep2(mul2(dr[p], scale2), (kb[i] >> (2 * p)) & 1u,
+                                  (kb[i] >> (2 * p + 1)) & 1u);
+                store_vec<T>(dres, v, IO<T>::pack2v(dr));
+                if (a.dY) store_vec<T>(dy, v, IO<T>::pack2v(dz));
                 if (a.want_dbias) {
                     if (ACC_SMEM) {
                         acc_add(2, v, dz);
-                    } else {
+                    } else if (ACC_REGS) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) ac[ACC_SMEM ? 0 : i][e] += dz[e];
+                        for (int p = 0; p < 4; ++p)
+                            ac[ACC_REGS ? i : 0][p] = add2(ac[ACC_REGS ? i : 0][p], dz[p]);
                     }
                 }
+            }
+            if (ACC_TMEM && a.want_dbias) {
+                __syncwarp();
+                tmem_add8(24 * i + 16, dz);
             }
         }
         pass_turn(1);
@@ -291,27 +377,53 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         if (G > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
         if (g != 0) return;
     }
+    if (ACC_TMEM) {
+        __syncwarp();
+        tmem_wait_st();
+    }
     float* ws = a.ws + (ACC_SMEM ? (size_t)blockIdx.x : (size_t)blockIdx.x * G + g) * 3 * a.h;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
         const int v = c + i * C;
+        uint32_t tr[24];
+        if (ACC_TMEM) {   // warp-wide
+            __syncwarp();
+            tmem_ld16(tacc + 24 * i, tr);
+            tmem_ld8(tacc + 24 * i + 16, tr + 16);
+        }
         if (v < hv) {
             for (int q = 0; q < 3; ++q) {
-                float4 lo, hi;
+                ulonglong2 lo, hi;
                 if (ACC_SMEM) {
                     lo = accs[((size_t)q * 2 + 0) * hv + v];
                     hi = accs[((size_t)q * 2 + 1) * hv + v];
+                } else if (ACC_TMEM) {
+                    const uint32_t* r = tr + 8 * q;
+                    lo = make_ulonglong2(f2(__uint_as_float(r[0]), __uint_as_float(r[1])).r,
+                                         f2(__uint_as_float(r[2]), __uint_as_float(r[3])).r);
+                    hi = make_ulonglong2(f2(__uint_as_float(r[4]), __uint_as_float(r[5])).r,
+                                         f2(__uint_as_float(r[6]), __uint_as_float(r[7])).r);
                 } else {
-                    const float* s_ = q == 0 ? ag[ACC_SMEM ? 0 : i]
-                                             : (q == 1 ? ab[ACC_SMEM ? 0 : i]
-                                                       : ac[ACC_SMEM ? 0 : i]);
-                    lo = make_float4(s_[0], s_[1], s_[2], s_[3]);
-                    hi = make_float4(s_[4], s_[5], s_[6], s_[7]);
+                    const F2* s_ = q == 0 ? ag[ACC_REGS ? i : 0]
+                                          : (q == 1 ? ab[ACC_REGS ? i : 0]
+                                                    : ac[ACC_REGS ? i : 0]);
+                    lo = make_ulonglong2(s_[0].r, s_[1].r);
+                    hi = make_ulonglong2(s_[2].r, s_[3].r);
                 }
-                float4* dst = reinterpret_cast<float4*>(ws + (size_t)q * a.h + 8 * (size_t)v);
+                ulonglong2* dst = reinterpret_cast<ulonglong2*>(ws + (size_t)q * a.h + 8 * (size_t)v);
                 dst[0] = lo;
                 dst[1] = hi;
             }
+        }
+    }
+    if (ACC_TMEM) {
+        // every consumer thread is done with its columns before warp 0,
+        // which allocated them, gives them back
+        tmem_fence_before_sync();
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
+        if (tid < 32) {
+            tmem_fence_after_sync();
+            tmem_dealloc(tail->tmem_base, a.tmem_cols);
         }
     }
 }

@@ -223,6 +223,94 @@ __device__ __forceinline__ uint64_t policy_evict_first()
 }
 
 // ---------------------------------------------------------------------------
+// Tensor memory (PTX ISA: tcgen05.alloc / ld / st / wait / dealloc).  Each SM
+// has 128 lanes x 512 columns of 32-bit cells; an address is
+// (lane << 16) | column.  Warp w of a CTA may touch only lanes
+// [32 * (w % 4), 32 * (w % 4) + 32), one lane per thread.  The kernels here
+// use it as per-thread scratch that does not take shared memory or registers.
+// ---------------------------------------------------------------------------
+// one whole warp: allocate ncols columns (a power of 2 in [32, 512]) and
+// write the base address to shared memory; waits while the SM's tensor
+// memory is held by other CTAs
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(dst_smem), "r"(ncols) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+// the warp that allocated, once no thread touches the columns any more
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// order tensor-memory operations across a thread barrier
+__device__ __forceinline__ void tmem_fence_before_sync()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_fence_after_sync()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// this thread's earlier stores have landed (before the cells are read again)
+__device__ __forceinline__ void tmem_wait_st()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 8 / 16 consecutive columns of this thread's lane.  The load and its wait
+// are one statement, so no use of the registers can be scheduled before the
+// data has arrived.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t r[8])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t r[16])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t r[8])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+          "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t r[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+          "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+          "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As
 // Easy as 1, 2, 3", SC'11).  Each round multiplies counter words 0 and 2 by
 // the two Philox constants; the new words are (hi1 ^ w1 ^ k0, lo1,
@@ -232,15 +320,43 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 w, uint32_t k0, uint32_t k1
 {
 #pragma unroll
     for (int r = 0; r < 10; ++r) {
-        const uint32_t lo0 = 0xD2511F53u * w.x;
-        const uint32_t hi0 = __umulhi(0xD2511F53u, w.x);
-        const uint32_t lo1 = 0xCD9E8D57u * w.z;
-        const uint32_t hi1 = __umulhi(0xCD9E8D57u, w.z);
-        w = make_uint4(hi1 ^ w.y ^ k0, lo1, hi0 ^ w.w ^ k1, lo0);
+        // one widening multiply gives both halves of each 64-bit product
+        const unsigned long long p0 = (unsigned long long)w.x * 0xD2511F53u;
+        const unsigned long long p1 = (unsigned long long)w.z * 0xCD9E8D57u;
+        w = make_uint4((uint32_t)(p1 >> 32) ^ w.y ^ k0, (uint32_t)p1,
+                       (uint32_t)(p0 >> 32) ^ w.w ^ k1, (uint32_t)p0);
         k0 += 0x9E3779B9u;
         k1 += 0xBB67AE85u;
     }
     return w;
+}
+
+// The same rounds with the key schedule precomputed: ks[r] = (k0, k1) of
+// round r, identical for every thread of a launch, so the rounds read it from
+// the kernel's parameters instead of advancing it per call.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 w, const uint32_t (&ks)[10][2])
+{
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+        const unsigned long long p0 = (unsigned long long)w.x * 0xD2511F53u;
+        const unsigned long long p1 = (unsigned long long)w.z * 0xCD9E8D57u;
+        w = make_uint4((uint32_t)(p1 >> 32) ^ w.y ^ ks[r][0], (uint32_t)p1,
+                       (uint32_t)(p0 >> 32) ^ w.w ^ ks[r][1], (uint32_t)p0);
+    }
+    return w;
+}
+
+// Keep bits of the 8 features [8v, 8v+8) of token row n (scheduled keys).
+__device__ __forceinline__ uint32_t keep_bits8(uint32_t v, uint32_t n, uint32_t off_lo,
+                                               uint32_t off_hi, const uint32_t (&ks)[10][2],
+                                               uint32_t thr)
+{
+    const uint4 a = philox4x32_10(make_uint4(2u * v, n, off_lo, off_hi), ks);
+    const uint4 b = philox4x32_10(make_uint4(2u * v + 1u, n, off_lo, off_hi), ks);
+    return (uint32_t)(a.x >= thr) | (uint32_t)(a.y >= thr) << 1 |
+           (uint32_t)(a.z >= thr) << 2 | (uint32_t)(a.w >= thr) << 3 |
+           (uint32_t)(b.x >= thr) << 4 | (uint32_t)(b.y >= thr) << 5 |
+           (uint32_t)(b.z >= thr) << 6 | (uint32_t)(b.w >= thr) << 7;
 }
 
 // Keep bits of the 8 features [8v, 8v+8) of token row n: counter
@@ -269,8 +385,79 @@ __device__ __forceinline__ uint32_t keep_bit(uint32_t j, uint32_t n, uint32_t of
 }
 
 // ---------------------------------------------------------------------------
+// Two fp32 values in one 64-bit register.  sm_100a adds, subtracts,
+// multiplies and fuses a multiply-add on both halves in one instruction (PTX
+// add / sub / mul / fma .rn.f32x2); each half is rounded exactly as the scalar
+// operation would round it, so pairing changes the instruction count, not
+// the arithmetic.  .x is the lower feature of the pair.
+// ---------------------------------------------------------------------------
+struct F2 {
+    unsigned long long r;
+};
+
+__device__ __forceinline__ F2 f2(float lo, float hi)
+{
+    F2 v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v.r) : "f"(lo), "f"(hi));
+    return v;
+}
+
+__device__ __forceinline__ F2 f2(float x) { return f2(x, x); }
+
+__device__ __forceinline__ float2 halves(F2 v)
+{
+    float2 o;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(v.r));
+    return o;
+}
+
+__device__ __forceinline__ F2 add2(F2 a, F2 b)
+{
+    F2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
+
+__device__ __forceinline__ F2 sub2(F2 a, F2 b)
+{
+    F2 d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
+
+__device__ __forceinline__ F2 mul2(F2 a, F2 b)
+{
+    F2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
+
+// a * b + c with one rounding per half
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c)
+{
+    F2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.r) : "l"(a.r), "l"(b.r), "l"(c.r));
+    return d;
+}
+
+// halves kept where bits b0 / b1 are set, else +0
+__device__ __forceinline__ F2 keep2(F2 v, uint32_t b0, uint32_t b1)
+{
+    const float2 x = halves(v);
+    return f2(b0 ? x.x : 0.f, b1 ? x.y : 0.f);
+}
+
+// sum of the two halves
+__device__ __forceinline__ float hsum(F2 v)
+{
+    const float2 x = halves(v);
+    return x.x + x.y;
+}
+
+// ---------------------------------------------------------------------------
 // I/O dtype: 8 consecutive elements are one "vector" (16 B of bf16, 32 B of
-// fp32).  Arithmetic is always fp32; stores round to nearest-even.
+// fp32).  Arithmetic is always fp32; stores round to nearest-even.  unpack2 /
+// pack2v move a vector to and from four fp32 pairs.
 // ---------------------------------------------------------------------------
 template <typename T>
 struct IO;
@@ -296,6 +483,25 @@ struct IO<__nv_bfloat16> {
     {
         __nv_bfloat162 h = __floats2bfloat162_rn(a, b);   // .x (low half) = a
         return *reinterpret_cast<uint32_t*>(&h);
+    }
+    __device__ static __forceinline__ void unpack2(const Vec& v, F2 f[4])
+    {
+        const uint32_t w[4] = {v.u[0].x, v.u[0].y, v.u[0].z, v.u[0].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            f[i] = f2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+    }
+    __device__ static __forceinline__ Vec pack2v(const F2 f[4])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 x = halves(f[i]);
+            w[i] = pack2(x.x, x.y);
+        }
+        Vec v;
+        v.u[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        return v;
     }
     __device__ static __forceinline__ Vec pack(const float f[8])
     {
@@ -337,6 +543,25 @@ struct IO<float> {
         f[5] = __uint_as_float(v.u[1].y);
         f[6] = __uint_as_float(v.u[1].z);
         f[7] = __uint_as_float(v.u[1].w);
+    }
+    __device__ static __forceinline__ void unpack2(const Vec& v, F2 f[4])
+    {
+        f[0] = f2(__uint_as_float(v.u[0].x), __uint_as_float(v.u[0].y));
+        f[1] = f2(__uint_as_float(v.u[0].z), __uint_as_float(v.u[0].w));
+        f[2] = f2(__uint_as_float(v.u[1].x), __uint_as_float(v.u[1].y));
+        f[3] = f2(__uint_as_float(v.u[1].z), __uint_as_float(v.u[1].w));
+    }
+    __device__ static __forceinline__ Vec pack2v(const F2 f[4])
+    {
+        float2 x[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = halves(f[i]);
+        Vec v;
+        v.u[0] = make_uint4(__float_as_uint(x[0].x), __float_as_uint(x[0].y),
+                            __float_as_uint(x[1].x), __float_as_uint(x[1].y));
+        v.u[1] = make_uint4(__float_as_uint(x[2].x), __float_as_uint(x[2].y),
+                            __float_as_uint(x[3].x), __float_as_uint(x[3].y));
+        return v;
     }
     __device__ static __forceinline__ Vec pack(const float f[8])
     {

@@ -55,6 +55,7 @@ struct FwdArgs {
     float scale;            // 1 / (1 - p)
     uint32_t thr;           // floor(p * 2^32)
     uint32_t seed_lo, seed_hi, off_lo, off_hi;
+    uint32_t keys[10][2];   // Philox key (k0, k1) of each round, from the seed
     int dropout;            // p > 0
 };
 
@@ -72,6 +73,7 @@ struct RingTail {
     float2 xslot[2][kMaxGroups][2];    // cluster split: the peer's sums
     float red[2][kMaxGroups][64];
     int abort;
+    uint32_t tmem_base;   // backward, tensor-memory accumulators: allocated base
 };
 
 // Position in a sub-ring of Sg stages starting at stage `base`: the i-th
@@ -275,17 +277,19 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
             if (lane == 0) mbar_arrive(smem_addr(&tail->empty[pos.abs()]));
             pos.next(Sg);
         };
+        const F2 scale2 = f2(a.scale);
         for (long long j = g;; j += G, parity ^= 1, ++rcount) {
             const long long i_row = cid + j * ncl;              // local row
             if (i_row >= a.rows) break;
             const long long n = a.row0 + i_row;                  // global row
 
-            // reduce-scatter: sum of the t partial rows, k ascending, from +0
-            float acc[V][8];
+            // reduce-scatter: sum of the t partial rows, k ascending, from +0;
+            // fp32 pairs throughout (features 2p, 2p+1 of a vector in pair p)
+            F2 acc[V][4];
 #pragma unroll
             for (int i = 0; i < V; ++i)
 #pragma unroll
-                for (int e = 0; e < 8; ++e) acc[i][e] = 0.f;
+                for (int p = 0; p < 4; ++p) acc[i][p] = f2(0.f);
             for (int k = 0; k < a.t; ++k) {
                 mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
@@ -293,10 +297,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 for (int i = 0; i < V; ++i) {
                     const int v = c + i * C;
                     if (v < hvc) {
-                        float f[8];
-                        IO<T>::unpack(load_vec<T>(buf, v), f);
+                        F2 f[4];
+                        IO<T>::unpack2(load_vec<T>(buf, v), f);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
+                        for (int p = 0; p < 4; ++p) acc[i][p] = add2(acc[i][p], f[p]);
                     }
                 }
                 release();
@@ -309,18 +313,19 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 const int v = c + i * C;
                 if (v < hvc) {
                     if (a.bias) {
-                        float f[8];
-                        IO<T>::unpack(load_vec<T>(sc, v), f);
+                        F2 f[4];
+                        IO<T>::unpack2(load_vec<T>(sc, v), f);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc[i][e] += f[e];
+                        for (int p = 0; p < 4; ++p) acc[i][p] = add2(acc[i][p], f[p]);
                     }
                     uint32_t kb = 0xFFu;
                     if (a.dropout) {
                         kb = keep_bits8((uint32_t)(vg0 + v), (uint32_t)n, a.off_lo, a.off_hi,
-                                        a.seed_lo, a.seed_hi, a.thr);
+                                        a.keys, a.thr);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            acc[i][e] = ((kb >> e) & 1u) ? acc[i][e] * a.scale : 0.f;
+                        for (int p = 0; p < 4; ++p)
+                            acc[i][p] = keep2(mul2(acc[i][p], scale2), (kb >> (2 * p)) & 1u,
+                                              (kb >> (2 * p + 1)) & 1u);
                     }
                     if (mrow) mrow[vg0 + v] = (uint8_t)kb;
                 }
@@ -339,13 +344,13 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 for (int i = 0; i < V; ++i) {
                     const int v = c + i * C;
                     if (v < hvc) {
-                        float f[8];
-                        IO<T>::unpack(load_vec<T>(buf, v), f);
+                        F2 f[4];
+                        IO<T>::unpack2(load_vec<T>(buf, v), f);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] += acc[i][e];
-                        const Vec r = IO<T>::pack(f);
+                        for (int p = 0; p < 4; ++p) f[p] = add2(f[p], acc[i][p]);
+                        const Vec r = IO<T>::pack2v(f);
                         if (a.residual_out) store_vec<T>(rout, vg0 + v, r);
-                        IO<T>::unpack(r, acc[i]);
+                        IO<T>::unpack2(r, acc[i]);
                     }
                 }
             }
@@ -355,52 +360,56 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
             // two reductions use the group's two scratch buffers)
             float mean = 0.f, rstd;
             if (LN) {
-                float s_ = 0.f;
+                F2 s2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i)
                     if (c + i * C < hvc)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) s_ += acc[i][e];
-                mean = row_sum(s_, tail->red[0][g], 0) / a.h_f;
-                float q = 0.f;
+                        for (int p = 0; p < 4; ++p) s2 = add2(s2, acc[i][p]);
+                mean = row_sum(hsum(s2), tail->red[0][g], 0) / a.h_f;
+                const F2 mean2 = f2(mean);
+                F2 q2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i)
                     if (c + i * C < hvc)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float d = acc[i][e] - mean;
-                            q += d * d;
+                        for (int p = 0; p < 4; ++p) {
+                            const F2 d = sub2(acc[i][p], mean2);
+                            q2 = fma2(d, d, q2);
                         }
-                const float var = row_sum(q, tail->red[1][g], 1) / a.h_f;
+                const float var = row_sum(hsum(q2), tail->red[1][g], 1) / a.h_f;
                 rstd = 1.0f / sqrtf(var + a.eps);
             } else {
-                float q = 0.f;
+                F2 q2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i)
                     if (c + i * C < hvc)
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) q += acc[i][e] * acc[i][e];
-                const float ms = row_sum(q, tail->red[parity][g], 0) / a.h_f;
+                        for (int p = 0; p < 4; ++p) q2 = fma2(acc[i][p], acc[i][p], q2);
+                const float ms = row_sum(hsum(q2), tail->red[parity][g], 0) / a.h_f;
                 rstd = 1.0f / sqrtf(ms + a.eps);
             }
 
+            const F2 mean2 = f2(mean), rstd2 = f2(rstd);
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
                 if (v < hvc) {
-                    float gm[8], b[8], o[8];
-                    IO<T>::unpack(load_vec<T>(sg, v), gm);
+                    F2 gm[4], o[4];
+                    IO<T>::unpack2(load_vec<T>(sg, v), gm);
                     if (LN && a.beta) {
-                        IO<T>::unpack(load_vec<T>(sb, v), b);
+                        F2 b[4];
+                        IO<T>::unpack2(load_vec<T>(sb, v), b);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p)
+                            o[p] = fma2(mul2(sub2(acc[i][p], mean2), rstd2), gm[p], b[p]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) b[e] = 0.f;
+                        for (int p = 0; p < 4; ++p)
+                            o[p] = mul2(mul2(LN ? sub2(acc[i][p], mean2) : acc[i][p], rstd2),
+                                        gm[p]);
                     }
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        o[e] = LN ? (acc[i][e] - mean) * rstd * gm[e] + b[e]
-                                  : acc[i][e] * rstd * gm[e];
-                    const Vec ov = IO<T>::pack(o);
+                    const Vec ov = IO<T>::pack2v(o);
                     for (int q = 0; q < a.n_gathered; ++q)
                         store_vec<T>(static_cast<unsigned char*>(a.gathered[q]) +
                                          (size_t)n * a.seg_bytes,

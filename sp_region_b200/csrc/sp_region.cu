@@ -106,47 +106,55 @@ long long general_grid(long long rows, int sms)
 // ---------------------------------------------------------------------------
 struct Plan {
     int V, G, maxT;
-    bool acc_smem;
+    int acc;   // backward parameter-gradient partials: 0 registers, 1 shared, 2 tensor memory
     int CS;   // CTAs per token row (a thread-block cluster when 2)
 };
 
 constexpr Plan kFwdPlans[] = {
-    {1, 1, 1024, false, 1},   // 0
-    {1, 2, 800, false, 1},    // 1
-    {1, 4, 1024, false, 1},   // 2
-    {2, 1, 544, false, 1},    // 3
-    {2, 2, 800, false, 1},    // 4
-    {3, 1, 544, false, 1},    // 5
-    {3, 2, 800, false, 1},    // 6
-    {4, 1, 544, false, 1},    // 7
-    {4, 2, 800, false, 1},    // 8
-    {2, 3, 800, false, 1},    // 9
-    {4, 4, 544, false, 1},    // 10
-    {4, 6, 800, false, 1},    // 11
-    {3, 3, 800, false, 1},    // 12
-    {4, 4, 800, false, 1},    // 13
-    {1, 2, 800, false, 2},    // 14
-    {2, 2, 800, false, 2},    // 15
-    {2, 1, 544, false, 2},    // 16
-    {1, 1, 1024, false, 2},   // 17
-    {4, 1, 544, false, 2},    // 18
+    {1, 1, 1024, 0, 1},   // 0
+    {1, 2, 800, 0, 1},    // 1
+    {1, 4, 1024, 0, 1},   // 2
+    {2, 1, 544, 0, 1},    // 3
+    {2, 2, 800, 0, 1},    // 4
+    {3, 1, 544, 0, 1},    // 5
+    {3, 2, 800, 0, 1},    // 6
+    {4, 1, 544, 0, 1},    // 7
+    {4, 2, 800, 0, 1},    // 8
+    {2, 3, 800, 0, 1},    // 9
+    {4, 4, 544, 0, 1},    // 10
+    {4, 6, 800, 0, 1},    // 11
+    {3, 3, 800, 0, 1},    // 12
+    {4, 4, 800, 0, 1},    // 13
+    {1, 2, 800, 0, 2},    // 14
+    {2, 2, 800, 0, 2},    // 15
+    {2, 1, 544, 0, 2},    // 16
+    {1, 1, 1024, 0, 2},   // 17
+    {4, 1, 544, 0, 2},    // 18
 };
 constexpr Plan kBwdPlans[] = {
-    {1, 1, 1024, false, 1},   // 0
-    {1, 1, 800, false, 1},    // 1
-    {1, 2, 800, false, 1},    // 2
-    {2, 1, 544, true, 1},     // 3
-    {2, 1, 800, false, 1},    // 4
-    {3, 1, 544, true, 1},     // 5
-    {4, 1, 544, true, 1},     // 6
-    {2, 1, 544, false, 1},    // 7
-    {2, 2, 800, true, 1},     // 8
-    {3, 2, 800, true, 1},     // 9
-    {4, 2, 800, true, 1},     // 10
-    {2, 3, 800, true, 1},     // 11
-    {4, 4, 544, true, 1},     // 12
-    {3, 3, 800, true, 1},     // 13
-    {4, 4, 800, true, 1},     // 14
+    {1, 1, 1024, 0, 1},   // 0
+    {1, 1, 800, 0, 1},    // 1
+    {1, 2, 800, 0, 1},    // 2
+    {2, 1, 544, 1, 1},     // 3
+    {2, 1, 800, 0, 1},    // 4
+    {3, 1, 544, 1, 1},     // 5
+    {4, 1, 544, 1, 1},     // 6
+    {2, 1, 544, 0, 1},    // 7
+    {2, 2, 800, 1, 1},     // 8
+    {3, 2, 800, 1, 1},     // 9
+    {4, 2, 800, 1, 1},     // 10
+    {2, 3, 800, 1, 1},     // 11
+    {4, 4, 544, 1, 1},     // 12
+    {3, 3, 800, 1, 1},     // 13
+    {4, 4, 800, 1, 1},     // 14
+    {2, 2, 800, 2, 1},        // 15
+    {3, 2, 800, 2, 1},        // 16
+    {3, 1, 544, 2, 1},        // 17
+    {2, 1, 800, 2, 1},        // 18
+    {4, 4, 544, 2, 1},        // 19
+    {2, 3, 800, 2, 1},        // 20
+    {4, 1, 544, 2, 1},        // 21
+    {2, 1, 544, 2, 1},        // 22
 };
 constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
 constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
@@ -163,7 +171,11 @@ constexpr int kFwdOrder[] = {10, 4, 9, 6, 8, 1, 2, 11, 0, 3, 5, 7, 12, 13, 15, 1
 // reductions dominate and more rows in flight per SM pay off first
 constexpr int kFwdEntryOrder[] = {13, 12, 11, 10, 4, 9, 6, 8, 1, 2, 0, 3, 5, 7, 15, 14, 16,
                                   17, 18};
-constexpr int kBwdOrder[] = {11, 8, 9, 12, 2, 3, 5, 10, 6, 1, 0, 4, 7, 13, 14};
+// backward: tensor-memory accumulators first; they leave shared memory to the
+// ring (measured on B200 for bf16 rows of h = 12288, t = 16: 2 -> 8 stages,
+// 4.9 -> 6.6 TB/s)
+constexpr int kBwdOrder[] = {19, 15, 16, 18, 17, 21, 20, 22, 11, 8, 9, 12,
+                             2, 3, 5, 10, 6, 1, 0, 4, 7, 13, 14};
 
 int group_threads(int hv, int V)
 {
@@ -198,7 +210,7 @@ const void* fwd_kernel(int id)
 #define SP_BWD_CASE(ID)                                                                 \
     case ID:                                                                            \
         return (const void*)k_bwd_tma<T, kBwdPlans[ID].V, kBwdPlans[ID].G,              \
-                                      kBwdPlans[ID].maxT, LN, kBwdPlans[ID].acc_smem>;
+                                      kBwdPlans[ID].maxT, LN, kBwdPlans[ID].acc>;
 
 template <typename T, bool LN>
 const void* bwd_kernel(int id)
@@ -207,6 +219,8 @@ const void* bwd_kernel(int id)
         SP_BWD_CASE(0) SP_BWD_CASE(1) SP_BWD_CASE(2) SP_BWD_CASE(3) SP_BWD_CASE(4)
         SP_BWD_CASE(5) SP_BWD_CASE(6) SP_BWD_CASE(7) SP_BWD_CASE(8) SP_BWD_CASE(9)
         SP_BWD_CASE(10) SP_BWD_CASE(11) SP_BWD_CASE(12) SP_BWD_CASE(13) SP_BWD_CASE(14)
+        SP_BWD_CASE(15) SP_BWD_CASE(16) SP_BWD_CASE(17) SP_BWD_CASE(18) SP_BWD_CASE(19)
+        SP_BWD_CASE(20) SP_BWD_CASE(21) SP_BWD_CASE(22)
     }
     return nullptr;
 }
@@ -348,12 +362,23 @@ FastLaunch plan_bwd(BwdArgs& a, const DevInfo& dev, int E, int hint)
         if (p.CS != 1) continue;
         const int C = group_threads(a.hv, p.V);
         if (p.G * C + 32 > p.maxT) continue;
-        const size_t accb = p.acc_smem ? (size_t)3 * 2 * a.hv * sizeof(float4) : 0;
+        uint32_t tcols = 0;
+        if (p.acc == 2) {
+            // 24 columns per vector for each warp; the warps of a lane
+            // quarter sit side by side; allocations are powers of 2 >= 32
+            const int per_quarter = ((p.G * C / 32) + 3) / 4;
+            const int need = per_quarter * 24 * p.V;
+            if (need > 512) continue;
+            tcols = 32;
+            while ((int)tcols < need) tcols <<= 1;
+        }
+        const size_t accb = p.acc == 1 ? (size_t)3 * 2 * a.hv * sizeof(float4) : 0;
         long long S = ring_stages(dev.smem_optin, (long long)(tailb + pstride + accb),
                                   a.stage_stride);
         S -= S % p.G;                 // G sub-rings of S / G stages each
         if (S < 2 * p.G) continue;
         a.stages = (int)S;
+        a.tmem_cols = tcols;
         a.param_off = (uint32_t)(S * a.stage_stride);
         a.acc_off = (uint32_t)(a.param_off + pstride);
         a.tail_off = (uint32_t)(a.acc_off + accb);
@@ -481,6 +506,10 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
     a.seed_hi = (uint32_t)(cfg->seed >> 32);
     a.off_lo = (uint32_t)cfg->offset;
     a.off_hi = (uint32_t)(cfg->offset >> 32);
+    for (int r = 0; r < 10; ++r) {   // Philox key schedule: Weyl increments per round
+        a.keys[r][0] = a.seed_lo + (uint32_t)r * 0x9E3779B9u;
+        a.keys[r][1] = a.seed_hi + (uint32_t)r * 0xBB67AE85u;
+    }
     a.dropout = cfg->p_drop > 0.0f ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
 
@@ -664,7 +693,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     if (h % 8 == 0 && all16) {
         const FastLaunch L = plan_bwd(a, dev, E, cfg->bwd_plan);
         if (L.plan >= 0) {
-            nparts = (long long)L.grid * (kBwdPlans[L.plan].acc_smem ? 1 : L.groups);
+            nparts = (long long)L.grid * (kBwdPlans[L.plan].acc == 1 ? 1 : L.groups);
             if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes)
                 return SP_ERR_INVALID_ARG;
             const void* kern = ln ? bwd_kernel_dt<true>(cfg->dtype, L.plan)
