@@ -53,7 +53,7 @@ struct BwdArgs {
     uint32_t param_off;      // shared-memory offsets (fast kernel): gamma copy,
     uint32_t acc_off;        //   parameter-gradient accumulators (ACC_SMEM),
     uint32_t tail_off;       //   barriers / scratch
-    float h_f;
+    float inv_h;             // 1 / h, rounded to fp32
     float scale;
     int want_dbeta;
     int want_dbias;
@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(C) : "memory");
             tot = warps_total2(red, C >> 5);
         }
-        const float mg = tot.x / a.h_f, mgx = tot.y / a.h_f;
+        const float mg = tot.x * a.inv_h, mgx = tot.y * a.inv_h;
         const F2 mg2 = f2(mg), nmgx2 = f2(-mgx);
 
         const unsigned char* rb = nullptr;
@@ -461,8 +461,8 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
             ws[j] += d * xh;
             if (a.want_dbeta) ws[h + j] += d;
         }
-        const float mg = block_sum(sg, red) / a.h_f;
-        const float mgx = block_sum(sgx, red) / a.h_f;
+        const float mg = block_sum(sg, red) * a.inv_h;
+        const float mgx = block_sum(sgx, red) * a.inv_h;
         for (int j = threadIdx.x; j < h; j += blockDim.x) {
             const float d = dns[j];
             const float xv = IO<T>::load1(a.x, lbase + j);

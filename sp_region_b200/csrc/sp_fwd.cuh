@@ -51,7 +51,7 @@ struct FwdArgs {
     uint32_t param_stride;  //   one slot of param_stride bytes each,
     uint32_t tail_off;      //   then the barriers / scratch
     float eps;
-    float h_f;
+    float inv_h;            // 1 / h, rounded to fp32
     float scale;            // 1 / (1 - p)
     uint32_t thr;           // floor(p * 2^32)
     uint32_t seed_lo, seed_hi, off_lo, off_hi;
@@ -284,12 +284,17 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
             const long long n = a.row0 + i_row;                  // global row
 
             // reduce-scatter: sum of the t partial rows, k ascending, from +0;
-            // fp32 pairs throughout (features 2p, 2p+1 of a vector in pair p)
+            // fp32 pairs throughout (features 2p, 2p+1 of a vector in pair p).
+            // With no partial sums, bias, dropout or stored sum (the entry into
+            // a TP region) the row is the input itself, already in the I/O dtype.
             F2 acc[V][4];
+            const bool direct = a.t == 0 && !a.bias && !a.dropout && !a.residual_out;
+            if (!direct) {
 #pragma unroll
-            for (int i = 0; i < V; ++i)
+                for (int i = 0; i < V; ++i)
 #pragma unroll
-                for (int p = 0; p < 4; ++p) acc[i][p] = f2(0.f);
+                    for (int p = 0; p < 4; ++p) acc[i][p] = f2(0.f);
+            }
             for (int k = 0; k < a.t; ++k) {
                 mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
@@ -336,7 +341,12 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
             // residual add; the sum is stored in the I/O dtype and the norm
             // reads the stored (rounded) value
             mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
-            {
+            if (direct) {
+                const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    if (c + i * C < hvc) IO<T>::unpack2(load_vec<T>(buf, c + i * C), acc[i]);
+            } else {
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
                 unsigned char* rout =
                     static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.seg_bytes;
@@ -366,7 +376,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                     if (c + i * C < hvc)
 #pragma unroll
                         for (int p = 0; p < 4; ++p) s2 = add2(s2, acc[i][p]);
-                mean = row_sum(hsum(s2), tail->red[0][g], 0) / a.h_f;
+                mean = row_sum(hsum(s2), tail->red[0][g], 0) * a.inv_h;
                 const F2 mean2 = f2(mean);
                 F2 q2 = f2(0.f);
 #pragma unroll
@@ -377,8 +387,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                             const F2 d = sub2(acc[i][p], mean2);
                             q2 = fma2(d, d, q2);
                         }
-                const float var = row_sum(hsum(q2), tail->red[1][g], 1) / a.h_f;
-                rstd = 1.0f / sqrtf(var + a.eps);
+                const float var = row_sum(hsum(q2), tail->red[1][g], 1) * a.inv_h;
+                rstd = rsqrtf(var + a.eps);
             } else {
                 F2 q2 = f2(0.f);
 #pragma unroll
@@ -386,8 +396,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                     if (c + i * C < hvc)
 #pragma unroll
                         for (int p = 0; p < 4; ++p) q2 = fma2(acc[i][p], acc[i][p], q2);
-                const float ms = row_sum(hsum(q2), tail->red[parity][g], 0) / a.h_f;
-                rstd = 1.0f / sqrtf(ms + a.eps);
+                const float ms = row_sum(hsum(q2), tail->red[parity][g], 0) * a.inv_h;
+                rstd = rsqrtf(ms + a.eps);
             }
 
             const F2 mean2 = f2(mean), rstd2 = f2(rstd);
@@ -472,17 +482,17 @@ __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ Fwd
         if (LN) {
             float s = 0.f;
             for (int j = threadIdx.x; j < h; j += blockDim.x) s += xs[j];
-            mean = block_sum(s, red) / a.h_f;
+            mean = block_sum(s, red) * a.inv_h;
             float q = 0.f;
             for (int j = threadIdx.x; j < h; j += blockDim.x) {
                 const float d = xs[j] - mean;
                 q += d * d;
             }
-            rstd = 1.0f / sqrtf(block_sum(q, red) / a.h_f + a.eps);
+            rstd = rsqrtf(block_sum(q, red) * a.inv_h + a.eps);
         } else {
             float q = 0.f;
             for (int j = threadIdx.x; j < h; j += blockDim.x) q += xs[j] * xs[j];
-            rstd = 1.0f / sqrtf(block_sum(q, red) / a.h_f + a.eps);
+            rstd = rsqrtf(block_sum(q, red) * a.inv_h + a.eps);
         }
         for (int j = threadIdx.x; j < h; j += blockDim.x) {
             const float g = IO<T>::load1(a.gamma, j);

@@ -499,7 +499,7 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
     a.stage_stride = (uint32_t)round128(a.seg_bytes);
     a.mask_row_bytes = 4 * ((h + 31) / 32);
     a.eps = cfg->eps;
-    a.h_f = (float)h;
+    a.inv_h = (float)(1.0 / (double)h);
     a.scale = 1.0f / (1.0f - cfg->p_drop);
     a.thr = drop_threshold(cfg->p_drop);
     a.seed_lo = (uint32_t)cfg->seed;
@@ -682,7 +682,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     a.seg_bytes = (uint32_t)(h * E);
     a.stage_stride = (uint32_t)round128(a.seg_bytes);
     a.mask_row_bytes = 4 * ((h + 31) / 32);
-    a.h_f = (float)h;
+    a.inv_h = (float)(1.0 / (double)h);
     a.scale = 1.0f / (1.0f - cfg->p_drop);
     a.want_dbeta = (ln && dbeta) ? 1 : 0;
     a.want_dbias = dbias ? 1 : 0;
