@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "sp_region.cu")
 DEPS = [os.path.join(HERE, "csrc", f) for f in
         ("sp_region.cu", "sp_device.cuh", "sp_fwd.cuh", "sp_bwd.cuh",
-         "sp_gather.cuh")] + [os.path.join(ROOT, "include", "sp_region.h")]
+         "sp_gather.cuh", "sp_entry.cuh")] + [os.path.join(ROOT, "include", "sp_region.h")]
 LIB = os.path.join(HERE, "libsp_region.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -5,11 +5,13 @@
 #include <math.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "sp_region.h"
 #include "sp_bwd.cuh"
 #include "sp_device.cuh"
+#include "sp_entry.cuh"
 #include "sp_fwd.cuh"
 #include "sp_gather.cuh"
 
@@ -223,6 +225,18 @@ const void* bwd_kernel(int id)
         SP_BWD_CASE(20) SP_BWD_CASE(21) SP_BWD_CASE(22)
     }
     return nullptr;
+}
+
+// entry kernel: V = 4 vectors per thread in bf16, 2 in fp32 (registers)
+template <typename T>
+const void* entry_kernel_t(bool ln, bool exact)
+{
+    constexpr int V = sizeof(T) == 2 ? 4 : 2;
+    if (ln)
+        return exact ? (const void*)k_norm_ag<T, V, true, true>
+                     : (const void*)k_norm_ag<T, V, true, false>;
+    return exact ? (const void*)k_norm_ag<T, V, false, true>
+                 : (const void*)k_norm_ag<T, V, false, false>;
 }
 
 template <bool LN>
@@ -512,6 +526,39 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
     }
     a.dropout = cfg->p_drop > 0.0f ? 1 : 0;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    // the entry (no partial sums) without a plan hint: registers instead of
+    // a staging ring, G groups of C threads per CTA
+    if (nparts == 0 && cfg->fwd_plan == 0 && h % 8 == 0 && all16) {
+        const int V = E == 2 ? 4 : 2;
+        const int C = group_threads(h / 8, V);
+        if (C <= kEntryThreads) {
+            EntryArgs e;
+            memset(&e, 0, sizeof(e));
+            e.x = residual;
+            e.gamma = gamma;
+            e.beta = ln ? beta : nullptr;
+            for (int q = 0; q < n_gathered; ++q) e.gathered[q] = gathered[q];
+            e.mean = ln ? mean : nullptr;
+            e.rstd = rstd;
+            e.rows = rows;
+            e.row0 = row0;
+            e.hv = h / 8;
+            e.C = C;
+            e.n_gathered = n_gathered;
+            e.seg_bytes = (uint32_t)(h * E);
+            e.param_stride = (uint32_t)round128((size_t)h * E);
+            e.inv_h = a.inv_h;
+            e.eps = cfg->eps;
+            const int G = std::min(8, kEntryThreads / C);
+            const size_t smem = 2 * (size_t)e.param_stride + (size_t)2 * G * 64 * sizeof(float);
+            const bool exact = C * V == h / 8;
+            const void* kern = cfg->dtype == SP_BF16 ? entry_kernel_t<__nv_bfloat16>(ln, exact)
+                                                     : entry_kernel_t<float>(ln, exact);
+            const int grid = (int)(rows < dev.sms ? rows : dev.sms);
+            return launch_kernel(kern, grid, G * C, smem, st, &e);
+        }
+    }
 
     if (h % 8 == 0 && all16) {
         const FastLaunch L = plan_fwd(a, dev, E, cfg->fwd_plan);

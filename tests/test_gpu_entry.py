@@ -24,6 +24,10 @@ CASES = {
     "ln_h12288_t16": dict(base="C5", s=160, b=1, outliers=0.0),
     "ln_general_h100": dict(base="C2", s=40, b=2, h=100, t=4),
     "f32_ln_h512": dict(base="C2", s=64, b=3, h=512, t=2, dtype="f32"),
+    # vectors per row not a multiple of the threads' share: guarded tail
+    "ln_h1000_ragged": dict(base="C2", s=64, b=2, h=1000, t=4),
+    "f32_rms_h520_ragged": dict(base="C3", s=48, b=2, h=520, t=2, dtype="f32"),
+    "ln_h2048_no_beta": dict(base="C2", s=64, b=2, h=2048, t=4, has_beta=False),
 }
 
 
@@ -34,7 +38,7 @@ def _w(name):
 
 def _params(w):
     bias, gamma, beta = sp_synth.draw_params(w)
-    return gamma, (beta if w.norm == "layernorm" else None)
+    return gamma, (beta if w.norm == "layernorm" and w.has_beta else None)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -44,8 +48,12 @@ def _needs_gpu():
     oracle.build()
 
 
+@pytest.mark.parametrize("plan", [0, 14])
 @pytest.mark.parametrize("name", sorted(CASES))
-def test_entry_forward_matches_oracle(name):
+def test_entry_forward_matches_oracle(name, plan):
+    """plan 0: the register-streaming entry kernel (or the general kernel for
+    h not a multiple of 8); plan 14: the staged-ring forward kernel run with
+    no partial sums, where the shape fits it."""
     w = _w(name)
     x = sp_synth.draw_residual(w)
     gamma, beta = _params(w)
@@ -54,7 +62,7 @@ def test_entry_forward_matches_oracle(name):
     outs = [Guarded((N, h), w.torch_dtype) for _ in range(2)]
     mean = Guarded((N,), torch.float32)
     rstd = Guarded((N,), torch.float32)
-    sp.sp_norm_all_gather_fwd(cfg_of(w), x.cuda(), gamma.cuda(),
+    sp.sp_norm_all_gather_fwd(cfg_of(w, fwd_plan=plan), x.cuda(), gamma.cuda(),
                               None if beta is None else beta.cuda(),
                               [o.t for o in outs], mean.t, rstd.t)
     torch.cuda.synchronize()
