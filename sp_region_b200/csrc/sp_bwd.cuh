@@ -65,7 +65,9 @@ struct BwdArgs {
 // groups update by turns.  2: tensor memory, one private set per thread:
 // warp w uses the columns [(w / 4) * 24V, (w / 4 + 1) * 24V) of its lane
 // quarter, 24 columns per vector i (dgamma, dbeta, dbias; 8 each).
-template <typename T, int V, int G, int MAXT, bool LN, int ACC>
+// EXACT: the threads' vectors tile the row exactly (C * V == hv), so the
+// per-vector bounds checks compile away.
+template <typename T, int V, int G, int MAXT, bool LN, int ACC, bool EXACT = false>
 __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ BwdArgs a)
 {
     constexpr bool ACC_SMEM = ACC == 1;
@@ -129,11 +131,11 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 #pragma unroll
     for (int i = 0; i < V; ++i) {
         const int v = c + i * C;
-        if (g == 0 && v < hv) store_vec<T>(sgam, v, load_vec<T>(a.gamma, v));
+        if (g == 0 && (EXACT || v < hv)) store_vec<T>(sgam, v, load_vec<T>(a.gamma, v));
         if (ACC_REGS) {
 #pragma unroll
             for (int p = 0; p < 4; ++p) ag[i][p] = ab[i][p] = ac[i][p] = f2(0.f);
-        } else if (ACC_SMEM && v < hv) {
+        } else if (ACC_SMEM && (EXACT || v < hv)) {
 #pragma unroll
             for (int q = 0; q < 3; ++q) {
                 accs[((size_t)q * 2 + 0) * hv + v] = make_ulonglong2(0ull, 0ull);
@@ -220,7 +222,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
-            kb[i] = (a.mask && v < hv) ? a.mask[(size_t)i_row * a.mask_row_bytes + v] : 0xFFu;
+            kb[i] = (a.mask && (EXACT || v < hv)) ? a.mask[(size_t)i_row * a.mask_row_bytes + v] : 0xFFu;
         }
 
         // reduce-scatter of the upstream gradient partials, k ascending, from +0
@@ -235,7 +237,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
-                if (v < hv) {
+                if (EXACT || v < hv) {
                     F2 f[4];
                     IO<T>::unpack2(load_vec<T>(buf, v), f);
 #pragma unroll
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
             F2 dgm[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
-            if (v < hv) {
+            if (EXACT || v < hv) {
                 F2 xv[4], gm[4];
                 IO<T>::unpack2(load_vec<T>(xb, v), xv);
                 IO<T>::unpack2(load_vec<T>(sgam, v), gm);
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
             F2 dz[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
-            if (v < hv) {
+            if (EXACT || v < hv) {
                 F2 xv[4], gm[4], dr[4];
                 IO<T>::unpack2(load_vec<T>(xb, v), xv);
                 IO<T>::unpack2(load_vec<T>(sgam, v), gm);
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             tmem_ld16(tacc + 24 * i, tr);
             tmem_ld8(tacc + 24 * i + 16, tr + 16);
         }
-        if (v < hv) {
+        if (EXACT || v < hv) {
             for (int q = 0; q < 3; ++q) {
                 ulonglong2 lo, hi;
                 if (ACC_SMEM) {

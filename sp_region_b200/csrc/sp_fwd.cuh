@@ -193,7 +193,9 @@ __device__ __forceinline__ void init_ring(RingTail* tail, int S, int warps_per_g
 // [r*hv/2, (r+1)*hv/2) of every row); the row's partial sums for mean and
 // variance are exchanged through distributed shared memory and added in rank
 // order, so both CTAs normalise with the same bits.
-template <typename T, int V, int G, int MAXT, bool LN, int CS = 1>
+// EXACT: the threads' vectors tile the row slice exactly (C * V == hv / CS),
+// so the per-vector bounds checks compile away.
+template <typename T, int V, int G, int MAXT, bool LN, int CS = 1, bool EXACT = false>
 __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ FwdArgs a)
 {
     using Vec = typename IO<T>::Vec;
@@ -241,7 +243,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
-                if (v < hvc) {
+                if (EXACT || v < hvc) {
                     store_vec<T>(sg, v, load_vec<T>(a.gamma, vg0 + v));
                     if (a.beta) store_vec<T>(sb, v, load_vec<T>(a.beta, vg0 + v));
                     if (a.bias) store_vec<T>(sc, v, load_vec<T>(a.bias, vg0 + v));
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
                     const int v = c + i * C;
-                    if (v < hvc) {
+                    if (EXACT || v < hvc) {
                         F2 f[4];
                         IO<T>::unpack2(load_vec<T>(buf, v), f);
 #pragma unroll
@@ -316,7 +318,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
-                if (v < hvc) {
+                if (EXACT || v < hvc) {
                     if (a.bias) {
                         F2 f[4];
                         IO<T>::unpack2(load_vec<T>(sc, v), f);
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
 #pragma unroll
                 for (int i = 0; i < V; ++i)
-                    if (c + i * C < hvc) IO<T>::unpack2(load_vec<T>(buf, c + i * C), acc[i]);
+                    if (EXACT || c + i * C < hvc) IO<T>::unpack2(load_vec<T>(buf, c + i * C), acc[i]);
             } else {
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
                 unsigned char* rout =
@@ -353,7 +355,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
                     const int v = c + i * C;
-                    if (v < hvc) {
+                    if (EXACT || v < hvc) {
                         F2 f[4];
                         IO<T>::unpack2(load_vec<T>(buf, v), f);
 #pragma unroll
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 F2 s2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i)
-                    if (c + i * C < hvc)
+                    if (EXACT || c + i * C < hvc)
 #pragma unroll
                         for (int p = 0; p < 4; ++p) s2 = add2(s2, acc[i][p]);
                 mean = row_sum(hsum(s2), tail->red[0][g], 0) * a.inv_h;
@@ -381,7 +383,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 F2 q2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i)
-                    if (c + i * C < hvc)
+                    if (EXACT || c + i * C < hvc)
 #pragma unroll
                         for (int p = 0; p < 4; ++p) {
                             const F2 d = sub2(acc[i][p], mean2);
@@ -393,7 +395,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                 F2 q2 = f2(0.f);
 #pragma unroll
                 for (int i = 0; i < V; ++i)
-                    if (c + i * C < hvc)
+                    if (EXACT || c + i * C < hvc)
 #pragma unroll
                         for (int p = 0; p < 4; ++p) q2 = fma2(acc[i][p], acc[i][p], q2);
                 const float ms = row_sum(hsum(q2), tail->red[parity][g], 0) * a.inv_h;
@@ -404,7 +406,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 #pragma unroll
             for (int i = 0; i < V; ++i) {
                 const int v = c + i * C;
-                if (v < hvc) {
+                if (EXACT || v < hvc) {
                     F2 gm[4], o[4];
                     IO<T>::unpack2(load_vec<T>(sg, v), gm);
                     if (LN && a.beta) {

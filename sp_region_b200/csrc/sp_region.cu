@@ -195,9 +195,9 @@ long long ring_stages(long long smem_optin, long long fixed, uint32_t stage_stri
 #define SP_FWD_CASE(ID)                                                                 \
     case ID:                                                                            \
         return (const void*)k_fwd_tma<T, kFwdPlans[ID].V, kFwdPlans[ID].G,              \
-                                      kFwdPlans[ID].maxT, LN, kFwdPlans[ID].CS>;
+                                      kFwdPlans[ID].maxT, LN, kFwdPlans[ID].CS, EXACT>;
 
-template <typename T, bool LN>
+template <typename T, bool LN, bool EXACT>
 const void* fwd_kernel(int id)
 {
     switch (id) {
@@ -212,9 +212,9 @@ const void* fwd_kernel(int id)
 #define SP_BWD_CASE(ID)                                                                 \
     case ID:                                                                            \
         return (const void*)k_bwd_tma<T, kBwdPlans[ID].V, kBwdPlans[ID].G,              \
-                                      kBwdPlans[ID].maxT, LN, kBwdPlans[ID].acc>;
+                                      kBwdPlans[ID].maxT, LN, kBwdPlans[ID].acc, EXACT>;
 
-template <typename T, bool LN>
+template <typename T, bool LN, bool EXACT>
 const void* bwd_kernel(int id)
 {
     switch (id) {
@@ -240,15 +240,23 @@ const void* entry_kernel_t(bool ln, bool exact)
 }
 
 template <bool LN>
-const void* fwd_kernel_dt(int dtype, int id)
+const void* fwd_kernel_dt(int dtype, int id, bool exact)
 {
-    return dtype == SP_BF16 ? fwd_kernel<__nv_bfloat16, LN>(id) : fwd_kernel<float, LN>(id);
+    if (exact)
+        return dtype == SP_BF16 ? fwd_kernel<__nv_bfloat16, LN, true>(id)
+                                : fwd_kernel<float, LN, true>(id);
+    return dtype == SP_BF16 ? fwd_kernel<__nv_bfloat16, LN, false>(id)
+                            : fwd_kernel<float, LN, false>(id);
 }
 
 template <bool LN>
-const void* bwd_kernel_dt(int dtype, int id)
+const void* bwd_kernel_dt(int dtype, int id, bool exact)
 {
-    return dtype == SP_BF16 ? bwd_kernel<__nv_bfloat16, LN>(id) : bwd_kernel<float, LN>(id);
+    if (exact)
+        return dtype == SP_BF16 ? bwd_kernel<__nv_bfloat16, LN, true>(id)
+                                : bwd_kernel<float, LN, true>(id);
+    return dtype == SP_BF16 ? bwd_kernel<__nv_bfloat16, LN, false>(id)
+                            : bwd_kernel<float, LN, false>(id);
 }
 
 int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream_t st,
@@ -317,6 +325,7 @@ struct FastLaunch {
     int grid = 0;
     int groups = 1;
     int cs = 1;
+    bool exact = false;   // C * V covers the row (slice) exactly
     size_t smem = 0;
 };
 
@@ -354,6 +363,7 @@ FastLaunch plan_fwd(FwdArgs& a, const DevInfo& dev, int E, int hint)
         L.grid = (int)(a.rows < dev.sms ? a.rows : dev.sms);
         L.groups = p.G;
         L.cs = p.CS;
+        L.exact = C * p.V == a.hv / p.CS;
         L.smem = (size_t)a.tail_off + tailb;
         return L;
     }
@@ -400,6 +410,7 @@ FastLaunch plan_bwd(BwdArgs& a, const DevInfo& dev, int E, int hint)
         L.block = p.G * C + 32;
         L.grid = (int)(a.rows < dev.sms ? a.rows : dev.sms);
         L.groups = p.G;
+        L.exact = C * p.V == a.hv;
         L.smem = (size_t)a.tail_off + tailb;
         return L;
     }
@@ -563,8 +574,8 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
     if (h % 8 == 0 && all16) {
         const FastLaunch L = plan_fwd(a, dev, E, cfg->fwd_plan);
         if (L.plan >= 0) {
-            const void* kern = ln ? fwd_kernel_dt<true>(cfg->dtype, L.plan)
-                                  : fwd_kernel_dt<false>(cfg->dtype, L.plan);
+            const void* kern = ln ? fwd_kernel_dt<true>(cfg->dtype, L.plan, L.exact)
+                                  : fwd_kernel_dt<false>(cfg->dtype, L.plan, L.exact);
             if (L.cs > 1) {
                 int grid = 0;
                 return launch_clusters(kern, rows, L.cs, L.block, L.smem, st, &a, &grid);
@@ -743,8 +754,8 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
             nparts = (long long)L.grid * (kBwdPlans[L.plan].acc == 1 ? 1 : L.groups);
             if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes)
                 return SP_ERR_INVALID_ARG;
-            const void* kern = ln ? bwd_kernel_dt<true>(cfg->dtype, L.plan)
-                                  : bwd_kernel_dt<false>(cfg->dtype, L.plan);
+            const void* kern = ln ? bwd_kernel_dt<true>(cfg->dtype, L.plan, L.exact)
+                                  : bwd_kernel_dt<false>(cfg->dtype, L.plan, L.exact);
             if ((rc = launch_kernel(kern, L.grid, L.block, L.smem, st, &a))) return rc;
             launched = true;
         }
