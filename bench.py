@@ -350,7 +350,8 @@ def run_ours(args):
     }
     dom = "fwd" if f_avg >= b_avg else "bwd"
     dk = kern[dom]
-    traffic = recorded_traffic(f"{dom}:{args.workload}")
+    traffic = recorded_traffic(f"{dom}:{args.workload}" +
+                               (":entry" if args.op == "entry" else ""))
     roofline = {"bound": "hbm", "achieved": round(dk["gbs"], 1),
                 "peak": peak, "unit": "GB/s",
                 "frac": round(dk["gbs"] / peak, 4), "traffic": traffic,
