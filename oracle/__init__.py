@@ -53,7 +53,8 @@ class Cfg(ctypes.Structure):
                 ("h", ctypes.c_int64), ("t", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("norm", ctypes.c_int32),
                 ("eps", ctypes.c_float), ("p_drop", ctypes.c_float),
-                ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
+                ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64),
+                ("res_dtype", ctypes.c_int32)]
 
 
 _lib_handle = None
@@ -117,17 +118,20 @@ def _torch_dtype(code: int) -> torch.dtype:
     return torch.float32 if code == F32 else torch.bfloat16
 
 
-def make_cfg(s, b, h, t, dtype, norm, eps, p_drop, seed=0, offset=0) -> Cfg:
+def make_cfg(s, b, h, t, dtype, norm, eps, p_drop, seed=0, offset=0,
+             res_dtype=None) -> Cfg:
+    """res_dtype: dtype of the residual stream tensors (None or "": dtype)."""
     return Cfg(s=s, b=b, h=h, t=t, dtype=_dtype_code(dtype),
                norm=LAYERNORM if norm in ("layernorm", LAYERNORM) else RMSNORM,
-               eps=eps, p_drop=p_drop, seed=seed, offset=offset)
+               eps=eps, p_drop=p_drop, seed=seed, offset=offset,
+               res_dtype=_dtype_code(res_dtype or dtype))
 
 
 def cfg_from(w, **over) -> Cfg:
     """Oracle configuration from a workload description (``sp_synth``)."""
     d = dict(s=w.s, b=w.b, h=w.h, t=w.t, dtype=w.dtype, norm=w.norm,
              eps=w.eps, p_drop=w.p_drop, seed=w.drop_seed,
-             offset=w.drop_offset)
+             offset=w.drop_offset, res_dtype=w.res)
     d.update(over)
     return make_cfg(**d)
 
@@ -230,13 +234,13 @@ def ring_bytes(t: int, kind: str, V: float) -> float:
 def fwd(cfg: Cfg, parts, bias, residual, gamma, beta, n_out: int = 1,
         want_mask: bool = True) -> dict:
     """Forward on all t emulated ranks.  Tensors are [s*b, h] / [h]."""
-    dt = cfg.dtype
+    dt, rdt = cfg.dtype, cfg.res_dtype
     tdt = _torch_dtype(dt)
     ps = [_cpu(p, dt) for p in parts]
-    bias, residual, gamma, beta = (_cpu(x, dt) for x in
-                                   (bias, residual, gamma, beta))
+    bias, gamma, beta = (_cpu(x, dt) for x in (bias, gamma, beta))
+    residual = _cpu(residual, rdt)
     N, h = cfg.s * cfg.b, cfg.h
-    rout = torch.empty((N, h), dtype=tdt)
+    rout = torch.empty((N, h), dtype=_torch_dtype(rdt))
     gathered = [torch.empty((N, h), dtype=tdt) for _ in range(n_out)]
     mask = (np.zeros((N, mask_words(h)), dtype=np.uint32) if want_mask
             else None)
@@ -255,14 +259,14 @@ def fwd(cfg: Cfg, parts, bias, residual, gamma, beta, n_out: int = 1,
 def fwd_rows(cfg: Cfg, row_ids, part_rows, bias, residual_rows, gamma,
              beta) -> dict:
     """Forward on selected global token rows; inputs are [nrows, h]."""
-    dt = cfg.dtype
+    dt, rdt = cfg.dtype, cfg.res_dtype
     tdt = _torch_dtype(dt)
     ids = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64))
     ps = [_cpu(p, dt) for p in part_rows]
-    bias, residual_rows, gamma, beta = (_cpu(x, dt) for x in
-                                        (bias, residual_rows, gamma, beta))
+    bias, gamma, beta = (_cpu(x, dt) for x in (bias, gamma, beta))
+    residual_rows = _cpu(residual_rows, rdt)
     n, h = len(ids), cfg.h
-    rout = torch.empty((n, h), dtype=tdt)
+    rout = torch.empty((n, h), dtype=_torch_dtype(rdt))
     out = torch.empty((n, h), dtype=tdt)
     mask = np.zeros((n, mask_words(h)), dtype=np.uint32)
     mean = np.zeros(n, dtype=np.float64)
@@ -282,7 +286,8 @@ def norm_ag_fwd(cfg: Cfg, x, gamma, beta, n_out: int = 1) -> dict:
     """Entry into a TP region: per-rank norm of x's shard, then all-gather."""
     dt = cfg.dtype
     tdt = _torch_dtype(dt)
-    x, gamma, beta = (_cpu(v, dt) for v in (x, gamma, beta))
+    gamma, beta = (_cpu(v, dt) for v in (gamma, beta))
+    x = _cpu(x, cfg.res_dtype)
     N, h = cfg.s * cfg.b, cfg.h
     gathered = [torch.empty((N, h), dtype=tdt) for _ in range(n_out)]
     mean = np.zeros(N)
@@ -299,16 +304,17 @@ def norm_ag_fwd(cfg: Cfg, x, gamma, beta, n_out: int = 1) -> dict:
 def bwd(cfg: Cfg, dparts, drnext, x, gamma, mask, mean, rstd,
         with_dbeta: bool = True, with_dbias: bool = True) -> dict:
     """Backward on all t emulated ranks (mask None: nothing was dropped)."""
-    dt = cfg.dtype
+    dt, rdt = cfg.dtype, cfg.res_dtype
     tdt = _torch_dtype(dt)
     ps = [_cpu(p, dt) for p in dparts]
-    drnext, x, gamma = (_cpu(v, dt) for v in (drnext, x, gamma))
+    gamma = _cpu(gamma, dt)
+    drnext, x = (_cpu(v, rdt) for v in (drnext, x))
     N, h = cfg.s * cfg.b, cfg.h
     mask = None if mask is None else np.ascontiguousarray(mask, np.uint32)
     mean = (np.zeros(N) if mean is None
             else np.ascontiguousarray(mean, np.float64))
     rstd = np.ascontiguousarray(rstd, np.float64)
-    dres = torch.empty((N, h), dtype=tdt)
+    dres = torch.empty((N, h), dtype=_torch_dtype(rdt))
     dY = torch.empty((N, h), dtype=tdt)
     dg = np.zeros(h)
     db = np.zeros(h) if with_dbeta else None
@@ -325,18 +331,18 @@ def bwd(cfg: Cfg, dparts, drnext, x, gamma, mask, mean, rstd,
 def bwd_rows(cfg: Cfg, dpart_rows, drnext_rows, x_rows, gamma, mask_rows,
              mean, rstd) -> dict:
     """Backward on selected rows (per-row outputs only)."""
-    dt = cfg.dtype
+    dt, rdt = cfg.dtype, cfg.res_dtype
     tdt = _torch_dtype(dt)
     ps = [_cpu(p, dt) for p in dpart_rows]
-    drnext_rows, x_rows, gamma = (_cpu(v, dt) for v in
-                                  (drnext_rows, x_rows, gamma))
+    gamma = _cpu(gamma, dt)
+    drnext_rows, x_rows = (_cpu(v, rdt) for v in (drnext_rows, x_rows))
     n, h = x_rows.shape
     mask_rows = (None if mask_rows is None
                  else np.ascontiguousarray(mask_rows, np.uint32))
     mean = (np.zeros(n) if mean is None
             else np.ascontiguousarray(mean, np.float64))
     rstd = np.ascontiguousarray(rstd, np.float64)
-    dres = torch.empty((n, h), dtype=tdt)
+    dres = torch.empty((n, h), dtype=_torch_dtype(rdt))
     dY = torch.empty((n, h), dtype=tdt)
     rc = _lib().orc_bwd_rows(ctypes.byref(cfg), n, _ptr_array(ps),
                              _ptr(drnext_rows), _ptr(x_rows), _ptr(gamma),

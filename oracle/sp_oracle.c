@@ -43,8 +43,13 @@
  *   - the mask is bit-packed: bit j&31 of word n*W + (j>>5), W = ceil(h/32);
  *   - LayerNorm uses the biased variance and eps inside the square root;
  *     RMSNorm has no mean and no beta;
- *   - the norm reads the residual sum after it is rounded to the I/O dtype
- *     (that rounded tensor is what is stored for the backward).
+ *   - the norm reads the residual sum after it is rounded to the residual
+ *     stream's dtype (that rounded tensor is what is stored for the
+ *     backward);
+ *   - the residual stream (residual in, the stored sum, the gradient arriving
+ *     on it and the residual gradient out) has its own dtype, res_dtype: the
+ *     I/O dtype, or fp32 beside bf16 partial sums, parameters and norm
+ *     outputs (a mixed-precision layer keeps its residual stream in fp32).
  *
  * Parity pins for every function here live in the oracle tests; none of the
  * functions is unpinned.
@@ -67,6 +72,7 @@ typedef struct {
     float eps;
     float p_drop;
     uint64_t seed, offset;
+    int32_t res_dtype;   /* dtype of the residual stream tensors */
 } orc_cfg;
 
 /* ------------------------------------------------------------------------- */
@@ -234,9 +240,9 @@ static void region_row_fwd(const orc_cfg* c, int64_t n, const double* y,
         int keep = orc_keep(c->seed, c->offset, n, j, c->p_drop);
         v = keep ? v * scale : 0.0;
         if (mask_row && keep) mask_row[j >> 5] |= 1u << (j & 31);
-        /* residual add; the sum is stored in the I/O dtype */
-        double r = orc_round(ld(resid, rrow * h + j, c->dtype) + v, c->dtype);
-        st(rout, rrow * h + j, c->dtype, r);
+        /* residual add; the sum is stored in the residual stream's dtype */
+        double r = orc_round(ld(resid, rrow * h + j, c->res_dtype) + v, c->res_dtype);
+        st(rout, rrow * h + j, c->res_dtype, r);
         x[j] = r;
     }
 
@@ -271,6 +277,7 @@ static int cfg_ok(const orc_cfg* c)
     if (c->s % c->t) return 0;
     if (!(c->p_drop >= 0.0f && c->p_drop < 1.0f)) return 0;
     if (!(c->eps > 0.0f)) return 0;
+    if (c->res_dtype != ORC_F32 && c->res_dtype != ORC_BF16) return 0;
     return 1;
 }
 
@@ -278,7 +285,7 @@ static int cfg_ok(const orc_cfg* c)
  * Forward of the whole boundary on t emulated ranks.
  *   parts[k]      rank k's partial output of the row-parallel linear, [s,b,h]
  *   residual      [s,b,h], rank r's shard is its rows
- *   residual_out  [s,b,h] (rank r writes its rows), I/O dtype
+ *   residual_out  [s,b,h] (rank r writes its rows), residual stream dtype
  *   gathered      n_out buffers [s,b,h]: the all-gathered norm output
  *   mask          [s*b][W] u32 or NULL;  mean/rstd [s*b] (mean NULL for RMS)
  * Returns 0, or -1 for an invalid configuration.
@@ -366,7 +373,7 @@ int orc_fwd_rows(const orc_cfg* c, int64_t nrows, const int64_t* row_ids,
  * first FFN linear).  Rank r normalises its rows of x; every requested
  * replica receives all ranks' shards in order.  No reduction, bias, dropout
  * or residual add: the SP region's sum was formed by the previous exit.
- *   x         [s,b,h] in the I/O dtype, rank r's shard is its rows
+ *   x         [s,b,h] in the residual stream's dtype, rank r's shard is its rows
  *   gathered  n_out buffers [s,b,h];  mean/rstd [s*b] (mean NULL for RMS)
  */
 int orc_norm_ag_fwd(const orc_cfg* c, const void* x, const void* gamma,
@@ -387,7 +394,7 @@ int orc_norm_ag_fwd(const orc_cfg* c, const void* x, const void* gamma,
         for (int64_t i = 0; i < per; ++i) {
             const int64_t n = (int64_t)r * per + i;
             double* o = shards[r] + i * h;
-            for (int64_t j = 0; j < h; ++j) xr[j] = ld(x, n * h + j, c->dtype);
+            for (int64_t j = 0; j < h; ++j) xr[j] = ld(x, n * h + j, c->res_dtype);
             double mu = 0.0, var = 0.0, rs;
             if (c->norm == ORC_LAYERNORM) {
                 for (int64_t j = 0; j < h; ++j) mu += xr[j];
@@ -430,7 +437,7 @@ int orc_norm_ag_fwd(const orc_cfg* c, const void* x, const void* gamma,
 /* reverse-mode through norm, residual add and dropout for one token row.
  *   dn    gradient w.r.t. the norm output of this row (after the
  *         reduce-scatter that is the all-gather's backward)
- *   x     the stored residual sum of the row (I/O dtype)
+ *   x     the stored residual sum of the row (residual stream dtype)
  *   acc   per-rank accumulators: dgamma[h], dbeta[h], dbias[h]
  *   dz    gradient w.r.t. the dropout input (the reduced partial sum) */
 static void region_row_bwd(const orc_cfg* c, const double* dn,
@@ -444,7 +451,7 @@ static void region_row_bwd(const orc_cfg* c, const double* dn,
     const double scale = 1.0 / (1.0 - (double)c->p_drop);
     double sum_g = 0.0, sum_gx = 0.0;
     for (int64_t j = 0; j < h; ++j) {
-        double xv = ld(x, row * h + j, c->dtype);
+        double xv = ld(x, row * h + j, c->res_dtype);
         xhat[j] = (c->norm == ORC_LAYERNORM) ? (xv - mean) * rstd : xv * rstd;
         double g = dn[j] * ld(gamma, j, c->dtype);
         sum_g += g;
@@ -459,8 +466,8 @@ static void region_row_bwd(const orc_cfg* c, const double* dn,
                         ? rstd * (g - mg - xhat[j] * mgx)
                         : rstd * (g - xhat[j] * mgx);
         /* the residual sum feeds both the norm and the next residual add */
-        double dr = dx + (drnext ? ld(drnext, row * h + j, c->dtype) : 0.0);
-        st(dres_in, row * h + j, c->dtype, dr);
+        double dr = dx + (drnext ? ld(drnext, row * h + j, c->res_dtype) : 0.0);
+        st(dres_in, row * h + j, c->res_dtype, dr);
         int keep = mask_row ? (int)((mask_row[j >> 5] >> (j & 31)) & 1u) : 1;
         dz[j] = keep ? dr * scale : 0.0;
         if (dbias) dbias[j] += dz[j];

@@ -72,6 +72,10 @@ class Workload:
     heads: int = 0       # attention heads for the activation-memory check
     backward: bool = False
     gather_replicas: bool = False  # also gather into t per-rank replicas
+    # dtype of the residual stream (residual in, stored sum, dR_next and the
+    # residual gradient): "" for the I/O dtype, or "f32" (an fp32 residual
+    # stream beside bf16 partial sums, parameters and norm outputs)
+    res_dtype: str = ""
 
     @property
     def rows(self) -> int:
@@ -84,6 +88,19 @@ class Workload:
     @property
     def elem_bytes(self) -> int:
         return 4 if self.dtype == "f32" else 2
+
+    @property
+    def res(self) -> str:
+        """dtype of the residual stream"""
+        return self.res_dtype or self.dtype
+
+    @property
+    def res_torch_dtype(self) -> torch.dtype:
+        return torch.float32 if self.res == "f32" else torch.bfloat16
+
+    @property
+    def res_elem_bytes(self) -> int:
+        return 4 if self.res == "f32" else 2
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -176,7 +193,7 @@ def draw_partials(w: Workload, device="cpu", rows: Optional[int] = None,
 def draw_residual(w: Workload, device="cpu", rows: Optional[int] = None):
     n = w.rows if rows is None else rows
     return _draw((n, w.h), w.dist, 1.0, 0.0, w.seed, _ID_RESIDUAL, device,
-                 w.torch_dtype)
+                 w.res_torch_dtype)
 
 
 def draw_params(w: Workload, device="cpu"):
@@ -215,7 +232,7 @@ def draw_residual_grad(w: Workload, device="cpu", rows: Optional[int] = None):
     """Optional gradient arriving on the residual stream from later layers."""
     n = w.rows if rows is None else rows
     return _draw((n, w.h), w.dist, 1.0, 0.0, w.seed, _ID_DRNEXT, device,
-                 w.torch_dtype)
+                 w.res_torch_dtype)
 
 
 def dyadic_atoms(rows: int, h: int, seed: int, n_atoms: int = 16,

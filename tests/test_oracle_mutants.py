@@ -59,7 +59,7 @@ MUTANTS = {
     "dropout backward not rescaled": (
         "dz[j] = keep ? dr * scale : 0.0;", "dz[j] = keep ? dr : 0.0;"),
     "residual-stream gradient dropped": (
-        "double dr = dx + (drnext ? ld(drnext, row * h + j, c->dtype) : 0.0);",
+        "double dr = dx + (drnext ? ld(drnext, row * h + j, c->res_dtype) : 0.0);",
         "double dr = dx;"),
     "dgamma without xhat": (
         "dgamma[j] += dn[j] * xhat[j];", "dgamma[j] += dn[j];"),
@@ -68,13 +68,19 @@ MUTANTS = {
         "coeff = 10.0 + 24.0 / (double)t + attn;"),
     "norm reads the unrounded residual sum": (
         "        x[j] = r;\n",
-        "        x[j] = ld(resid, rrow * h + j, c->dtype) + v;\n"),
+        "        x[j] = ld(resid, rrow * h + j, c->res_dtype) + v;\n"),
     "entry norm drops beta": (
         "o[j] = (xr[j] - mu) * rs * ld(gamma, j, c->dtype) + b;",
         "o[j] = (xr[j] - mu) * rs * ld(gamma, j, c->dtype) + 0 * b;"),
     "entry norm uses the unbiased variance": (
         "var += (xr[j] - mu) * (xr[j] - mu);\n                var /= (double)h;",
         "var += (xr[j] - mu) * (xr[j] - mu);\n                var /= (double)(h - 1);"),
+    "residual sum stored in the I/O dtype": (
+        "double r = orc_round(ld(resid, rrow * h + j, c->res_dtype) + v, c->res_dtype);",
+        "double r = orc_round(ld(resid, rrow * h + j, c->res_dtype) + v, c->dtype);"),
+    "residual gradient stored in the I/O dtype": (
+        "st(dres_in, row * h + j, c->res_dtype, dr);",
+        "st(dres_in, row * h + j, c->dtype, dr);"),
     "ring volume without (t-1)/t": (
         "double phase = (double)(t - 1) / (double)t * V;",
         "double phase = V;"),

@@ -630,3 +630,92 @@ def test_entry_norm_matches_torch_and_gathers_in_rank_order(orc, norm):
     fo = orc.fwd(orc.cfg_from(w, p_drop=0.0), [torch.zeros_like(x)] * w.t, None, x,
                  gamma, beta)
     assert torch.equal(fo["gathered"][0], out["gathered"][0])
+
+
+# ----------------------------------------------------------------------------
+# fp32 residual stream beside bf16 partial sums, parameters and norm outputs
+# ----------------------------------------------------------------------------
+
+def _mixed(norm="layernorm", **over):
+    d = dict(s=12, b=2, h=96, t=4, norm=norm, dtype="bf16", res_dtype="f32",
+             p_drop=0.25, has_bias=True, has_beta=norm == "layernorm")
+    d.update(over)
+    return sp_synth.WORKLOADS["C2"].replace(**d)
+
+
+def _keep_matrix(orc, w):
+    p = float(np.float32(w.p_drop))
+    return np.array([[orc.keep(w.drop_seed, w.drop_offset, n, j, p)
+                      for j in range(w.h)] for n in range(w.rows)])
+
+
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+def test_fp32_residual_stream_forward(orc, norm):
+    """The stored sum is the fp32 rounding of residual + dropout(sum of
+    partials + bias), formed in float64 here by torch; the norm output is
+    the library norm of that fp32 tensor, rounded to bf16."""
+    w = _mixed(norm)
+    cfg = orc.cfg_from(w)
+    parts = sp_synth.draw_partials(w)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    beta = beta if norm == "layernorm" else None
+    res = sp_synth.draw_residual(w)
+    assert res.dtype == torch.float32 and parts[0].dtype == torch.bfloat16
+    out = orc.fwd(cfg, parts, bias, res, gamma, beta)
+    y = torch.stack([p.double() for p in parts]).sum(0) + bias.double()
+    scale = 1.0 / (1.0 - float(np.float32(w.p_drop)))
+    keep = torch.from_numpy(_keep_matrix(orc, w))
+    z = torch.where(keep, y * scale, torch.zeros_like(y))
+    want = (res.double() + z).float()
+    assert out["residual_out"].dtype == torch.float32
+    assert torch.equal(out["residual_out"], want)
+    # the pin has power: bf16 storage of the sum would differ
+    assert not torch.equal(want.bfloat16().float(), want)
+    eps = float(np.float32(w.eps))
+    x = want.double()
+    if norm == "layernorm":
+        ref = F.layer_norm(x, (w.h,), gamma.double(), beta.double(), eps)
+    else:
+        ref = F.rms_norm(x, (w.h,), gamma.double(), eps)
+    got = out["gathered"][0]
+    assert got.dtype == torch.bfloat16
+    r = ref.numpy()
+    assert (np.abs(got.double().numpy() - r) <= _ulp_bf16(r) * 0.5 + 1e-12 * np.abs(r)).all()
+
+
+def test_fp32_residual_stream_backward(orc):
+    """Reverse mode against torch autograd in float64: the residual gradient
+    (with one arriving on the stream) is stored in fp32, dY in bf16."""
+    w = _mixed()
+    cfg = orc.cfg_from(w)
+    parts = sp_synth.draw_partials(w)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    res = sp_synth.draw_residual(w)
+    fo = orc.fwd(cfg, parts, bias, res, gamma, beta)
+    dparts = sp_synth.draw_grad_partials(w)
+    drn = sp_synth.draw_residual_grad(w)
+    assert drn.dtype == torch.float32
+    bo = orc.bwd(cfg, dparts, drn, fo["residual_out"], gamma, fo["mask"],
+                 fo["mean"], fo["rstd"])
+    dn = torch.stack([d.double() for d in dparts]).sum(0)
+    y = torch.stack([p.double() for p in parts]).sum(0)
+    ref = _torch_reference_grads(w, y, bias, fo["residual_out"], gamma, beta,
+                                 fo["mask"], dn, drn)
+    assert bo["dresidual_in"].dtype == torch.float32
+    assert torch.equal(bo["dresidual_in"], ref["dresidual_in"].float())
+    r = ref["dY"].numpy()
+    assert (np.abs(bo["dY"].double().numpy() - r) <= _ulp_bf16(r) * 0.5 + 1e-12 * np.abs(r)).all()
+    for k in ("dgamma", "dbeta", "dbias"):
+        assert np.allclose(bo[k], ref[k].numpy(), rtol=1e-10, atol=1e-10), k
+
+
+def test_fp32_residual_stream_entry(orc):
+    """The entry normalises an fp32 residual stream into bf16 outputs."""
+    w = _mixed(p_drop=0.0, has_bias=False, s=16, h=64)
+    x = sp_synth.draw_residual(w)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    out = orc.norm_ag_fwd(orc.cfg_from(w), x, gamma, beta)
+    ref = F.layer_norm(x.double(), (w.h,), gamma.double(), beta.double(),
+                       float(np.float32(w.eps))).numpy()
+    got = out["gathered"][0].double().numpy()
+    assert (np.abs(got - ref) <= _ulp_bf16(ref) * 0.5 + 1e-12 * np.abs(ref)).all()
