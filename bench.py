@@ -46,46 +46,57 @@ FALLBACK_HBM_GBS = 6650.0
 # algorithmic bytes (per call), from the data each call must move
 # ----------------------------------------------------------------------------
 
+# E: bytes per element of the I/O dtype; Er: of the residual stream
+# (residual, residual_out, x, dR_next, dresidual_in), fp32 with --residual-f32
 def fwd_bytes(w, n_gathered=1):
-    E, N, h = w.elem_bytes, w.rows, w.h
+    E, Er, N, h = w.elem_bytes, w.res_elem_bytes, w.rows, w.h
     sbh = N * h
     W = (h + 31) // 32
     params = h * E * (1 + (1 if w.has_bias else 0) +
                       (1 if (w.has_beta and w.norm == "layernorm") else 0))
-    rd = (w.t + 1) * E * sbh + params
+    rd = w.t * E * sbh + Er * sbh + params
     stats = (8 if w.norm == "layernorm" else 4) * N
-    wr = E * sbh * (1 + n_gathered) + 4 * W * N + stats
+    wr = Er * sbh + E * sbh * n_gathered + 4 * W * N + stats
     return rd + wr
 
 
 def bwd_bytes(w, with_drnext=False):
-    E, N, h = w.elem_bytes, w.rows, w.h
+    E, Er, N, h = w.elem_bytes, w.res_elem_bytes, w.rows, w.h
     sbh = N * h
     W = (h + 31) // 32
     stats = (8 if w.norm == "layernorm" else 4) * N
-    rd = w.t * E * sbh + E * sbh + 4 * W * N + stats + h * E
+    rd = w.t * E * sbh + Er * sbh + 4 * W * N + stats + h * E
     if with_drnext:
-        rd += E * sbh
+        rd += Er * sbh
     ngrad = 1 + (1 if w.norm == "layernorm" else 0) + (1 if w.has_bias else 0)
-    wr = 2 * E * sbh + 4 * h * ngrad
+    wr = Er * sbh + E * sbh + 4 * h * ngrad
     return rd + wr
 
 
 def entry_fwd_bytes(w, n_gathered=1):
     """Entry into a TP region: read x, write the gathered norm output."""
-    E, N, h = w.elem_bytes, w.rows, w.h
+    E, Er, N, h = w.elem_bytes, w.res_elem_bytes, w.rows, w.h
     params = h * E * (1 + (1 if w.norm == "layernorm" else 0))
     stats = (8 if w.norm == "layernorm" else 4) * N
-    return E * N * h + params + n_gathered * E * N * h + stats
+    return Er * N * h + params + n_gathered * E * N * h + stats
 
 
 def entry_bwd_bytes(w):
     """Its backward: reduce-scatter of t upstream partials, norm backward from
     x and the statistics, the residual-stream gradient written."""
-    E, N, h = w.elem_bytes, w.rows, w.h
+    E, Er, N, h = w.elem_bytes, w.res_elem_bytes, w.rows, w.h
     stats = (8 if w.norm == "layernorm" else 4) * N
     ngrad = 1 + (1 if w.norm == "layernorm" else 0)
-    return (w.t + 1) * E * N * h + stats + h * E + E * N * h + 4 * h * ngrad
+    return (w.t * E + Er) * N * h + stats + h * E + Er * N * h + 4 * h * ngrad
+
+
+def workload_of(args):
+    """The named workload; --residual-f32 keeps its residual stream in fp32."""
+    import sp_synth
+    w = sp_synth.WORKLOADS[args.workload]
+    if getattr(args, "residual_f32", False) and w.dtype == "bf16":
+        w = w.replace(res_dtype="f32")
+    return w
 
 
 def measured_peak():
@@ -235,13 +246,15 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
-    w = sp_synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     w = w.replace(seed=w.seed + 1000 * rank)   # each replica its own batch
     N, h, t = w.rows, w.h, w.t
     dt = w.torch_dtype
+    res_f32 = w.res != w.dtype
     cfg = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm, eps=w.eps,
                       p_drop=w.p_drop, seed=w.drop_seed, offset=w.drop_offset,
-                      fwd_plan=args.fwd_plan, bwd_plan=args.bwd_plan)
+                      fwd_plan=args.fwd_plan, bwd_plan=args.bwd_plan,
+                      res_f32=res_f32)
 
     parts = sp_synth.draw_partials(w, dev)
     bias, gamma, beta = sp_synth.draw_params(w, dev)
@@ -251,12 +264,13 @@ def run_ours(args):
         beta = None
     res = sp_synth.draw_residual(w, dev)
     dparts = sp_synth.draw_grad_partials(w, dev)
-    rout = torch.empty((N, h), dtype=dt, device=dev)
+    rdt = w.res_torch_dtype
+    rout = torch.empty((N, h), dtype=rdt, device=dev)
     out = torch.empty((N, h), dtype=dt, device=dev)
     mask = torch.empty((N, (h + 31) // 32), dtype=torch.int32, device=dev)
     mean = torch.empty(N, dtype=torch.float32, device=dev)
     rstd = torch.empty(N, dtype=torch.float32, device=dev)
-    dres = torch.empty((N, h), dtype=dt, device=dev)
+    dres = torch.empty((N, h), dtype=rdt, device=dev)
     dY = torch.empty((N, h), dtype=dt, device=dev)
     dg = torch.empty(h, dtype=torch.float32, device=dev)
     db = torch.empty(h, dtype=torch.float32, device=dev) \
@@ -282,7 +296,7 @@ def run_ours(args):
         # backward: reduce-scatter of the upstream partials, norm backward
         cfg0 = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm,
                            eps=w.eps, p_drop=0.0, fwd_plan=args.fwd_plan,
-                           bwd_plan=args.bwd_plan)
+                           bwd_plan=args.bwd_plan, res_f32=res_f32)
 
         def fwd():
             sp.sp_norm_all_gather_fwd(cfg0, res, gamma, beta, [out], mean,
@@ -351,7 +365,8 @@ def run_ours(args):
     dom = "fwd" if f_avg >= b_avg else "bwd"
     dk = kern[dom]
     traffic = recorded_traffic(f"{dom}:{args.workload}" +
-                               (":entry" if args.op == "entry" else ""))
+                               (":entry" if args.op == "entry" else "") +
+                               (":res_f32" if w.res != w.dtype else ""))
     roofline = {"bound": "hbm", "achieved": round(dk["gbs"], 1),
                 "peak": peak, "unit": "GB/s",
                 "frac": round(dk["gbs"] / peak, 4), "traffic": traffic,
@@ -376,10 +391,12 @@ def run_ours(args):
             "workload": (f"{w.name}: SP boundary fwd+bwd, s={w.s} b={w.b} "
                          f"h={h} t={t} emulated ranks, {w.dtype} I/O, "
                          f"{w.norm}, p={w.p_drop}, bias"
+                         + (", fp32 residual stream" if w.res != w.dtype else "")
                          if args.op == "boundary" else
                          f"{w.name} shape: entry into a TP region (norm + "
                          f"all-gather) fwd+bwd, s={w.s} b={w.b} h={h} t={t}, "
-                         f"{w.dtype} I/O, {w.norm}"),
+                         f"{w.dtype} I/O, {w.norm}"
+                         + (", fp32 residual stream" if w.res != w.dtype else "")),
             "s": w.s, "b": w.b, "h": h, "t": t,
             "global_batch": w.b * world, "seq_len": w.s,
             "parallelism": f"{world} independent replicas (t={t} ranks "
@@ -435,13 +452,14 @@ def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
         dev_in = [None if x is None else torch.empty_like(x, device=dev)
                   for x in ins]
         bufs.append(dev_in)
-    outs_d = dict(rout=torch.empty((N, h), dtype=dt, device=dev),
+    rdt = w.res_torch_dtype
+    outs_d = dict(rout=torch.empty((N, h), dtype=rdt, device=dev),
                   out=torch.empty((N, h), dtype=dt, device=dev),
                   mask=torch.empty((N, (h + 31) // 32), dtype=torch.int32,
                                    device=dev),
                   mean=torch.empty(N, dtype=torch.float32, device=dev),
                   rstd=torch.empty(N, dtype=torch.float32, device=dev),
-                  dres=torch.empty((N, h), dtype=dt, device=dev),
+                  dres=torch.empty((N, h), dtype=rdt, device=dev),
                   dY=torch.empty((N, h), dtype=dt, device=dev),
                   dg=torch.empty(h, dtype=torch.float32, device=dev),
                   db=torch.empty(h, dtype=torch.float32, device=dev),
@@ -625,7 +643,7 @@ def run_reference(args):
     import oracle as orc
     import sp_synth
     orc.build()
-    w = sp_synth.WORKLOADS[args.workload]
+    w = workload_of(args)
     cfg = orc.cfg_from(w)
     fb, bb = fwd_bytes(w), bwd_bytes(w)
     per_row = (fb + bb) / w.rows
@@ -650,7 +668,9 @@ def run_reference(args):
         "impl": "reference",
         "config": {"workload": (f"{w.name}: SP boundary fwd+bwd, s={w.s} "
                                 f"b={w.b} h={w.h} t={w.t}, {w.dtype} I/O, "
-                                f"{w.norm}, p={w.p_drop}, bias"),
+                                f"{w.norm}, p={w.p_drop}, bias"
+                                + (", fp32 residual stream" if w.res != w.dtype
+                                   else "")),
                    "s": w.s, "b": w.b, "h": w.h, "t": w.t,
                    "sample_rows_per_step": rows},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
@@ -677,6 +697,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--residual-f32", action="store_true",
+                    help="keep the residual stream in fp32 beside bf16 I/O")
     ap.add_argument("--fwd-plan", type=int, default=0,
                     help="forward kernel plan hint (0: library's choice)")
     ap.add_argument("--bwd-plan", type=int, default=0,

@@ -32,7 +32,9 @@
  *             [r*N/t, (r+1)*N/t), which is contiguous because the shard is
  *             along s, the outermost dimension.
  * Dtypes      cfg->dtype applies to partial sums, residual, gamma, beta,
- *             bias and every [s,b,h] output; mean, rstd and the parameter
+ *             bias and every [s,b,h] output, except that with cfg->res_f32
+ *             the residual stream's tensors (residual, residual_out, the
+ *             entry's x, dR_next, dresidual_in) are fp32; mean, rstd and the parameter
  *             gradients are always fp32.  Arithmetic is fp32.
  * Memory      every pointer argument named "device" is a CUDA device
  *             pointer on the current device; arrays of pointers
@@ -107,7 +109,17 @@ typedef enum { SP_LAYERNORM = 0, SP_RMSNORM = 1 } sp_norm;
  *            dropout counter uses the global row, so a split into ranges
  *            gives exactly the rows of the whole call.  Parameter gradients
  *            of a range cover its rows only; summing them over the ranges
- *            (the all-reduce of replicated parameters) gives the total. */
+ *            (the all-reduce of replicated parameters) gives the total.
+ *   res_f32  0: the residual stream has the I/O dtype.  1 (with dtype
+ *            SP_BF16): the residual stream is fp32 -- residual, residual_out
+ *            and the entry's x, and in the backward residual_out (x),
+ *            dR_next and dresidual_in -- while partials, bias, gamma, beta,
+ *            gathered outputs and dY stay bf16.  The pages fix no precision
+ *            for the residual ("SP: Partition Activations Alongside TP",
+ *            section "Normalize and add residuals by token"); a
+ *            mixed-precision layer keeps it in fp32.  The residual sum is
+ *            then stored exactly as computed in fp32 and the norm reads it.
+ *            Ignored for SP_F32.  Other values: SP_ERR_INVALID_ARG. */
 typedef struct {
     int64_t s, b, h;
     int32_t t;
@@ -118,6 +130,7 @@ typedef struct {
     uint64_t seed, offset;
     int32_t fwd_plan, bwd_plan;
     int64_t row_begin, row_end;
+    int32_t res_f32;
 } sp_cfg;
 
 /* Number of fast-kernel plans of the forward and the backward (valid hint
@@ -140,7 +153,8 @@ int sp_plan_count(int32_t* fwd_plans, int32_t* bwd_plans);
  *   y       = sum_{k=0..t-1} partials[k][n, :]      fp32, k ascending
  *   y      += bias                                   (once, if bias != NULL)
  *   z       = keep(n, j) ? y / (1 - p_drop) : 0      inverted dropout
- *   r_out   = round(residual[n, :] + z)              stored in cfg->dtype
+ *   r_out   = round(residual[n, :] + z)              stored in the residual
+ *                                                    stream's dtype (res_f32)
  *   LN:  o  = (r_out - mean) * rstd * gamma + beta,
  *        mean, var = mean and biased variance of r_out over h,
  *        rstd = 1 / sqrt(var + eps)
@@ -154,10 +168,10 @@ int sp_plan_count(int32_t* fwd_plans, int32_t* bwd_plans);
  * Arguments (device unless stated):
  *   partials     HOST array of t device pointers, each [s,b,h]
  *   bias         [h] or NULL
- *   residual     [s,b,h]
+ *   residual     [s,b,h] (fp32 with cfg->res_f32)
  *   gamma        [h]
  *   beta         [h] or NULL (LayerNorm without shift; ignored for RMSNorm)
- *   residual_out [s,b,h], may alias residual (in-place update)
+ *   residual_out [s,b,h] (fp32 with cfg->res_f32), may alias residual (in-place update)
  *   gathered     HOST array of n_gathered device pointers, each [s,b,h]; on
  *                one GPU the shard-major norm output is already the gathered
  *                tensor, so n_gathered = 1 is the plain case and n_gathered
@@ -195,7 +209,8 @@ int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg,
  * cfg->p_drop is ignored (no dropout here); nothing is reduced.
  *
  * Arguments (device unless stated):
- *   x          [s,b,h] (the caller's shard when a row range is given)
+ *   x          [s,b,h] (the caller's shard when a row range is given;
+ *              fp32 with cfg->res_f32)
  *   gamma      [h];  beta [h] or NULL (ignored for RMSNorm)
  *   gathered   HOST array of n_gathered device pointers, each [s,b,h],
  *              indexed by global row
@@ -249,11 +264,12 @@ int sp_all_gather(const sp_cfg* cfg, const void* const* shards,
  *
  * Arguments (device unless stated):
  *   dn_partials  HOST array of t device pointers, each [s,b,h]
- *   dR_next      [s,b,h] or NULL
+ *   dR_next      [s,b,h] or NULL (fp32 with cfg->res_f32)
  *   residual_out, mask_bits, mean, rstd   the forward's outputs (mask_bits
  *                may be NULL only when p_drop == 0; mean unused for RMS)
  *   gamma        [h]
- *   dresidual_in [s,b,h]; dY [s,b,h] or NULL (not written; the backward of
+ *   dresidual_in [s,b,h] (fp32 with cfg->res_f32, like residual_out);
+ *                dY [s,b,h] or NULL (not written; the backward of
  *                the entry into a TP region has no dropout input)
  *   dgamma [h] fp32; dbeta [h] fp32 or NULL; dbias [h] fp32 or NULL
  *   workspace    device scratch of at least sp_bwd_workspace_bytes() bytes,

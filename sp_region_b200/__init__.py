@@ -49,7 +49,8 @@ class sp_cfg(ctypes.Structure):
                 ("eps", ctypes.c_float), ("p_drop", ctypes.c_float),
                 ("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64),
                 ("fwd_plan", ctypes.c_int32), ("bwd_plan", ctypes.c_int32),
-                ("row_begin", ctypes.c_int64), ("row_end", ctypes.c_int64)]
+                ("row_begin", ctypes.c_int64), ("row_end", ctypes.c_int64),
+                ("res_f32", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -102,13 +103,16 @@ def make_cfg(s: int, b: int, h: int, t: int, dtype="bf16",
              norm="layernorm", eps: float = 1e-5, p_drop: float = 0.0,
              seed: int = 0, offset: int = 0, fwd_plan: int = 0,
              bwd_plan: int = 0, row_begin: int = 0,
-             row_end: int = 0) -> sp_cfg:
+             row_end: int = 0, res_f32: bool = False) -> sp_cfg:
+    """res_f32: the residual stream (residual, residual_out, the entry's x,
+    dR_next, dresidual_in) is fp32 beside bf16 partials and outputs."""
     dt = {"f32": SP_F32, "bf16": SP_BF16, torch.float32: SP_F32,
           torch.bfloat16: SP_BF16}[dtype]
     nm = {"layernorm": SP_LAYERNORM, "rmsnorm": SP_RMSNORM}[norm]
     return sp_cfg(s=s, b=b, h=h, t=t, dtype=dt, norm=nm, eps=eps,
                   p_drop=p_drop, seed=seed, offset=offset, fwd_plan=fwd_plan,
-                  bwd_plan=bwd_plan, row_begin=row_begin, row_end=row_end)
+                  bwd_plan=bwd_plan, row_begin=row_begin, row_end=row_end,
+                  res_f32=1 if res_f32 else 0)
 
 
 def _p(x: Optional[torch.Tensor]) -> Optional[int]:

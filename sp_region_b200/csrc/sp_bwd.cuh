@@ -48,6 +48,8 @@ struct BwdArgs {
     int t;
     int stages;
     uint32_t seg_bytes;
+    uint32_t res_seg_bytes;  // h * residual stream elem bytes (x, dR_next, dres)
+    int res_f32;             // residual stream in fp32 (I/O dtype bf16)
     uint32_t stage_stride;
     int mask_row_bytes;
     uint32_t param_off;      // shared-memory offsets (fast kernel): gamma copy,
@@ -104,8 +106,9 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
                                            (size_t)(a.row0 + i) * a.seg_bytes;
                                 return static_cast<const unsigned char*>(k == a.t ? a.x
                                                                                   : a.drnext) +
-                                       (size_t)i * a.seg_bytes;
-                            });
+                                       (size_t)i * a.res_seg_bytes;
+                            },
+                            a.t, a.res_seg_bytes);
         return;
     }
 
@@ -182,6 +185,13 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             r[2 * p + 1] = __float_as_uint(x.y);
         }
         tmem_st16(tacc + col, r);
+    };
+    // a vector of a residual-stream tensor (x, dR_next) from shared memory
+    auto load_res = [&](const unsigned char* buf, int v, F2 f[4]) {
+        if (a.res_f32)
+            IO<float>::unpack2(load_vec<float>(buf, v), f);
+        else
+            IO<T>::unpack2(load_vec<T>(buf, v), f);
     };
     auto release_at = [&](uint32_t s_) {
         __syncwarp();
@@ -267,7 +277,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             F2 dgm[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
             if (EXACT || v < hv) {
                 F2 xv[4], gm[4];
-                IO<T>::unpack2(load_vec<T>(xb, v), xv);
+                load_res(xb, v, xv);
                 IO<T>::unpack2(load_vec<T>(sgam, v), gm);
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
@@ -321,7 +331,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         // pass 2: input gradient, residual gradient, dropout backward
         take_turn(1, j);
         unsigned char* dres =
-            static_cast<unsigned char*>(a.dres) + (size_t)i_row * a.seg_bytes;   // shard
+            static_cast<unsigned char*>(a.dres) + (size_t)i_row * a.res_seg_bytes;   // shard
         unsigned char* dy =
             static_cast<unsigned char*>(a.dY) + (size_t)n * a.seg_bytes;       // gathered
 #pragma unroll
@@ -330,7 +340,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
             F2 dz[4] = {f2(0.f), f2(0.f), f2(0.f), f2(0.f)};
             if (EXACT || v < hv) {
                 F2 xv[4], gm[4], dr[4];
-                IO<T>::unpack2(load_vec<T>(xb, v), xv);
+                load_res(xb, v, xv);
                 IO<T>::unpack2(load_vec<T>(sgam, v), gm);
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
@@ -342,7 +352,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
                 }
                 if (rb) {
                     F2 rn[4];
-                    IO<T>::unpack2(load_vec<T>(rb, v), rn);
+                    load_res(rb, v, rn);
 #pragma unroll
                     for (int p = 0; p < 4; ++p) dr[p] = add2(dr[p], rn[p]);
                 }
@@ -350,7 +360,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
                 for (int p = 0; p < 4; ++p)
                     dz[p] = keep2(mul2(dr[p], scale2), (kb[i] >> (2 * p)) & 1u,
                                   (kb[i] >> (2 * p + 1)) & 1u);
-                store_vec<T>(dres, v, IO<T>::pack2v(dr));
+                if (a.res_f32)
+                    store_vec<float>(dres, v, IO<float>::pack2v(dr));
+                else
+                    store_vec<T>(dres, v, IO<T>::pack2v(dr));
                 if (a.dY) store_vec<T>(dy, v, IO<T>::pack2v(dz));
                 if (a.want_dbias) {
                     if (ACC_SMEM) {
@@ -455,7 +468,8 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
             for (int k = 0; k < a.t; ++k) d = (k == 0) ? IO<T>::load1(a.dparts[k], base + j)
                                                        : d + IO<T>::load1(a.dparts[k], base + j);
             dns[j] = d;
-            const float xv = IO<T>::load1(a.x, lbase + j);
+            const float xv = a.res_f32 ? IO<float>::load1(a.x, lbase + j)
+                                       : IO<T>::load1(a.x, lbase + j);
             const float xh = LN ? (xv - mean) * rstd : xv * rstd;
             const float gg = d * IO<T>::load1(a.gamma, j);
             sg += gg;
@@ -467,12 +481,19 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
         const float mgx = block_sum(sgx, red) * a.inv_h;
         for (int j = threadIdx.x; j < h; j += blockDim.x) {
             const float d = dns[j];
-            const float xv = IO<T>::load1(a.x, lbase + j);
+            const float xv = a.res_f32 ? IO<float>::load1(a.x, lbase + j)
+                                       : IO<T>::load1(a.x, lbase + j);
             const float xh = LN ? (xv - mean) * rstd : xv * rstd;
             const float gg = d * IO<T>::load1(a.gamma, j);
             const float dx = LN ? rstd * (gg - mg - xh * mgx) : rstd * (gg - xh * mgx);
-            const float dr = dx + (a.drnext ? IO<T>::load1(a.drnext, lbase + j) : 0.f);
-            IO<T>::store1(a.dres, lbase + j, dr);
+            float dr = dx;
+            if (a.res_f32) {
+                if (a.drnext) dr += IO<float>::load1(a.drnext, lbase + j);
+                IO<float>::store1(a.dres, lbase + j, dr);
+            } else {
+                if (a.drnext) dr += IO<T>::load1(a.drnext, lbase + j);
+                IO<T>::store1(a.dres, lbase + j, dr);
+            }
             uint32_t keep = 1u;
             if (a.mask) keep = (a.mask[(size_t)i_row * a.mask_row_bytes + (j >> 3)] >> (j & 7)) & 1u;
             const float dz = keep ? dr * a.scale : 0.f;

@@ -6,7 +6,7 @@
 // Partition Activations Alongside TP", sections "Normalize and add residuals
 // by token" and "Connect SP and TP across a layer"):
 //   reduce-scatter of the t partial sums -> + bias -> inverted dropout ->
-//   + residual (stored in the I/O dtype) -> LayerNorm / RMSNorm -> written to
+//   + residual (stored in the residual stream's dtype) -> LayerNorm / RMSNorm -> written to
 //   every gathered replica (the all-gather).
 //
 // k_fwd_tma: persistent, one CTA per SM.  The last warp is a producer: one
@@ -45,7 +45,9 @@ struct FwdArgs {
     int n_gathered;
     int stages;
     uint32_t seg_bytes;     // h * elem bytes
-    uint32_t stage_stride;  // seg_bytes rounded up to 128
+    uint32_t res_seg_bytes; // h * residual stream elem bytes (residual, residual_out)
+    int res_f32;            // residual stream in fp32 (I/O dtype bf16)
+    uint32_t stage_stride;  // largest segment rounded up to 128
     int mask_row_bytes;     // 4 * ceil(h / 32)
     uint32_t param_off;     // shared-memory offsets (fast kernel): parameters,
     uint32_t param_stride;  //   one slot of param_stride bytes each,
@@ -98,14 +100,16 @@ struct RingPos {
 // The producer lane: streams every segment of this CTA's rows, in row order.
 // Row j of the CTA belongs to consumer group j % G and goes to that group's
 // sub-ring (stages [g*Sg, (g+1)*Sg)).  nsrc sources per row; src(k, i) gives
-// the address of source k's segment for local row i.
+// the address of source k's segment for local row i.  Sources k >= k_split
+// (the residual stream's tensors) move seg2 bytes from slice_off2 instead.
 template <int G, typename SrcFn>
 __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail,
                                              volatile int* abort, long long rows,
                                              int nsrc, uint32_t seg_bytes,
                                              uint32_t stage_stride, int S, SrcFn src,
+                                             int k_split, uint32_t seg2,
                                              long long first = -1, long long stride = 0,
-                                             uint32_t slice_off = 0)
+                                             uint32_t slice_off = 0, uint32_t slice_off2 = 0)
 {
     // rows first, first + stride, ... (default: this CTA's blockIdx rows);
     // each copy moves seg_bytes starting slice_off bytes into the segment
@@ -138,10 +142,13 @@ __device__ __forceinline__ void ring_produce(unsigned char* smem, RingTail* tail
                     ok = false;
                     break;
                 }
-                const void* p = static_cast<const unsigned char*>(src(k, i)) + slice_off;
+                const bool second = k >= k_split;
+                const uint32_t nb = second ? seg2 : seg_bytes;
+                const void* p = static_cast<const unsigned char*>(src(k, i)) +
+                                (second ? slice_off2 : slice_off);
                 const uint32_t bar = smem_addr(&tail->full[st]);
-                mbar_arrive_expect_tx(bar, seg_bytes);
-                bulk_load(smem_addr(smem + (size_t)st * stage_stride), p, seg_bytes, bar, pol);
+                mbar_arrive_expect_tx(bar, nb);
+                bulk_load(smem_addr(smem + (size_t)st * stage_stride), p, nb, bar, pol);
                 ++issued[g];
                 if (++stage[g] == (uint32_t)Sg) {
                     stage[g] = 0;
@@ -216,6 +223,11 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
     const int hvc = a.hv / CS;                // vectors of this CTA's slice
     const int vg0 = (int)rank * hvc;          // first global vector of the slice
     const uint32_t slice_bytes = a.seg_bytes / CS;
+    const uint32_t res_slice_bytes = a.res_seg_bytes / CS;
+    // the fp32 residual stream is compiled out of the plans with the most
+    // live registers per thread (the host does not pick them for it)
+    constexpr bool kResF32 = !(V >= 4 && MAXT <= 544);
+    const bool res_f32 = kResF32 && a.res_f32;
 
     init_ring(tail, S, C / 32);
     if (CS > 1) cluster_sync_all();   // the peer's barriers exist before any remote arrive
@@ -229,9 +241,10 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
                                 return k < a.t ? static_cast<const unsigned char*>(a.parts[k]) +
                                                      (size_t)(a.row0 + i) * a.seg_bytes
                                                : static_cast<const unsigned char*>(a.residual) +
-                                                     (size_t)i * a.seg_bytes;
+                                                     (size_t)i * a.res_seg_bytes;
                             },
-                            cid, ncl, rank * slice_bytes);
+                            a.t, res_slice_bytes, cid, ncl, rank * slice_bytes,
+                            rank * res_slice_bytes);
     } else {
         // consumers: group g handles every G-th row of this CTA (cluster);
         // thread c of a group owns slice vectors v = c + i*C (8 features each)
@@ -340,18 +353,40 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
             if (mrow && c == 0 && rank == 0)
                 for (int pbyte = a.hv; pbyte < a.mask_row_bytes; ++pbyte) mrow[pbyte] = 0;
 
-            // residual add; the sum is stored in the I/O dtype and the norm
-            // reads the stored (rounded) value
+            // residual add; the sum is stored in the residual stream's dtype
+            // and the norm reads the stored (rounded) value
             mbar_wait(smem_addr(&tail->full[pos.abs()]), pos.phase, abort, ERR_WAIT_FULL);
             if (direct) {
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
 #pragma unroll
                 for (int i = 0; i < V; ++i)
-                    if (EXACT || c + i * C < hvc) IO<T>::unpack2(load_vec<T>(buf, c + i * C), acc[i]);
+                    if (EXACT || c + i * C < hvc) {
+                        if (res_f32)
+                            IO<float>::unpack2(load_vec<float>(buf, c + i * C), acc[i]);
+                        else
+                            IO<T>::unpack2(load_vec<T>(buf, c + i * C), acc[i]);
+                    }
+            } else if (res_f32) {
+                // fp32 residual stream: the sum is exact in its storage format
+                const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
+                unsigned char* rout =
+                    static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.res_seg_bytes;
+#pragma unroll
+                for (int i = 0; i < V; ++i) {
+                    const int v = c + i * C;
+                    if (EXACT || v < hvc) {
+                        F2 f[4];
+                        IO<float>::unpack2(load_vec<float>(buf, v), f);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) acc[i][p] = add2(f[p], acc[i][p]);
+                        if (a.residual_out)
+                            store_vec<float>(rout, vg0 + v, IO<float>::pack2v(acc[i]));
+                    }
+                }
             } else {
                 const unsigned char* buf = smem + (size_t)pos.abs() * a.stage_stride;
                 unsigned char* rout =
-                    static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.seg_bytes;
+                    static_cast<unsigned char*>(a.residual_out) + (size_t)i_row * a.res_seg_bytes;
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
                     const int v = c + i * C;
@@ -470,8 +505,14 @@ __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ Fwd
                 y = keep ? y * a.scale : 0.f;
             }
             if (keep) atomicOr(&mw[j >> 5], 1u << (j & 31));
-            const float r = IO<T>::round1(IO<T>::load1(a.residual, lbase + j) + y);
-            if (a.residual_out) IO<T>::store1(a.residual_out, lbase + j, r);
+            float r;
+            if (a.res_f32) {   // fp32 residual stream: the sum is its own rounding
+                r = IO<float>::load1(a.residual, lbase + j) + y;
+                if (a.residual_out) IO<float>::store1(a.residual_out, lbase + j, r);
+            } else {
+                r = IO<T>::round1(IO<T>::load1(a.residual, lbase + j) + y);
+                if (a.residual_out) IO<T>::store1(a.residual_out, lbase + j, r);
+            }
             xs[j] = r;
         }
         __syncthreads();

@@ -67,6 +67,7 @@ int check_cfg(const sp_cfg* c)
     if (!(c->row_begin == 0 && c->row_end == 0) &&
         !(c->row_begin >= 0 && c->row_begin < c->row_end && c->row_end <= c->s * c->b))
         return SP_ERR_INVALID_ARG;
+    if (c->res_f32 != 0 && c->res_f32 != 1) return SP_ERR_INVALID_ARG;
     return SP_OK;
 }
 
@@ -83,6 +84,9 @@ void call_rows(const sp_cfg* c, long long* r0, long long* nrows)
 }
 
 int elem_bytes(const sp_cfg* c) { return c->dtype == SP_F32 ? 4 : 2; }
+
+// bytes per element of the residual stream tensors (fp32 when res_f32)
+int res_elem_bytes(const sp_cfg* c) { return c->res_f32 ? 4 : elem_bytes(c); }
 
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
@@ -345,10 +349,12 @@ FastLaunch plan_fwd(FwdArgs& a, const DevInfo& dev, int E, int hint)
         const int id = order[oi];
         const Plan& p = kFwdPlans[id];
         if (a.hv % p.CS) continue;
+        if (a.res_f32 && p.V >= 4 && p.maxT <= 544) continue;   // compiled without it
         const int C = group_threads(a.hv / p.CS, p.V);
         if (p.G * C + 32 > p.maxT) continue;
         // each CTA stages and keeps parameters for its 1/CS of the row
-        const uint32_t stride = (uint32_t)round128(a.seg_bytes / p.CS);
+        const uint32_t seg_max = a.res_seg_bytes > a.seg_bytes ? a.res_seg_bytes : a.seg_bytes;
+        const uint32_t stride = (uint32_t)round128(seg_max / p.CS);
         const size_t pstride_c = round128((size_t)a.h * E / p.CS);
         long long S = ring_stages(dev.smem_optin, (long long)(tailb + 3 * pstride_c), stride);
         S -= S % p.G;                 // G sub-rings of S / G stages each
@@ -487,9 +493,14 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
         if (!gathered[q] || !aligned(gathered[q], E)) return SP_ERR_INVALID_ARG;
         all16 = all16 && aligned(gathered[q], 16);
     }
-    const void* elem_ptrs[] = {residual, gamma, residual_out, bias, ln ? beta : nullptr};
+    const int Er = res_elem_bytes(cfg);
+    const void* elem_ptrs[] = {gamma, bias, ln ? beta : nullptr};
     for (const void* p : elem_ptrs) {
         if (p && !aligned(p, E)) return SP_ERR_INVALID_ARG;
+        all16 = all16 && (!p || aligned(p, 16));
+    }
+    for (const void* p : {residual, (const void*)residual_out}) {   // the residual stream
+        if (p && !aligned(p, Er)) return SP_ERR_INVALID_ARG;
         all16 = all16 && (!p || aligned(p, 16));
     }
     if ((mask_bits && !aligned(mask_bits, 4)) || (mean && !aligned(mean, 4)) ||
@@ -521,7 +532,10 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
     a.t = nparts;
     a.n_gathered = n_gathered;
     a.seg_bytes = (uint32_t)(h * E);
-    a.stage_stride = (uint32_t)round128(a.seg_bytes);
+    a.res_seg_bytes = (uint32_t)(h * Er);
+    a.res_f32 = Er != E ? 1 : 0;
+    a.stage_stride = (uint32_t)round128(a.res_seg_bytes > a.seg_bytes ? a.res_seg_bytes
+                                                                       : a.seg_bytes);
     a.mask_row_bytes = 4 * ((h + 31) / 32);
     a.eps = cfg->eps;
     a.inv_h = (float)(1.0 / (double)h);
@@ -540,7 +554,7 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
 
     // the entry (no partial sums) without a plan hint: registers instead of
     // a staging ring, G groups of C threads per CTA
-    if (nparts == 0 && cfg->fwd_plan == 0 && h % 8 == 0 && all16) {
+    if (nparts == 0 && cfg->fwd_plan == 0 && !a.res_f32 && h % 8 == 0 && all16) {
         const int V = E == 2 ? 4 : 2;
         const int C = group_threads(h / 8, V);
         if (C <= kEntryThreads) {
@@ -704,9 +718,14 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
         if (!dn_partials[k] || !aligned(dn_partials[k], E)) return SP_ERR_INVALID_ARG;
         all16 = all16 && aligned(dn_partials[k], 16);
     }
-    const void* elem_ptrs[] = {dR_next, residual_out, gamma, dresidual_in, dY};
+    const int Er = res_elem_bytes(cfg);
+    const void* elem_ptrs[] = {gamma, dY};
     for (const void* p : elem_ptrs) {
         if (p && !aligned(p, E)) return SP_ERR_INVALID_ARG;
+        all16 = all16 && (!p || aligned(p, 16));
+    }
+    for (const void* p : {dR_next, residual_out, (const void*)dresidual_in}) {   // residual stream
+        if (p && !aligned(p, Er)) return SP_ERR_INVALID_ARG;
         all16 = all16 && (!p || aligned(p, 16));
     }
     const void* f4_ptrs[] = {mask_bits, mean, rstd, dgamma, dbeta, dbias};
@@ -738,7 +757,10 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     a.hv = h / 8;
     a.t = cfg->t;
     a.seg_bytes = (uint32_t)(h * E);
-    a.stage_stride = (uint32_t)round128(a.seg_bytes);
+    a.res_seg_bytes = (uint32_t)(h * Er);
+    a.res_f32 = Er != E ? 1 : 0;
+    a.stage_stride = (uint32_t)round128(a.res_seg_bytes > a.seg_bytes ? a.res_seg_bytes
+                                                                       : a.seg_bytes);
     a.mask_row_bytes = 4 * ((h + 31) / 32);
     a.inv_h = (float)(1.0 / (double)h);
     a.scale = 1.0f / (1.0f - cfg->p_drop);

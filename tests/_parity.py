@@ -118,7 +118,7 @@ def cfg_of(w, fwd_plan=0, bwd_plan=0):
     return sp.make_cfg(w.s, w.b, w.h, w.t, dtype=w.dtype, norm=w.norm,
                        eps=w.eps, p_drop=w.p_drop, seed=w.drop_seed,
                        offset=w.drop_offset, fwd_plan=fwd_plan,
-                       bwd_plan=bwd_plan)
+                       bwd_plan=bwd_plan, res_f32=w.res != w.dtype)
 
 
 def gpu_fwd(w, parts, bias, residual, gamma, beta, n_gathered=1,
@@ -130,25 +130,26 @@ def gpu_fwd(w, parts, bias, residual, gamma, beta, n_gathered=1,
     16-byte boundary (exercises the general kernel)."""
     dev = "cuda"
     dt = w.torch_dtype
+    rdt = w.res_torch_dtype
     N, h = w.rows, w.h
     W = (h + 31) // 32
 
-    def dcopy(x):
+    def dcopy(x, dtype=dt):
         if x is None:
             return None, None
-        g = Guarded(tuple(x.shape), dt, dev, offset_elems)
+        g = Guarded(tuple(x.shape), dtype, dev, offset_elems)
         g.t.copy_(x.to(dev))
         return g, g.t
 
     gp = [dcopy(p) for p in parts]
-    gres, res_t = dcopy(residual)
+    gres, res_t = dcopy(residual, rdt)
     gb = dcopy(bias)[1]
     gg = dcopy(gamma)[1]
     gbe = dcopy(beta)[1]
     if inplace:
         rout_g, rout = gres, res_t
     else:
-        rout_g = Guarded((N, h), dt, dev, offset_elems)
+        rout_g = Guarded((N, h), rdt, dev, offset_elems)
         rout = rout_g.t
     gath = [Guarded((N, h), dt, dev, offset_elems) for _ in range(n_gathered)]
     mask_g = Guarded((N, W), torch.int32, dev) if with_mask else None
@@ -185,9 +186,10 @@ def gpu_bwd(w, dparts, drnext, x, gamma, mask, mean, rstd, with_dbeta=True,
         g.t.copy_(torch.as_tensor(x_).to(dev))
         return g.t
 
+    rdt = w.res_torch_dtype
     dp = [dcopy(p) for p in dparts]
-    drn = dcopy(drnext)
-    xt = dcopy(x)
+    drn = dcopy(drnext, rdt)
+    xt = dcopy(x, rdt)
     gt = dcopy(gamma)
     mt = (None if mask is None else
           dcopy(torch.from_numpy(np.ascontiguousarray(mask).view(np.int32)),
@@ -197,7 +199,7 @@ def gpu_bwd(w, dparts, drnext, x, gamma, mask, mean, rstd, with_dbeta=True,
                     torch.float32, 0))
     rstd_t = dcopy(torch.from_numpy(np.asarray(rstd, np.float32)),
                    torch.float32, 0)
-    dres_g = Guarded((N, h), dt, dev, offset_elems)
+    dres_g = Guarded((N, h), w.res_torch_dtype, dev, offset_elems)
     dy_g = Guarded((N, h), dt, dev, offset_elems)
     dgam_g = Guarded((h,), torch.float32, dev)
     dbet_g = Guarded((h,), torch.float32, dev) if with_dbeta else None
@@ -295,7 +297,7 @@ def check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered=1,
     """Compare a device forward with the oracle's (same rows)."""
     dt = w.torch_dtype
     assert_close("residual_out", got["residual_out"], ref["residual_out"],
-                 mag_residual_out(w, parts, bias, res), dt)
+                 mag_residual_out(w, parts, bias, res), w.res_torch_dtype)
     ex_o, ex_m, ex_r = propagated_dx(w, got["residual_out"],
                                      ref["residual_out"], ref["mean"],
                                      ref["rstd"], gamma)
