@@ -60,6 +60,7 @@ struct BwdArgs {
     int want_dbeta;
     int want_dbias;
     uint32_t tmem_cols;      // tensor-memory columns allocated (ACC = 2)
+    int fold;                // ACC = 2, G > 1: the groups' sums are added in the CTA
 };
 
 // ACC: where the per-CTA parameter-gradient partials live.  0: registers,
@@ -387,7 +388,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 
     // partial sums -> workspace: register accumulators give one slice per
     // group ([cta * G + g][q][h]); the shared set gives one slice per CTA
-    // ([cta][q][h]), written by group 0 once every group has finished
+    // ([cta][q][h]), written by group 0 once every group has finished; the
+    // tensor-memory sets give one per group, or one per CTA when folded
     if (ACC_SMEM) {
         if (G > 1) asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
         if (g != 0) return;
@@ -396,38 +398,87 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         __syncwarp();
         tmem_wait_st();
     }
-    float* ws = a.ws + (ACC_SMEM ? (size_t)blockIdx.x : (size_t)blockIdx.x * G + g) * 3 * a.h;
+    // tensor-memory sums of a thread, vector i: 24 words (dgamma, dbeta, dbias)
+    auto tmem_sums = [&](int i, uint32_t tr[24]) {   // warp-wide
+        __syncwarp();
+        tmem_ld16(tacc + 24 * i, tr);
+        tmem_ld8(tacc + 24 * i + 16, tr + 16);
+    };
+    auto pair_of = [](const uint32_t* r) {   // 4 words -> two fp32 pairs
+        return make_ulonglong2(f2(__uint_as_float(r[0]), __uint_as_float(r[1])).r,
+                               f2(__uint_as_float(r[2]), __uint_as_float(r[3])).r);
+    };
+    if (ACC_TMEM && G > 1 && a.fold) {
+        // One slice per CTA: once every row is consumed the ring is idle;
+        // groups 1..G-1 stage their sums there ([g-1][q][2][hv] of 16
+        // bytes) and group 0 adds them to its own in group order.
+        ulonglong2* stg = reinterpret_cast<ulonglong2*>(smem);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
+        if (g > 0) {
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-        const int v = c + i * C;
-        uint32_t tr[24];
-        if (ACC_TMEM) {   // warp-wide
-            __syncwarp();
-            tmem_ld16(tacc + 24 * i, tr);
-            tmem_ld8(tacc + 24 * i + 16, tr + 16);
+            for (int i = 0; i < V; ++i) {
+                const int v = c + i * C;
+                uint32_t tr[24];
+                tmem_sums(i, tr);
+                if (EXACT || v < hv)
+                    for (int q = 0; q < 3; ++q) {
+                        ulonglong2* d = stg + ((size_t)(g - 1) * 3 + q) * 2 * hv;
+                        d[v] = pair_of(tr + 8 * q);
+                        d[hv + v] = pair_of(tr + 8 * q + 4);
+                    }
+            }
         }
-        if (EXACT || v < hv) {
-            for (int q = 0; q < 3; ++q) {
-                ulonglong2 lo, hi;
-                if (ACC_SMEM) {
-                    lo = accs[((size_t)q * 2 + 0) * hv + v];
-                    hi = accs[((size_t)q * 2 + 1) * hv + v];
-                } else if (ACC_TMEM) {
-                    const uint32_t* r = tr + 8 * q;
-                    lo = make_ulonglong2(f2(__uint_as_float(r[0]), __uint_as_float(r[1])).r,
-                                         f2(__uint_as_float(r[2]), __uint_as_float(r[3])).r);
-                    hi = make_ulonglong2(f2(__uint_as_float(r[4]), __uint_as_float(r[5])).r,
-                                         f2(__uint_as_float(r[6]), __uint_as_float(r[7])).r);
-                } else {
-                    const F2* s_ = q == 0 ? ag[ACC_REGS ? i : 0]
-                                          : (q == 1 ? ab[ACC_REGS ? i : 0]
-                                                    : ac[ACC_REGS ? i : 0]);
-                    lo = make_ulonglong2(s_[0].r, s_[1].r);
-                    hi = make_ulonglong2(s_[2].r, s_[3].r);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + kMaxGroups), "r"(G * C) : "memory");
+        if (g == 0) {
+            float* wsc = a.ws + (size_t)blockIdx.x * 3 * a.h;
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                const int v = c + i * C;
+                uint32_t tr[24];
+                tmem_sums(i, tr);
+                if (EXACT || v < hv)
+                    for (int q = 0; q < 3; ++q) {
+                        ulonglong2 lo = pair_of(tr + 8 * q), hi = pair_of(tr + 8 * q + 4);
+                        for (int gg = 1; gg < G; ++gg) {
+                            const ulonglong2* d = stg + ((size_t)(gg - 1) * 3 + q) * 2 * hv;
+                            const ulonglong2 x = d[v], y = d[hv + v];
+                            lo = make_ulonglong2(add2(F2{lo.x}, F2{x.x}).r, add2(F2{lo.y}, F2{x.y}).r);
+                            hi = make_ulonglong2(add2(F2{hi.x}, F2{y.x}).r, add2(F2{hi.y}, F2{y.y}).r);
+                        }
+                        ulonglong2* dst =
+                            reinterpret_cast<ulonglong2*>(wsc + (size_t)q * a.h + 8 * (size_t)v);
+                        dst[0] = lo;
+                        dst[1] = hi;
+                    }
+            }
+        }
+    } else {
+        float* ws = a.ws + (ACC_SMEM ? (size_t)blockIdx.x : (size_t)blockIdx.x * G + g) * 3 * a.h;
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const int v = c + i * C;
+            uint32_t tr[24];
+            if (ACC_TMEM) tmem_sums(i, tr);
+            if (EXACT || v < hv) {
+                for (int q = 0; q < 3; ++q) {
+                    ulonglong2 lo, hi;
+                    if (ACC_SMEM) {
+                        lo = accs[((size_t)q * 2 + 0) * hv + v];
+                        hi = accs[((size_t)q * 2 + 1) * hv + v];
+                    } else if (ACC_TMEM) {
+                        lo = pair_of(tr + 8 * q);
+                        hi = pair_of(tr + 8 * q + 4);
+                    } else {
+                        const F2* s_ = q == 0 ? ag[ACC_REGS ? i : 0]
+                                              : (q == 1 ? ab[ACC_REGS ? i : 0]
+                                                        : ac[ACC_REGS ? i : 0]);
+                        lo = make_ulonglong2(s_[0].r, s_[1].r);
+                        hi = make_ulonglong2(s_[2].r, s_[3].r);
+                    }
+                    ulonglong2* dst = reinterpret_cast<ulonglong2*>(ws + (size_t)q * a.h + 8 * (size_t)v);
+                    dst[0] = lo;
+                    dst[1] = hi;
                 }
-                ulonglong2* dst = reinterpret_cast<ulonglong2*>(ws + (size_t)q * a.h + 8 * (size_t)v);
-                dst[0] = lo;
-                dst[1] = hi;
             }
         }
     }

@@ -180,7 +180,7 @@ constexpr int kFwdEntryOrder[] = {13, 12, 11, 10, 4, 9, 6, 8, 1, 2, 0, 3, 5, 7, 
 // backward: tensor-memory accumulators first; they leave shared memory to the
 // ring (measured on B200 for bf16 rows of h = 12288, t = 16: 2 -> 8 stages,
 // 4.9 -> 6.6 TB/s)
-constexpr int kBwdOrder[] = {19, 15, 16, 18, 17, 21, 20, 22, 11, 8, 9, 12,
+constexpr int kBwdOrder[] = {19, 15, 18, 16, 17, 21, 20, 22, 11, 8, 9, 12,
                              2, 3, 5, 10, 6, 1, 0, 4, 7, 13, 14};
 
 int group_threads(int hv, int V)
@@ -409,6 +409,11 @@ FastLaunch plan_bwd(BwdArgs& a, const DevInfo& dev, int E, int hint)
         if (S < 2 * p.G) continue;
         a.stages = (int)S;
         a.tmem_cols = tcols;
+        // tensor-memory groups fold their sums in the CTA when the staging
+        // ((G-1) x 3 x 2 planes of 16 bytes per vector) fits in the ring
+        a.fold = (p.acc == 2 && p.G > 1 &&
+                  (size_t)(p.G - 1) * 96 * (size_t)a.hv <= (size_t)S * a.stage_stride)
+                     ? 1 : 0;
         a.param_off = (uint32_t)(S * a.stage_stride);
         a.acc_off = (uint32_t)(a.param_off + pstride);
         a.tail_off = (uint32_t)(a.acc_off + accb);
@@ -773,7 +778,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
     if (h % 8 == 0 && all16) {
         const FastLaunch L = plan_bwd(a, dev, E, cfg->bwd_plan);
         if (L.plan >= 0) {
-            nparts = (long long)L.grid * (kBwdPlans[L.plan].acc == 1 ? 1 : L.groups);
+            nparts = (long long)L.grid * ((kBwdPlans[L.plan].acc == 1 || a.fold) ? 1 : L.groups);
             if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes)
                 return SP_ERR_INVALID_ARG;
             const void* kern = ln ? bwd_kernel_dt<true>(cfg->dtype, L.plan, L.exact)
