@@ -98,6 +98,7 @@ def _fake_call_fwd(lib, cfg, t, n_gathered=1, ptr=0x1000):
     dict(eps=0.0), dict(eps=float("inf")),
     dict(dtype=7), dict(norm=5),
     dict(s=2 ** 33, t=1),         # token row beyond the 32-bit counter
+    dict(res_f32=2), dict(res_f32=-1),   # residual-stream flag is 0 or 1
 ])
 def test_forward_validation_rejects_before_launch(lib, bad):
     import sp_region_b200 as sp
@@ -160,3 +161,27 @@ def test_all_gather_validation(lib):
     cfg.s = 7
     assert lib.sp_all_gather(ctypes.byref(cfg), sh, outs, 1, None) == \
         sp.SP_ERR_INVALID_ARG
+
+
+def test_fp32_residual_stream_needs_fp32_alignment(lib):
+    """With res_f32 the residual-stream tensors are fp32: a pointer aligned
+    for bf16 only is rejected before any launch, forward and backward."""
+    import sp_region_b200 as sp
+    cfg = sp.make_cfg(8, 2, 64, 4, dtype="bf16", p_drop=0.0, res_f32=True)
+    A, M = ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1002)
+    parts = (ctypes.c_void_p * 4)(*([0x1000] * 4))
+    outs = (ctypes.c_void_p * 1)(0x1000)
+    for residual, rout in ((M, A), (A, M)):
+        rc = lib.sp_rs_bias_dropout_add_norm_fwd(
+            ctypes.byref(cfg), parts, None, residual, A, None, rout, outs, 1,
+            None, None, None, None)
+        assert rc == sp.SP_ERR_INVALID_ARG
+    rc = lib.sp_norm_all_gather_fwd(ctypes.byref(cfg), M, A, None, outs, 1,
+                                    None, None, None)
+    assert rc == sp.SP_ERR_INVALID_ARG
+    # backward: x (residual_out), dR_next and dresidual_in are fp32
+    for drn, x, dres in ((M, A, A), (A, M, A), (A, A, M)):
+        rc = lib.sp_rs_norm_dropout_bwd(ctypes.byref(cfg), parts, drn, x, A,
+                                        None, A, A, dres, A, A, None, None, A,
+                                        1 << 20, None)
+        assert rc == sp.SP_ERR_INVALID_ARG
