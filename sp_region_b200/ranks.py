@@ -48,13 +48,17 @@ class Rendezvous:
     arrive(tag) publishes this rank's arrival and waits, at most timeout_s,
     for every rank's.  fail(exc) publishes this rank's failure, so that the
     others stop waiting at once.  Every call uses fresh keys (a per-instance
-    sequence number), so points can repeat."""
+    sequence number), so points can repeat.  Once every rank has arrived at a
+    point, every rank is done waiting at the one before, so each rank then
+    deletes its own key of that earlier point: the store stays small over a
+    long run."""
 
     def __init__(self, store, rank: int, world: int, timeout_s: float = 30.0,
                  prefix: str = "sp_boundary", poll_s: float = 0.005):
         self.store, self.rank, self.world = store, rank, world
         self.timeout_s, self.prefix, self.poll_s = timeout_s, prefix, poll_s
         self.seq = 0
+        self._last_key = None
 
     def _key(self, seq: int, tag: str, r: int) -> str:
         return f"{self.prefix}/{seq}/{tag}/{r}"
@@ -75,6 +79,9 @@ class Rendezvous:
         while True:
             missing = [r for r, k in enumerate(want) if not self.store.check([k])]
             if not missing:
+                if self._last_key is not None:
+                    self.store.delete_key(self._last_key)
+                self._last_key = want[self.rank]
                 return
             failed = self._failures()
             if failed or time.monotonic() > deadline:

@@ -101,8 +101,14 @@ def _worker(rank, port, scenario, bufs, q):
         dg, db = torch.empty(H), torch.empty(H)
         sb.backward(cfg, bufs["dparts"], None, rout, None, None, None, None, dres,
                     dY, dg, db, None, None)
+        # the store keeps only each rank's key of the latest rendezvous
+        rdv = sb.rdv
+        old_keys = [rdv._key(q_, tag, rank) for q_, tag in
+                    ((0, "forward inputs written"), (1, "forward outputs pushed"),
+                     (2, "backward inputs written"))]
+        kept = [k for k in old_keys if rdv.store.check([k])]
         q.put((rank, "ok", gathered_ok, bool((dY == 30.0).all()),
-               dg.tolist(), db.tolist(), bool((dres == 30.0).all())))
+               dg.tolist(), db.tolist(), bool((dres == 30.0).all()), kept))
     finally:
         dist.destroy_process_group()
 
@@ -133,8 +139,9 @@ def _run(scenario):
 def test_two_ranks_order_the_pushes_and_sum_parameter_gradients():
     out = _run("ok")
     for r in range(WORLD):
-        kind, gathered_ok, dy_ok, dg, db, dres_ok = out[r]
+        kind, gathered_ok, dy_ok, dg, db, dres_ok, kept = out[r]
         assert kind == "ok"
+        assert kept == [], "keys of earlier rendezvous left in the store"
         assert gathered_ok, "gathered read before the peer's rows landed"
         assert dy_ok and dres_ok
         assert dg == [3.0] * H and db == [30.0] * H
