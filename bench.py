@@ -557,14 +557,26 @@ def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
 # the CPU oracle (baseline leg and reference arm)
 # ----------------------------------------------------------------------------
 
-def _oracle_rows(w, row0, nrows, orc, sp_synth, cfg):
+_DRAWN = {}
+
+
+def _oracle_rows(w, row0, nrows, orc, sp_synth, cfg, reuse=False):
     """Oracle forward + backward on token rows [row0, row0 + nrows), inputs
-    drawn on the host with the workload's recipe (rows seeded by row0)."""
-    ww = w.replace(seed=w.seed + 7919 * (row0 + 1))
-    parts = sp_synth.draw_partials(ww, rows=nrows)
-    bias, gamma, beta = sp_synth.draw_params(w)
-    res = sp_synth.draw_residual(ww, rows=nrows)
-    dparts = sp_synth.draw_grad_partials(ww, rows=nrows)
+    drawn on the host with the workload's recipe (rows seeded by row0).
+    reuse=True draws one sample of nrows rows per process and runs it for
+    every row0 (the oracle's work per row does not depend on the values);
+    only the oracle's own time is returned either way."""
+    key = (repr(w), nrows)
+    if reuse and key in _DRAWN:
+        parts, bias, gamma, beta, res, dparts = _DRAWN[key]
+    else:
+        ww = w.replace(seed=w.seed + 7919 * (row0 + 1))
+        parts = sp_synth.draw_partials(ww, rows=nrows)
+        bias, gamma, beta = sp_synth.draw_params(w)
+        res = sp_synth.draw_residual(ww, rows=nrows)
+        dparts = sp_synth.draw_grad_partials(ww, rows=nrows)
+        if reuse:
+            _DRAWN[key] = (parts, bias, gamma, beta, res, dparts)
     ids = list(range(row0, row0 + nrows))
     t0 = time.perf_counter()
     fo = orc.fwd_rows(cfg, ids, parts, bias, res, gamma, beta)
@@ -576,10 +588,19 @@ def _oracle_rows(w, row0, nrows, orc, sp_synth, cfg):
 def _oracle_chunk(job):
     """One job of the all-cores baseline, in a spawned worker process: the
     oracle on rows [row0, row0 + nrows) of a workload (compute time)."""
-    w, row0, nrows = job
+    w, row0, nrows, reuse = job
+    import torch
+    torch.set_num_threads(1)   # one process per core
     import oracle as orc
     import sp_synth
-    return _oracle_rows(w, row0, nrows, orc, sp_synth, orc.cfg_from(w))
+    return _oracle_rows(w, row0, nrows, orc, sp_synth, orc.cfg_from(w), reuse)
+
+
+def _host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
 
 
 def cpu_baseline_all_cores(w, fb, bb, budget_s=10.0, max_procs=64):
@@ -587,21 +608,17 @@ def cpu_baseline_all_cores(w, fb, bb, budget_s=10.0, max_procs=64):
     (spawned, never forked from a process that touched the GPU).  Throughput
     counts each batch at its slowest worker's compute time."""
     import multiprocessing as mp
-    try:
-        ncpu = len(os.sched_getaffinity(0))
-    except AttributeError:
-        ncpu = os.cpu_count() or 1
-    procs = max(1, min(ncpu, max_procs))
+    procs = max(1, min(_host_cores(), max_procs))
     per_row = (fb + bb) / w.rows
     chunk = 64
     rows_done, secs, row0 = 0, 0.0, 0
     with mp.get_context("spawn").Pool(procs) as pool:
-        pool.map(_oracle_chunk, [(w, 0, 1)] * procs)   # imports, oracle load
+        pool.map(_oracle_chunk, [(w, 0, 1, False)] * procs)   # imports, oracle load
         while secs < budget_s and row0 < w.rows:
             jobs = []
             while len(jobs) < procs and row0 < w.rows:
                 n = min(chunk, w.rows - row0)
-                jobs.append((w, row0, n))
+                jobs.append((w, row0, n, False))
                 row0 += n
             secs += max(pool.map(_oracle_chunk, jobs))
             rows_done += sum(j[2] for j in jobs)
@@ -647,17 +664,34 @@ def run_reference(args):
     cfg = orc.cfg_from(w)
     fb, bb = fwd_bytes(w), bwd_bytes(w)
     per_row = (fb + bb) / w.rows
-    # per-step sample sized so that warm-up + timed steps take ~2 minutes
+    procs = max(1, min(args.reference_cores or _host_cores(), 64))
+    # per-step sample sized so that warm-up + timed steps take ~2 minutes;
+    # with several processes a step is one batch of rows on every process,
+    # timed at its slowest worker
     t_row = _oracle_rows(w, 0, 8, orc, sp_synth, cfg) / 8
-    rows = int(max(1, min(256, 120.0 / max(1, args.steps + args.warmup)
-                          / max(t_row, 1e-6))))
-    for i in range(args.warmup):
-        _oracle_rows(w, (i * rows) % w.rows, min(rows, w.rows), orc, sp_synth,
-                     cfg)
+    per_proc = int(max(1, min(256, 120.0 / max(1, args.steps + args.warmup)
+                              / max(t_row, 1e-6))))
+    per_proc = min(per_proc, max(1, w.rows // procs))
+    rows = per_proc * procs
+
+    def step_jobs(i):
+        base = (i * rows) % max(1, w.rows - rows + 1)
+        return [(w, base + k * per_proc, per_proc, True) for k in range(procs)]
+
     secs = 0.0
-    for i in range(args.steps):
-        r0 = ((args.warmup + i) * rows) % max(1, w.rows - rows + 1)
-        secs += _oracle_rows(w, r0, rows, orc, sp_synth, cfg)
+    if procs == 1:
+        for i in range(args.warmup + args.steps):
+            (wj, r0, n, reuse), = step_jobs(i)
+            t = _oracle_rows(wj, r0, n, orc, sp_synth, cfg, reuse)
+            if i >= args.warmup:
+                secs += t
+    else:
+        import multiprocessing as mp
+        with mp.get_context("spawn").Pool(procs) as pool:
+            for i in range(args.warmup + args.steps):
+                t = max(pool.map(_oracle_chunk, step_jobs(i)))
+                if i >= args.warmup:
+                    secs += t
     value = per_row * rows * args.steps / secs / 1e9
     line = {
         "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
@@ -674,8 +708,9 @@ def run_reference(args):
                    "s": w.s, "b": w.b, "h": w.h, "t": w.t,
                    "sample_rows_per_step": rows},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s",
-                         "cores": 1, "kind": "oracle",
-                         "sample": f"{rows} token rows of {w.name} per step, "
+                         "cores": procs, "kind": "oracle",
+                         "sample": f"{rows} token rows of {w.name} per step "
+                                   f"({per_proc} on each of {procs} processes), "
                                    "forward + backward"},
         "e2e": {"value": round(value, 4), "unit": "GB/s",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -696,6 +731,8 @@ def main():
                          "+ epilogue + all-gather); entry: norm + all-gather")
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--reference-cores", type=int, default=0,
+                    help="processes for --impl reference (0: every core, up to 64)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
     ap.add_argument("--residual-f32", action="store_true",
                     help="keep the residual stream in fp32 beside bf16 I/O")
