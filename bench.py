@@ -110,10 +110,13 @@ def measured_peak():
 
 
 def kernel_sources_sha():
+    """Hash of every source the library is built from (csrc/*, the header)."""
     h = hashlib.sha1()
-    for f in ("sp_region.cu", "sp_device.cuh", "sp_fwd.cuh", "sp_bwd.cuh",
-              "sp_gather.cuh", "sp_entry.cuh"):
-        with open(os.path.join(ROOT, "sp_region_b200", "csrc", f), "rb") as fh:
+    csrc = os.path.join(ROOT, "sp_region_b200", "csrc")
+    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc)
+                   if f.endswith((".cu", ".cuh", ".h")))
+    for f in files + [os.path.join(ROOT, "include", "sp_region.h")]:
+        with open(f, "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:12]
 

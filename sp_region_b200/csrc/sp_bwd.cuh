@@ -559,7 +559,8 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
 // partials.  A block covers 32 consecutive columns of one quantity: lane =
 // column, warp w sums partials w, w+8, w+16, ... in order, then warp 0 adds
 // the 8 warp totals in order.  Deterministic for a given partial count.
-__global__ void __launch_bounds__(256)
+// (static: one copy per translation unit that launches it)
+static __global__ void __launch_bounds__(256)
     k_colreduce(const float* __restrict__ ws, int nparts, int h, float* dgamma, float* dbeta,
                 float* dbias)
 {

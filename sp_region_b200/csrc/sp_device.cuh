@@ -12,9 +12,25 @@ namespace spk {
 // ---------------------------------------------------------------------------
 // Device-side error word.  A bounded wait that runs out records its code here
 // (first error wins) and the kernel winds down instead of hanging; the host
-// reads it with sp_device_error().
+// reads it with sp_device_error().  Each translation unit of the library is
+// its own device module with its own word (static); SPK_ERROR_WORD_ACCESSOR
+// defines the host function that reads and clears the word of the unit it
+// is expanded in.
 // ---------------------------------------------------------------------------
-__device__ unsigned int g_error;
+static __device__ unsigned int g_error;
+
+#define SPK_ERROR_WORD_ACCESSOR(NAME)                                                \
+    int NAME(unsigned* v, int clear)                                                 \
+    {                                                                                \
+        if (cudaMemcpyFromSymbol(v, g_error, sizeof(unsigned)) != cudaSuccess)       \
+            return -1;                                                               \
+        if (clear) {                                                                 \
+            const unsigned zero = 0;                                                 \
+            if (cudaMemcpyToSymbol(g_error, &zero, sizeof(zero)) != cudaSuccess)     \
+                return -1;                                                           \
+        }                                                                            \
+        return 0;                                                                    \
+    }
 
 enum : unsigned {
     ERR_WAIT_FULL = 1,      // a consumer waited too long for a staged row

@@ -14,8 +14,13 @@
 #include "sp_entry.cuh"
 #include "sp_fwd.cuh"
 #include "sp_gather.cuh"
+#include "sp_plans.h"
 
 using namespace spk;
+
+namespace spk {
+SPK_ERROR_WORD_ACCESSOR(error_word_host)
+}  // namespace spk
 
 namespace {
 
@@ -103,67 +108,6 @@ long long general_grid(long long rows, int sms)
     return rows < g ? rows : g;
 }
 
-// ---------------------------------------------------------------------------
-// Fast-kernel plans: V vectors of 8 features per consumer thread, G consumer
-// groups (each takes every G-th row of the CTA), at most maxT threads (which
-// sets the register budget), and for the backward the parameter-gradient
-// partials in registers or shared memory.  A group needs
-// C = 32 * ceil(ceil(hv / V) / 32) threads; a launch has G*C + 32.
-// ---------------------------------------------------------------------------
-struct Plan {
-    int V, G, maxT;
-    int acc;   // backward parameter-gradient partials: 0 registers, 1 shared, 2 tensor memory
-    int CS;   // CTAs per token row (a thread-block cluster when 2)
-};
-
-constexpr Plan kFwdPlans[] = {
-    {1, 1, 1024, 0, 1},   // 0
-    {1, 2, 800, 0, 1},    // 1
-    {1, 4, 1024, 0, 1},   // 2
-    {2, 1, 544, 0, 1},    // 3
-    {2, 2, 800, 0, 1},    // 4
-    {3, 1, 544, 0, 1},    // 5
-    {3, 2, 800, 0, 1},    // 6
-    {4, 1, 544, 0, 1},    // 7
-    {4, 2, 800, 0, 1},    // 8
-    {2, 3, 800, 0, 1},    // 9
-    {4, 4, 544, 0, 1},    // 10
-    {4, 6, 800, 0, 1},    // 11
-    {3, 3, 800, 0, 1},    // 12
-    {4, 4, 800, 0, 1},    // 13
-    {1, 2, 800, 0, 2},    // 14
-    {2, 2, 800, 0, 2},    // 15
-    {2, 1, 544, 0, 2},    // 16
-    {1, 1, 1024, 0, 2},   // 17
-    {4, 1, 544, 0, 2},    // 18
-};
-constexpr Plan kBwdPlans[] = {
-    {1, 1, 1024, 0, 1},   // 0
-    {1, 1, 800, 0, 1},    // 1
-    {1, 2, 800, 0, 1},    // 2
-    {2, 1, 544, 1, 1},     // 3
-    {2, 1, 800, 0, 1},    // 4
-    {3, 1, 544, 1, 1},     // 5
-    {4, 1, 544, 1, 1},     // 6
-    {2, 1, 544, 0, 1},    // 7
-    {2, 2, 800, 1, 1},     // 8
-    {3, 2, 800, 1, 1},     // 9
-    {4, 2, 800, 1, 1},     // 10
-    {2, 3, 800, 1, 1},     // 11
-    {4, 4, 544, 1, 1},     // 12
-    {3, 3, 800, 1, 1},     // 13
-    {4, 4, 800, 1, 1},     // 14
-    {2, 2, 800, 2, 1},        // 15
-    {3, 2, 800, 2, 1},        // 16
-    {3, 1, 544, 2, 1},        // 17
-    {2, 1, 800, 2, 1},        // 18
-    {4, 4, 544, 2, 1},        // 19
-    {2, 3, 800, 2, 1},        // 20
-    {4, 1, 544, 2, 1},        // 21
-    {2, 1, 544, 2, 1},        // 22
-};
-constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
-constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);
 
 // Preference order when the caller gives no hint: the first feasible plan
 // wins.  A hinted plan is tried first.  Plans that split a row across a
@@ -196,41 +140,6 @@ long long ring_stages(long long smem_optin, long long fixed, uint32_t stage_stri
     return S > 64 ? 64 : S;
 }
 
-#define SP_FWD_CASE(ID)                                                                 \
-    case ID:                                                                            \
-        return (const void*)k_fwd_tma<T, kFwdPlans[ID].V, kFwdPlans[ID].G,              \
-                                      kFwdPlans[ID].maxT, LN, kFwdPlans[ID].CS, EXACT>;
-
-template <typename T, bool LN, bool EXACT>
-const void* fwd_kernel(int id)
-{
-    switch (id) {
-        SP_FWD_CASE(0) SP_FWD_CASE(1) SP_FWD_CASE(2) SP_FWD_CASE(3) SP_FWD_CASE(4)
-        SP_FWD_CASE(5) SP_FWD_CASE(6) SP_FWD_CASE(7) SP_FWD_CASE(8) SP_FWD_CASE(9)
-        SP_FWD_CASE(10) SP_FWD_CASE(11) SP_FWD_CASE(12) SP_FWD_CASE(13) SP_FWD_CASE(14)
-        SP_FWD_CASE(15) SP_FWD_CASE(16) SP_FWD_CASE(17) SP_FWD_CASE(18)
-    }
-    return nullptr;
-}
-
-#define SP_BWD_CASE(ID)                                                                 \
-    case ID:                                                                            \
-        return (const void*)k_bwd_tma<T, kBwdPlans[ID].V, kBwdPlans[ID].G,              \
-                                      kBwdPlans[ID].maxT, LN, kBwdPlans[ID].acc, EXACT>;
-
-template <typename T, bool LN, bool EXACT>
-const void* bwd_kernel(int id)
-{
-    switch (id) {
-        SP_BWD_CASE(0) SP_BWD_CASE(1) SP_BWD_CASE(2) SP_BWD_CASE(3) SP_BWD_CASE(4)
-        SP_BWD_CASE(5) SP_BWD_CASE(6) SP_BWD_CASE(7) SP_BWD_CASE(8) SP_BWD_CASE(9)
-        SP_BWD_CASE(10) SP_BWD_CASE(11) SP_BWD_CASE(12) SP_BWD_CASE(13) SP_BWD_CASE(14)
-        SP_BWD_CASE(15) SP_BWD_CASE(16) SP_BWD_CASE(17) SP_BWD_CASE(18) SP_BWD_CASE(19)
-        SP_BWD_CASE(20) SP_BWD_CASE(21) SP_BWD_CASE(22)
-    }
-    return nullptr;
-}
-
 // entry kernel: V = 4 vectors per thread in bf16, 2 in fp32 (registers)
 template <typename T>
 const void* entry_kernel_t(bool ln, bool exact)
@@ -243,24 +152,18 @@ const void* entry_kernel_t(bool ln, bool exact)
                  : (const void*)k_norm_ag<T, V, false, false>;
 }
 
-template <bool LN>
-const void* fwd_kernel_dt(int dtype, int id, bool exact)
+// kernel of a fast plan for the I/O dtype and norm (defined by the
+// instantiation units sp_inst_fwd.cu / sp_inst_bwd.cu)
+const void* fwd_kernel_of(int dtype, bool ln, int id, bool exact)
 {
-    if (exact)
-        return dtype == SP_BF16 ? fwd_kernel<__nv_bfloat16, LN, true>(id)
-                                : fwd_kernel<float, LN, true>(id);
-    return dtype == SP_BF16 ? fwd_kernel<__nv_bfloat16, LN, false>(id)
-                            : fwd_kernel<float, LN, false>(id);
+    if (dtype == SP_BF16) return ln ? fwd_kernel_bf16_ln(id, exact) : fwd_kernel_bf16_rms(id, exact);
+    return ln ? fwd_kernel_f32_ln(id, exact) : fwd_kernel_f32_rms(id, exact);
 }
 
-template <bool LN>
-const void* bwd_kernel_dt(int dtype, int id, bool exact)
+const void* bwd_kernel_of(int dtype, bool ln, int id, bool exact)
 {
-    if (exact)
-        return dtype == SP_BF16 ? bwd_kernel<__nv_bfloat16, LN, true>(id)
-                                : bwd_kernel<float, LN, true>(id);
-    return dtype == SP_BF16 ? bwd_kernel<__nv_bfloat16, LN, false>(id)
-                            : bwd_kernel<float, LN, false>(id);
+    if (dtype == SP_BF16) return ln ? bwd_kernel_bf16_ln(id, exact) : bwd_kernel_bf16_rms(id, exact);
+    return ln ? bwd_kernel_f32_ln(id, exact) : bwd_kernel_f32_rms(id, exact);
 }
 
 int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream_t st,
@@ -593,8 +496,7 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
     if (h % 8 == 0 && all16) {
         const FastLaunch L = plan_fwd(a, dev, E, cfg->fwd_plan);
         if (L.plan >= 0) {
-            const void* kern = ln ? fwd_kernel_dt<true>(cfg->dtype, L.plan, L.exact)
-                                  : fwd_kernel_dt<false>(cfg->dtype, L.plan, L.exact);
+            const void* kern = fwd_kernel_of(cfg->dtype, ln, L.plan, L.exact);
             if (L.cs > 1) {
                 int grid = 0;
                 return launch_clusters(kern, rows, L.cs, L.block, L.smem, st, &a, &grid);
@@ -781,8 +683,7 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
             nparts = (long long)L.grid * ((kBwdPlans[L.plan].acc == 1 || a.fold) ? 1 : L.groups);
             if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes)
                 return SP_ERR_INVALID_ARG;
-            const void* kern = ln ? bwd_kernel_dt<true>(cfg->dtype, L.plan, L.exact)
-                                  : bwd_kernel_dt<false>(cfg->dtype, L.plan, L.exact);
+            const void* kern = bwd_kernel_of(cfg->dtype, ln, L.plan, L.exact);
             if ((rc = launch_kernel(kern, L.grid, L.block, L.smem, st, &a))) return rc;
             launched = true;
         }
@@ -815,13 +716,21 @@ int sp_device_error(int32_t device, int32_t* code, int32_t clear)
         cudaGetLastError();
         return SP_ERR_INVALID_ARG;
     }
-    unsigned v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_error, sizeof(v)) != cudaSuccess) return SP_ERR_CUDA;
-    *code = (int32_t)v;
-    if (clear) {
-        const unsigned zero = 0;
-        if (cudaMemcpyToSymbol(g_error, &zero, sizeof(zero)) != cudaSuccess) return SP_ERR_CUDA;
+    // every unit's word, in a fixed order; the first nonzero one is reported
+    int (*const words[])(unsigned*, int) = {
+        error_word_host,         error_word_fwd_bf16_ln, error_word_fwd_bf16_rms,
+        error_word_fwd_f32_ln,   error_word_fwd_f32_rms, error_word_bwd_bf16_ln,
+        error_word_bwd_bf16_rms, error_word_bwd_f32_ln,  error_word_bwd_f32_rms};
+    unsigned first = 0;
+    for (auto fn : words) {
+        unsigned v = 0;
+        if (fn(&v, clear) != 0) {
+            cudaGetLastError();
+            return SP_ERR_CUDA;
+        }
+        if (!first) first = v;
     }
+    *code = (int32_t)first;
     return SP_OK;
 }
 
