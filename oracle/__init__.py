@@ -92,7 +92,8 @@ def _lib():
         L.orc_bwd.argtypes = [vp, vp, vp, vp, vp, vp, dp, dp, vp, vp, dp, dp,
                               dp]
         L.orc_bwd.restype = ctypes.c_int
-        L.orc_bwd_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, dp, dp, vp, vp]
+        L.orc_bwd_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, dp, dp, vp, vp,
+                                   dp, dp, dp]
         L.orc_bwd_rows.restype = ctypes.c_int
         L.orc_activation_bytes.argtypes = [i64, i64, i64, i64, i32, i32,
                                            ctypes.c_double]
@@ -329,8 +330,10 @@ def bwd(cfg: Cfg, dparts, drnext, x, gamma, mask, mean, rstd,
 
 
 def bwd_rows(cfg: Cfg, dpart_rows, drnext_rows, x_rows, gamma, mask_rows,
-             mean, rstd) -> dict:
-    """Backward on selected rows (per-row outputs only)."""
+             mean, rstd, with_params: bool = False) -> dict:
+    """Backward on selected rows.  with_params: also return the rows' share
+    of dgamma / dbeta / dbias (float64 sums over these rows; summing the
+    shares of a partition of all tokens gives the full gradients)."""
     dt, rdt = cfg.dtype, cfg.res_dtype
     tdt = _torch_dtype(dt)
     ps = [_cpu(p, dt) for p in dpart_rows]
@@ -344,10 +347,15 @@ def bwd_rows(cfg: Cfg, dpart_rows, drnext_rows, x_rows, gamma, mask_rows,
     rstd = np.ascontiguousarray(rstd, np.float64)
     dres = torch.empty((n, h), dtype=_torch_dtype(rdt))
     dY = torch.empty((n, h), dtype=tdt)
+    pg = [np.zeros(h) for _ in range(3)] if with_params else [None] * 3
     rc = _lib().orc_bwd_rows(ctypes.byref(cfg), n, _ptr_array(ps),
                              _ptr(drnext_rows), _ptr(x_rows), _ptr(gamma),
                              _ptr(mask_rows), mean.ctypes.data,
-                             rstd.ctypes.data, _ptr(dres), _ptr(dY))
+                             rstd.ctypes.data, _ptr(dres), _ptr(dY),
+                             *(_ptr(g) for g in pg))
     if rc != 0:
         raise ValueError(f"oracle backward rejected the configuration ({rc})")
-    return dict(dresidual_in=dres, dY=dY)
+    out = dict(dresidual_in=dres, dY=dY)
+    if with_params:
+        out.update(dgamma=pg[0], dbeta=pg[1], dbias=pg[2])
+    return out

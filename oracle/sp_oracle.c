@@ -540,13 +540,17 @@ int orc_bwd(const orc_cfg* c, const void* const* dparts, const void* drnext,
 }
 
 /*
- * Backward on selected rows (no parameter gradients: those are sums over all
- * tokens).  Inputs and outputs are [nrows, ...] in sample order.
+ * Backward on selected rows.  Inputs and outputs are [nrows, ...] in sample
+ * order.  dgamma, dbeta, dbias (each [h] or NULL) receive the chunk's share
+ * of the parameter gradients, the sums over these rows only in sample order;
+ * the parameters are replicated, so the gradient over all tokens is the sum
+ * of the chunks' shares (the same all-reduce orc_bwd performs over ranks).
  */
 int orc_bwd_rows(const orc_cfg* c, int64_t nrows, const void* const* dparts,
                  const void* drnext, const void* x, const void* gamma,
                  const uint32_t* mask, const double* mean, const double* rstd,
-                 void* dres_in, void* dY)
+                 void* dres_in, void* dY, double* dgamma, double* dbeta,
+                 double* dbias)
 {
     if (!cfg_ok(c)) return -1;
     const int64_t h = c->h, W = orc_mask_words(h);
@@ -568,6 +572,11 @@ int orc_bwd_rows(const orc_cfg* c, int64_t nrows, const void* const* dparts,
                        (c->norm == ORC_LAYERNORM) ? mean[i] : 0.0, rstd[i],
                        dres_in, dz, acc, acc + h, acc + 2 * h, xhat);
         for (int64_t j = 0; j < h; ++j) st(dY, i * h + j, c->dtype, dz[j]);
+    }
+    for (int64_t j = 0; j < h; ++j) {
+        if (dgamma) dgamma[j] = acc[j];
+        if (dbeta) dbeta[j] = acc[h + j];
+        if (dbias) dbias[j] = acc[2 * h + j];
     }
     free(dn); free(xhat); free(dz); free(acc);
     return 0;

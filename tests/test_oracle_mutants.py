@@ -81,6 +81,12 @@ MUTANTS = {
     "residual gradient stored in the I/O dtype": (
         "st(dres_in, row * h + j, c->res_dtype, dr);",
         "st(dres_in, row * h + j, c->dtype, dr);"),
+    "entry mean stored at the rank-local row": (
+        "if (mean) mean[n] = mu;", "if (mean) mean[i] = mu;"),
+    "entry rstd stored at the rank-local row": (
+        "if (rstd) rstd[n] = rs;", "if (rstd) rstd[i] = rs;"),
+    "row-chunk shares: dbeta reported as dgamma": (
+        "if (dgamma) dgamma[j] = acc[j];", "if (dgamma) dgamma[j] = acc[h + j];"),
     "ring volume without (t-1)/t": (
         "double phase = (double)(t - 1) / (double)t * V;",
         "double phase = V;"),

@@ -552,6 +552,48 @@ def test_backward_rows_agrees_with_full(orc):
     assert np.array_equal(fr["mask"], fo["mask"][rows])
 
 
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+def test_backward_rows_parameter_shares_match_autograd(orc, norm):
+    """The rows' shares of dgamma / dbeta / dbias: each chunk's share equals
+    torch autograd's parameter gradient of the loss over that chunk's rows
+    alone, and the shares of a partition of all rows add up to autograd's
+    full gradient (float64)."""
+    w = sp_synth.WORKLOADS["C2"].replace(s=12, b=2, h=48, t=4, norm=norm,
+                                          dtype="f32", p_drop=0.25,
+                                          has_beta=norm == "layernorm")
+    cfg = orc.cfg_from(w)
+    parts = sp_synth.draw_partials(w)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    res = sp_synth.draw_residual(w)
+    fo = orc.fwd(cfg, parts, bias, res, gamma, beta)
+    dparts = sp_synth.draw_grad_partials(w)
+    dn = torch.stack([d.double() for d in dparts]).sum(0)
+    y = torch.stack([p.double() for p in parts]).sum(0)
+    chunks = [list(range(0, 7)), list(range(7, 8)), list(range(8, 24))]
+    total = {k: np.zeros(w.h) for k in ("dgamma", "dbeta", "dbias")}
+    for rows in chunks:
+        sh = orc.bwd_rows(cfg, [d[rows] for d in dparts], None,
+                          fo["residual_out"][rows], gamma, fo["mask"][rows],
+                          None if fo["mean"] is None else fo["mean"][rows],
+                          fo["rstd"][rows], with_params=True)
+        only = torch.zeros_like(dn)
+        only[rows] = dn[rows]      # the loss restricted to this chunk
+        ref = _torch_reference_grads(w, y, bias, fo["residual_out"], gamma,
+                                     beta, fo["mask"], only, None)
+        for k in total:
+            if ref[k] is None:
+                continue
+            assert np.allclose(sh[k], ref[k].numpy(), rtol=1e-10,
+                               atol=1e-12), (k, rows)
+            total[k] += sh[k]
+    full = _torch_reference_grads(w, y, bias, fo["residual_out"], gamma, beta,
+                                  fo["mask"], dn, None)
+    for k in total:
+        if full[k] is not None:
+            assert np.allclose(total[k], full[k].numpy(), rtol=1e-10,
+                               atol=1e-12), k
+
+
 # ----------------------------------------------------------------------------
 # activation-memory closed forms
 # ----------------------------------------------------------------------------
@@ -630,6 +672,34 @@ def test_entry_norm_matches_torch_and_gathers_in_rank_order(orc, norm):
     fo = orc.fwd(orc.cfg_from(w, p_drop=0.0), [torch.zeros_like(x)] * w.t, None, x,
                  gamma, beta)
     assert torch.equal(fo["gathered"][0], out["gathered"][0])
+
+
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+def test_entry_statistics_match_torch_var_mean(orc, norm):
+    """The entry's per-token statistics at t = 4, indexed by global token row:
+    mean and biased variance from torch.var_mean in float64, rstd =
+    1/sqrt(var + eps) (LayerNorm) or 1/sqrt(mean(x^2) + eps) (RMSNorm)."""
+    w = sp_synth.WORKLOADS["C2"].replace(s=16, b=2, h=72, t=4, norm=norm,
+                                          dtype="bf16")
+    cfg = orc.cfg_from(w)
+    x = sp_synth.draw_residual(w)
+    # rows of very different scale, so a statistic stored at the wrong row
+    # cannot pass by chance
+    x = (x.float() * torch.arange(1, w.rows + 1,
+                                  dtype=torch.float32)[:, None]).to(x.dtype)
+    bias, gamma, beta = sp_synth.draw_params(w)
+    beta = beta if norm == "layernorm" else None
+    out = orc.norm_ag_fwd(cfg, x, gamma, beta)
+    xd = x.double()
+    eps = float(np.float32(w.eps))
+    if norm == "layernorm":
+        var, mu = torch.var_mean(xd, dim=1, unbiased=False)
+        assert np.allclose(out["mean"], mu.numpy(), rtol=1e-13, atol=1e-13)
+        rstd = 1.0 / torch.sqrt(var + eps)
+    else:
+        assert out["mean"] is None
+        rstd = 1.0 / torch.sqrt(xd.pow(2).mean(1) + eps)
+    assert np.allclose(out["rstd"], rstd.numpy(), rtol=1e-13, atol=0)
 
 
 # ----------------------------------------------------------------------------
