@@ -48,7 +48,7 @@ FALLBACK_HBM_GBS = 6650.0
 
 # E: bytes per element of the I/O dtype; Er: of the residual stream
 # (residual, residual_out, x, dR_next, dresidual_in), fp32 with --residual-f32
-def fwd_bytes(w, n_gathered=1):
+def fwd_bytes(w, n_gathered=1, with_mask=True):
     E, Er, N, h = w.elem_bytes, w.res_elem_bytes, w.rows, w.h
     sbh = N * h
     W = (h + 31) // 32
@@ -56,8 +56,13 @@ def fwd_bytes(w, n_gathered=1):
                       (1 if (w.has_beta and w.norm == "layernorm") else 0))
     rd = w.t * E * sbh + Er * sbh + params
     stats = (8 if w.norm == "layernorm" else 4) * N
-    wr = Er * sbh + E * sbh * n_gathered + 4 * W * N + stats
+    wr = Er * sbh + E * sbh * n_gathered + (4 * W * N if with_mask else 0) + stats
     return rd + wr
+
+
+def all_gather_bytes(w, n_out):
+    """Standalone all-gather: every shard read once, written n_out times."""
+    return w.elem_bytes * w.rows * w.h * (1 + n_out)
 
 
 def bwd_bytes(w, with_drnext=False):
@@ -379,8 +384,11 @@ def run_ours(args):
 
     e2e = None
     cpu = None
+    workloads = None
     if args.op == "boundary":
         e2e = run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world)
+        if world == 1 and args.workloads:
+            workloads = time_workloads(args, sp, torch, dev, peak)
         if rank == 0 and world == 1 and not args.skip_cpu_baseline:
             cpu = cpu_baseline(w, fb, bb, budget_s=args.cpu_seconds)
 
@@ -411,6 +419,7 @@ def run_ours(args):
         "pct_of_measured_peak": round(100 * value / world / peak, 2),
         "roofline": roofline,
         "kernels": kern,
+        "workloads": workloads,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 3 * K,
@@ -422,6 +431,114 @@ def run_ours(args):
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def time_launches(torch, stream, fn, steps, warmup):
+    """Average device time of one call of fn, from CUDA events recorded on
+    the launching stream around each of `steps` calls (after `warmup`)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in evs:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.mean(a.elapsed_time(b) for a, b in evs)
+
+
+def time_workloads(args, sp, torch, dev, peak):
+    """Forward and backward of every workload at full size (C2 to C5), each
+    timed on its own with CUDA events, plus C3's forward with the all-gather
+    written as t per-rank replicas and the standalone all-gather into t
+    replicas.  Inputs are resident in HBM and larger than L2."""
+    import gc
+    import sp_synth
+    out = {}
+    stream = torch.cuda.current_stream(dev)
+    for name in args.workloads.split(","):
+        if not name:
+            continue
+        w = sp_synth.WORKLOADS[name]
+        N, h, t = w.rows, w.h, w.t
+        dt = w.torch_dtype
+        cfg = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm,
+                          eps=w.eps, p_drop=w.p_drop, seed=w.drop_seed,
+                          offset=w.drop_offset)
+        parts = sp_synth.draw_partials(w, dev)
+        bias, gamma, beta = sp_synth.draw_params(w, dev)
+        if not w.has_bias:
+            bias = None
+        if not w.has_beta or w.norm == "rmsnorm":
+            beta = None
+        res = sp_synth.draw_residual(w, dev)
+        with_mask = w.p_drop > 0
+        rout = torch.empty((N, h), dtype=dt, device=dev)
+        gath = [torch.empty((N, h), dtype=dt, device=dev)
+                for _ in range(t if w.gather_replicas else 1)]
+        mask = (torch.empty((N, (h + 31) // 32), dtype=torch.int32,
+                            device=dev) if with_mask else None)
+        mean = torch.empty(N, dtype=torch.float32, device=dev)
+        rstd = torch.empty(N, dtype=torch.float32, device=dev)
+        rec = {"workload": f"{name}: s={w.s} b={w.b} h={h} t={t} {w.dtype} "
+                           f"{w.norm} p={w.p_drop}"
+                           + (" bias" if w.has_bias else "")
+                           + (" 1% x100 outliers" if w.outliers else "")}
+        K = 10 if N * h > 2e8 else 40
+
+        def entry(kernel, nbytes, ms):
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            return {"kernel": kernel, "bytes_per_launch": nbytes,
+                    "avg_ms": round(ms, 5), "gbs": round(gbs, 1),
+                    "frac": round(gbs / peak, 4),
+                    "pct_of_8TBs": round(100 * gbs / NOMINAL_HBM_GBS, 2)}
+
+        def fwd(n=1):
+            sp.sp_rs_bias_dropout_add_norm_fwd(cfg, parts, bias, res, gamma,
+                                               beta, rout, gath[:n], mask,
+                                               mean if w.norm == "layernorm"
+                                               else None, rstd, stream=stream)
+        ms = time_launches(torch, stream, fwd, K, 3)
+        rec["fwd"] = entry("k_fwd_tma", fwd_bytes(w, 1, with_mask), ms)
+        if w.gather_replicas:
+            ms = time_launches(torch, stream, lambda: fwd(t), K, 3)
+            rec["fwd_all_gather_replicas"] = entry(
+                "k_fwd_tma (t gathered replicas)", fwd_bytes(w, t, with_mask),
+                ms)
+            shards = [gath[0][r * (N // t):(r + 1) * (N // t)]
+                      for r in range(t)]
+            ms = time_launches(torch, stream, lambda: sp.sp_all_gather(
+                cfg, shards, gath[1:], stream=stream), K, 3)
+            rec["all_gather"] = entry(f"k_all_gather ({t - 1} replicas)",
+                                      all_gather_bytes(w, t - 1), ms)
+        del parts
+        gc.collect()
+        dparts = sp_synth.draw_grad_partials(w, dev)
+        dres = torch.empty((N, h), dtype=dt, device=dev)
+        dY = torch.empty((N, h), dtype=dt, device=dev)
+        dg = torch.empty(h, dtype=torch.float32, device=dev)
+        db = torch.empty(h, dtype=torch.float32, device=dev) \
+            if w.norm == "layernorm" else None
+        dc = torch.empty(h, dtype=torch.float32, device=dev) \
+            if bias is not None else None
+        ws = torch.empty(sp.sp_bwd_workspace_bytes(cfg, dev.index) // 4,
+                         dtype=torch.float32, device=dev)
+
+        def bwd():
+            sp.sp_rs_norm_dropout_bwd(cfg, dparts, None, rout, gamma, mask,
+                                      mean if w.norm == "layernorm" else None,
+                                      rstd, dres, dY, dg, db, dc, ws,
+                                      stream=stream)
+        ms = time_launches(torch, stream, bwd, K, 3)
+        rec["bwd"] = entry("k_bwd_tma + k_colreduce", bwd_bytes(w), ms)
+        out[name] = rec
+        del dparts, dres, dY, rout, gath, res, ws
+        gc.collect()
+        torch.cuda.empty_cache()
+    assert sp.sp_device_error(dev.index) == 0, "device-side wait timed out"
+    return out
 
 
 def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
@@ -737,6 +854,9 @@ def main():
     ap.add_argument("--reference-cores", type=int, default=0,
                     help="processes for --impl reference (0: every core, up to 64)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="C2,C3,C4,C5",
+                    help="after the timed steps, time the forward and backward "
+                         "of these workloads one by one (N = 1; '' for none)")
     ap.add_argument("--residual-f32", action="store_true",
                     help="keep the residual stream in fp32 beside bf16 I/O")
     ap.add_argument("--fwd-plan", type=int, default=0,

@@ -273,7 +273,8 @@ int sp_all_gather(const sp_cfg* cfg, const void* const* shards,
  *                the entry into a TP region has no dropout input)
  *   dgamma [h] fp32; dbeta [h] fp32 or NULL; dbias [h] fp32 or NULL
  *   workspace    device scratch of at least sp_bwd_workspace_bytes() bytes,
- *                16-byte aligned; no initial contents needed
+ *                16-byte aligned; no initial contents needed.  Calls that
+ *                overlap on the GPU must not share a workspace.
  * The parameter gradients are deterministic: per-CTA partial sums in a
  * fixed order, then one fixed-order sum over CTAs.
  */
@@ -286,7 +287,15 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
                            size_t workspace_bytes, void* stream);
 
 /* Bytes of device scratch sp_rs_norm_dropout_bwd needs for cfg on CUDA
- * device `device` (it depends on the device's SM count).  Host-only. */
+ * device `device`: the slices of 3*h fp32 parameter-gradient partial sums
+ * that the kernel the call picks writes, for 16-byte aligned pointers or for
+ * misaligned ones (the general kernel), whichever is more.  With the
+ * library's own plan choice that is one slice per CTA, min(s*b, SMs) slices
+ * (one per SM at most); a plan hint (cfg->bwd_plan) may pick a plan with
+ * one slice per consumer group (up to 4 per CTA).  Host-only; it reads the
+ * device's SM count and shared-memory limit.  SP_ERR_UNSUPPORTED when no
+ * backward kernel takes the shape.  Departs from a plain size_t return so
+ * that it can report errors like every other call. */
 int sp_bwd_workspace_bytes(const sp_cfg* cfg, int32_t device, size_t* bytes);
 
 /*
@@ -339,12 +348,19 @@ int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream);
  * is a 64 MiB array of this library's device image, reserved on every GPU
  * that loads the library and held until the process exits.
  *
- * Limit   a configuration whose sp_bwd_workspace_bytes() exceeds 64 MiB is
- *         rejected with SP_ERR_UNSUPPORTED before any launch (on a 148-SM
- *         B200 that is h > 9447).
- * Set-up  the first call on a device looks up the array's device address
- *         (cudaGetSymbolAddress) and caches it; make that first call before
- *         any stream capture.
+ * Limit   the call picks its kernel for the given pointers exactly as
+ *         sp_rs_norm_dropout_bwd does; if the scratch that kernel writes
+ *         (its slices times 12*h bytes) exceeds 64 MiB, it returns
+ *         SP_ERR_UNSUPPORTED before any launch.  With the library's own plan
+ *         choice a call writes min(s*b, SMs) slices, so on a 148-SM B200
+ *         every shape with h <= 37786 fits (the fast kernels take h up to
+ *         16384 in bf16 and fp32; the general kernel up to about 57000).  A
+ *         plan hint that picks one slice per consumer group divides the
+ *         limit by the group count.
+ * Set-up  every call looks up the array's device address on the current
+ *         device (cudaGetSymbolAddress); the first call on a device also
+ *         loads the library's device code there, so make it before any
+ *         stream capture.
  * Sharing every call on a device uses the same array and leaves its
  *         contents behind; the kernels write every part of it they read, so
  *         nothing needs clearing, but calls that overlap on the GPU (other

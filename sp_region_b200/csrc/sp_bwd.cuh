@@ -494,11 +494,12 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
     }
 }
 
-// General backward: any h.  One CTA per row (grid stride); the reduced dn row
-// lives in shared memory, the CTA's parameter-gradient partials in its own
-// workspace slice (zeroed first, owned column by column by one thread each).
+// General backward: any h.  One CTA per row (grid stride over at most one CTA
+// per SM); the reduced dn row lives in shared memory, the CTA's
+// parameter-gradient partials in its own workspace slice (zeroed first, owned
+// column by column by one thread each).
 template <typename T, bool LN>
-__global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ BwdArgs a)
+__global__ void __launch_bounds__(1024) k_bwd_general(const __grid_constant__ BwdArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     float* dns = reinterpret_cast<float*>(smem);
@@ -555,19 +556,26 @@ __global__ void __launch_bounds__(256) k_bwd_general(const __grid_constant__ Bwd
     }
 }
 
-// dgamma / dbeta / dbias: fixed-order sum of the per-CTA (per-group)
-// partials.  A block covers 32 consecutive columns of one quantity: lane =
-// column, warp w sums partials w, w+8, w+16, ... in order, then warp 0 adds
-// the 8 warp totals in order.  Deterministic for a given partial count.
+// dgamma / dbeta / dbias: fixed-order sum of the nparts workspace slices
+// ([nparts][3][h] fp32).  A block covers 32 consecutive columns of one
+// quantity with kColreduceWarps warps: lane = column; warp w sums slices w,
+// w + W, w + 2W, ... in ascending order, loading up to 16 of them at once so
+// that their latencies overlap; then warp 0 adds the W warp totals in warp
+// order.  Deterministic for a given slice count.
 // (static: one copy per translation unit that launches it)
-static __global__ void __launch_bounds__(256)
+constexpr int kColreduceWarps = 16;
+
+static __global__ void __launch_bounds__(kColreduceWarps * 32)
     k_colreduce(const float* __restrict__ ws, int nparts, int h, float* dgamma, float* dbeta,
                 float* dbias)
 {
-    __shared__ float part[8][33];
+    constexpr int W = kColreduceWarps;
+    constexpr int kBatch = 16;
+    __shared__ float part[W][33];
     const int tiles = (h + 31) / 32;
     const int q = blockIdx.x / tiles;
-    const int j = (blockIdx.x - q * tiles) * 32 + (threadIdx.x & 31);
+    const int lane = threadIdx.x & 31;
+    const int j = (blockIdx.x - q * tiles) * 32 + lane;
     const int w = threadIdx.x >> 5;
     float* out = q == 0 ? dgamma : (q == 1 ? dbeta : dbias);
     if (!out) return;   // uniform over the block
@@ -575,22 +583,24 @@ static __global__ void __launch_bounds__(256)
     if (j < h) {
         const float* p = ws + (size_t)q * h + j;
         const size_t stride = (size_t)3 * h;
-        int k = w;
-        for (; k + 24 < nparts; k += 32) {
-            const float v0 = p[(size_t)k * stride], v1 = p[(size_t)(k + 8) * stride];
-            const float v2 = p[(size_t)(k + 16) * stride], v3 = p[(size_t)(k + 24) * stride];
-            s += v0;
-            s += v1;
-            s += v2;
-            s += v3;
+        for (int k0 = w; k0 < nparts; k0 += kBatch * W) {
+            float v[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int k = k0 + u * W;
+                v[u] = k < nparts ? __ldcg(p + (size_t)k * stride) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                if (k0 + u * W < nparts) s += v[u];
         }
-        for (; k < nparts; k += 8) s += p[(size_t)k * stride];
     }
-    part[w][threadIdx.x & 31] = s;
+    part[w][lane] = s;
     __syncthreads();
     if (w == 0 && j < h) {
         float t = 0.f;
-        for (int i = 0; i < 8; ++i) t += part[i][threadIdx.x];
+#pragma unroll
+        for (int i = 0; i < W; ++i) t += part[i][lane];
         out[j] = t;
     }
 }

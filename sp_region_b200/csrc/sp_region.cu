@@ -6,7 +6,6 @@
 #include <string.h>
 
 #include <algorithm>
-#include <mutex>
 
 #include "sp_region.h"
 #include "sp_bwd.cuh"
@@ -520,6 +519,159 @@ int fwd_impl(const sp_cfg* cfg, int nparts, const void* const* partials, const v
 
 }  // namespace
 
+namespace {
+// ---------------------------------------------------------------------------
+// Backward launch decision, shared by the two backward entry points and the
+// workspace query: the kernel, its launch shape and the workspace slices
+// (3 * h fp32 each) it writes.
+// ---------------------------------------------------------------------------
+constexpr int kBwdGeneralThreads = 1024;
+
+struct BwdChoice {
+    bool fast = false;
+    FastLaunch L;            // fast kernel: plan, block, grid, shared memory
+    long long slices = 0;    // workspace slices written
+    size_t general_smem = 0;
+};
+
+// The shape fields of the backward's arguments (everything but pointers).
+void bwd_shape(const sp_cfg* cfg, BwdArgs* a)
+{
+    memset(a, 0, sizeof(*a));
+    long long row0 = 0, rows = 0;
+    call_rows(cfg, &row0, &rows);
+    const int h = (int)cfg->h;
+    const int E = elem_bytes(cfg), Er = res_elem_bytes(cfg);
+    a->rows = rows;
+    a->row0 = row0;
+    a->h = h;
+    a->hv = h / 8;
+    a->t = cfg->t;
+    a->seg_bytes = (uint32_t)(h * E);
+    a->res_seg_bytes = (uint32_t)(h * Er);
+    a->res_f32 = Er != E ? 1 : 0;
+    a->stage_stride = (uint32_t)round128(a->res_seg_bytes > a->seg_bytes ? a->res_seg_bytes
+                                                                          : a->seg_bytes);
+    a->mask_row_bytes = 4 * ((h + 31) / 32);
+    a->inv_h = (float)(1.0 / (double)h);
+    a->scale = 1.0f / (1.0f - cfg->p_drop);
+}
+
+// fast_ok: every [s,b,h] pointer is 16-byte aligned.  Fills the planner's
+// fields of *a (stages, offsets, fold).  SP_ERR_UNSUPPORTED when no kernel
+// takes the shape.
+int choose_bwd(const sp_cfg* cfg, const DevInfo& dev, bool fast_ok, BwdArgs& a, BwdChoice* ch)
+{
+    *ch = BwdChoice();
+    const int h = (int)cfg->h;
+    if (fast_ok && h % 8 == 0) {
+        const FastLaunch L = plan_bwd(a, dev, elem_bytes(cfg), cfg->bwd_plan);
+        if (L.plan >= 0) {
+            ch->fast = true;
+            ch->L = L;
+            // one slice per CTA (shared-memory sums, or tensor-memory sums
+            // folded in the CTA), else one per consumer group
+            ch->slices = (long long)L.grid *
+                         ((kBwdPlans[L.plan].acc == 1 || a.fold) ? 1 : L.groups);
+            return SP_OK;
+        }
+    }
+    const size_t smem = (size_t)h * 4;
+    if (smem > (size_t)dev.smem_optin - 1024) return SP_ERR_UNSUPPORTED;
+    ch->general_smem = smem;
+    ch->slices = a.rows < dev.sms ? a.rows : dev.sms;   // one CTA per SM at most
+    return SP_OK;
+}
+
+int noalloc_scratch(int dev, size_t need, void** out);
+
+// The backward; workspace == nullptr takes the scratch from the library's
+// fixed device array (sp_rs_norm_dropout_bwd_noalloc).
+int bwd_impl(const sp_cfg* cfg, const void* const* dn_partials, const void* dR_next,
+             const void* residual_out, const void* gamma, const uint32_t* mask_bits,
+             const float* mean, const float* rstd, void* dresidual_in, void* dY, float* dgamma,
+             float* dbeta, float* dbias, void* workspace, size_t workspace_bytes, void* stream)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    const bool ln = cfg->norm == SP_LAYERNORM;
+    if (!dn_partials || !residual_out || !gamma || !rstd || !dresidual_in || !dgamma)
+        return SP_ERR_INVALID_ARG;
+    if (ln && !mean) return SP_ERR_INVALID_ARG;
+    if (!mask_bits && cfg->p_drop > 0.0f) return SP_ERR_INVALID_ARG;
+    const int E = elem_bytes(cfg);
+    bool all16 = true;
+    for (int k = 0; k < cfg->t; ++k) {
+        if (!dn_partials[k] || !aligned(dn_partials[k], E)) return SP_ERR_INVALID_ARG;
+        all16 = all16 && aligned(dn_partials[k], 16);
+    }
+    const int Er = res_elem_bytes(cfg);
+    const void* elem_ptrs[] = {gamma, dY};
+    for (const void* p : elem_ptrs) {
+        if (p && !aligned(p, E)) return SP_ERR_INVALID_ARG;
+        all16 = all16 && (!p || aligned(p, 16));
+    }
+    for (const void* p : {dR_next, residual_out, (const void*)dresidual_in}) {   // residual stream
+        if (p && !aligned(p, Er)) return SP_ERR_INVALID_ARG;
+        all16 = all16 && (!p || aligned(p, 16));
+    }
+    const void* f4_ptrs[] = {mask_bits, mean, rstd, dgamma, dbeta, dbias};
+    for (const void* p : f4_ptrs)
+        if (p && !aligned(p, 4)) return SP_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return SP_ERR_INVALID_ARG;
+
+    DevInfo dev;
+    if ((rc = use_device_of(residual_out, &dev))) return rc;
+
+    const int h = (int)cfg->h;
+    BwdArgs a;
+    bwd_shape(cfg, &a);
+    BwdChoice ch;
+    if ((rc = choose_bwd(cfg, dev, all16, a, &ch))) return rc;
+    const size_t need = (size_t)ch.slices * 3 * h * sizeof(float);
+    if (!workspace) {
+        if ((rc = noalloc_scratch(dev.id, need, &workspace))) return rc;
+    } else if (need > workspace_bytes) {
+        return SP_ERR_INVALID_ARG;
+    }
+    for (int k = 0; k < cfg->t; ++k) a.dparts[k] = dn_partials[k];
+    a.drnext = dR_next;
+    a.x = residual_out;
+    a.gamma = gamma;
+    a.mask = reinterpret_cast<const uint8_t*>(mask_bits);
+    a.mean = ln ? mean : nullptr;
+    a.rstd = rstd;
+    a.dres = dresidual_in;
+    a.dY = dY;
+    a.ws = static_cast<float*>(workspace);
+    a.want_dbeta = (ln && dbeta) ? 1 : 0;
+    a.want_dbias = dbias ? 1 : 0;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+    if (ch.fast) {
+        const void* kern = bwd_kernel_of(cfg->dtype, ln, ch.L.plan, ch.L.exact);
+        if ((rc = launch_kernel(kern, ch.L.grid, ch.L.block, ch.L.smem, st, &a))) return rc;
+    } else {
+        const void* kern;
+        if (cfg->dtype == SP_BF16)
+            kern = ln ? (const void*)k_bwd_general<__nv_bfloat16, true>
+                      : (const void*)k_bwd_general<__nv_bfloat16, false>;
+        else
+            kern = ln ? (const void*)k_bwd_general<float, true>
+                      : (const void*)k_bwd_general<float, false>;
+        if ((rc = launch_kernel(kern, (int)ch.slices, kBwdGeneralThreads, ch.general_smem, st,
+                                &a)))
+            return rc;
+    }
+    const int tiles = (h + 31) / 32;
+    k_colreduce<<<3 * tiles, kColreduceWarps * 32, 0, st>>>(
+        a.ws, (int)ch.slices, h, dgamma, a.want_dbeta ? dbeta : nullptr,
+        a.want_dbias ? dbias : nullptr);
+    return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+}  // namespace
+
 extern "C" {
 
 int sp_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, const void* const* partials,
@@ -589,19 +741,26 @@ int sp_bwd_workspace_bytes(const sp_cfg* cfg, int32_t device, size_t* bytes)
     int rc = check_cfg(cfg);
     if (rc) return rc;
     if (!bytes) return SP_ERR_INVALID_ARG;
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
+    DevInfo dev;
+    dev.id = device;
+    if (cudaDeviceGetAttribute(&dev.sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&dev.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin,
+                               device) != cudaSuccess) {
         cudaGetLastError();
         return SP_ERR_CUDA;
     }
-    // partial sums of dgamma, dbeta, dbias, one slice per CTA (fast kernels:
-    // per consumer group, at most SMs x 4 groups; general kernel: its grid of
-    // at most 4 x SMs)
-    long long row0 = 0, rows = 0;
-    call_rows(cfg, &row0, &rows);
-    const long long fast = (rows < sms ? rows : sms) * (long long)kMaxGroups;
-    const long long gen = general_grid(rows, sms);
-    *bytes = (size_t)(fast > gen ? fast : gen) * 3 * (size_t)cfg->h * sizeof(float);
+    // the slices of the kernel the backward picks for 16-byte aligned
+    // pointers, or of the general kernel (misaligned pointers), whichever is
+    // larger
+    BwdArgs a;
+    bwd_shape(cfg, &a);
+    BwdChoice fast, general;
+    const int rf = choose_bwd(cfg, dev, true, a, &fast);
+    const int rg = choose_bwd(cfg, dev, false, a, &general);
+    if (rf && rg) return rf;
+    long long slices = rf ? 0 : fast.slices;
+    if (!rg && general.slices > slices) slices = general.slices;
+    *bytes = (size_t)slices * 3 * (size_t)cfg->h * sizeof(float);
     return SP_OK;
 }
 
@@ -611,102 +770,9 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
                            void* dresidual_in, void* dY, float* dgamma, float* dbeta,
                            float* dbias, void* workspace, size_t workspace_bytes, void* stream)
 {
-    int rc = check_cfg(cfg);
-    if (rc) return rc;
-    const bool ln = cfg->norm == SP_LAYERNORM;
-    if (!dn_partials || !residual_out || !gamma || !rstd || !dresidual_in || !dgamma ||
-        !workspace)
-        return SP_ERR_INVALID_ARG;
-    if (ln && !mean) return SP_ERR_INVALID_ARG;
-    if (!mask_bits && cfg->p_drop > 0.0f) return SP_ERR_INVALID_ARG;
-    const int E = elem_bytes(cfg);
-    bool all16 = true;
-    for (int k = 0; k < cfg->t; ++k) {
-        if (!dn_partials[k] || !aligned(dn_partials[k], E)) return SP_ERR_INVALID_ARG;
-        all16 = all16 && aligned(dn_partials[k], 16);
-    }
-    const int Er = res_elem_bytes(cfg);
-    const void* elem_ptrs[] = {gamma, dY};
-    for (const void* p : elem_ptrs) {
-        if (p && !aligned(p, E)) return SP_ERR_INVALID_ARG;
-        all16 = all16 && (!p || aligned(p, 16));
-    }
-    for (const void* p : {dR_next, residual_out, (const void*)dresidual_in}) {   // residual stream
-        if (p && !aligned(p, Er)) return SP_ERR_INVALID_ARG;
-        all16 = all16 && (!p || aligned(p, 16));
-    }
-    const void* f4_ptrs[] = {mask_bits, mean, rstd, dgamma, dbeta, dbias};
-    for (const void* p : f4_ptrs)
-        if (p && !aligned(p, 4)) return SP_ERR_INVALID_ARG;
-    if (!aligned(workspace, 16)) return SP_ERR_INVALID_ARG;
-
-    DevInfo dev;
-    if ((rc = use_device_of(residual_out, &dev))) return rc;
-
-    long long row0 = 0, rows = 0;
-    call_rows(cfg, &row0, &rows);
-    const int h = (int)cfg->h;
-    BwdArgs a;
-    memset(&a, 0, sizeof(a));
-    for (int k = 0; k < cfg->t; ++k) a.dparts[k] = dn_partials[k];
-    a.drnext = dR_next;
-    a.x = residual_out;
-    a.gamma = gamma;
-    a.mask = reinterpret_cast<const uint8_t*>(mask_bits);
-    a.mean = ln ? mean : nullptr;
-    a.rstd = rstd;
-    a.dres = dresidual_in;
-    a.dY = dY;
-    a.ws = static_cast<float*>(workspace);
-    a.rows = rows;
-    a.row0 = row0;
-    a.h = h;
-    a.hv = h / 8;
-    a.t = cfg->t;
-    a.seg_bytes = (uint32_t)(h * E);
-    a.res_seg_bytes = (uint32_t)(h * Er);
-    a.res_f32 = Er != E ? 1 : 0;
-    a.stage_stride = (uint32_t)round128(a.res_seg_bytes > a.seg_bytes ? a.res_seg_bytes
-                                                                       : a.seg_bytes);
-    a.mask_row_bytes = 4 * ((h + 31) / 32);
-    a.inv_h = (float)(1.0 / (double)h);
-    a.scale = 1.0f / (1.0f - cfg->p_drop);
-    a.want_dbeta = (ln && dbeta) ? 1 : 0;
-    a.want_dbias = dbias ? 1 : 0;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-
-    long long nparts = 0;
-    bool launched = false;
-    if (h % 8 == 0 && all16) {
-        const FastLaunch L = plan_bwd(a, dev, E, cfg->bwd_plan);
-        if (L.plan >= 0) {
-            nparts = (long long)L.grid * ((kBwdPlans[L.plan].acc == 1 || a.fold) ? 1 : L.groups);
-            if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes)
-                return SP_ERR_INVALID_ARG;
-            const void* kern = bwd_kernel_of(cfg->dtype, ln, L.plan, L.exact);
-            if ((rc = launch_kernel(kern, L.grid, L.block, L.smem, st, &a))) return rc;
-            launched = true;
-        }
-    }
-    if (!launched) {
-        const size_t smem = (size_t)h * 4;
-        if (smem > (size_t)dev.smem_optin - 1024) return SP_ERR_UNSUPPORTED;
-        nparts = general_grid(rows, dev.sms);
-        if ((size_t)nparts * 3 * h * sizeof(float) > workspace_bytes) return SP_ERR_INVALID_ARG;
-        const void* kern;
-        if (cfg->dtype == SP_BF16)
-            kern = ln ? (const void*)k_bwd_general<__nv_bfloat16, true>
-                      : (const void*)k_bwd_general<__nv_bfloat16, false>;
-        else
-            kern = ln ? (const void*)k_bwd_general<float, true>
-                      : (const void*)k_bwd_general<float, false>;
-        if ((rc = launch_kernel(kern, (int)nparts, kGeneralThreads, smem, st, &a))) return rc;
-    }
-    const int tiles = (h + 31) / 32;
-    k_colreduce<<<3 * tiles, 256, 0, st>>>(a.ws, (int)nparts, h, dgamma,
-                                           a.want_dbeta ? dbeta : nullptr,
-                                           a.want_dbias ? dbias : nullptr);
-    return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+    if (!workspace) return SP_ERR_INVALID_ARG;
+    return bwd_impl(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits, mean, rstd,
+                    dresidual_in, dY, dgamma, dbeta, dbias, workspace, workspace_bytes, stream);
 }
 
 int sp_device_error(int32_t device, int32_t* code, int32_t clear)
@@ -768,7 +834,6 @@ int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream)
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;   // 64 MiB per GPU
-constexpr int kNoAllocMaxDevices = 64;
 
 }  // namespace
 
@@ -778,24 +843,20 @@ static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / 
 
 namespace {
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-// Device address of the scratch array on device `dev`, which must be the
-// current device.  Looked up on the first call per device, then cached.
-int noalloc_scratch(int dev, void** out)
+// Device address of the scratch array on device `dev`, which the caller has
+// made current, once `need` bytes are known to fit.  The address is looked up
+// on every call (cheap once the library's device code is loaded), so it stays
+// right if the device's context is torn down and created again.
+int noalloc_scratch(int dev, size_t need, void** out)
 {
-    if (dev < 0 || dev >= kNoAllocMaxDevices) return SP_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-            cudaGetLastError();
-            return SP_ERR_CUDA;
-        }
-        g_noalloc_ptr[dev] = p;
+    (void)dev;
+    if (need > kNoAllocScratchBytes) return SP_ERR_UNSUPPORTED;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
     }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return SP_OK;
 }
 
@@ -807,17 +868,8 @@ extern "C" int sp_rs_norm_dropout_bwd_noalloc(
     const float* rstd, void* dresidual_in, void* dY, float* dgamma, float* dbeta, float* dbias,
     void* stream)
 {
-    int rc = check_cfg(cfg);
-    if (rc) return rc;
-    if (!residual_out) return SP_ERR_INVALID_ARG;
-    DevInfo dev;
-    if ((rc = use_device_of(residual_out, &dev))) return rc;   // makes it current
-    size_t need = 0;
-    if ((rc = sp_bwd_workspace_bytes(cfg, dev.id, &need))) return rc;
-    if (need > kNoAllocScratchBytes) return SP_ERR_UNSUPPORTED;
-    void* scratch = nullptr;
-    if ((rc = noalloc_scratch(dev.id, &scratch))) return rc;
-    return sp_rs_norm_dropout_bwd(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits,
-                                  mean, rstd, dresidual_in, dY, dgamma, dbeta, dbias, scratch,
-                                  kNoAllocScratchBytes, stream);
+    // the backward picks its kernel for the actual pointers, then checks that
+    // the slices that kernel writes fit the array
+    return bwd_impl(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits, mean, rstd,
+                    dresidual_in, dY, dgamma, dbeta, dbias, nullptr, 0, stream);
 }

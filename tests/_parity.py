@@ -294,19 +294,37 @@ def assert_close_extra(name, gpu, ref, mag, dtype, extra, k=K_FP32):
 
 def check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered=1,
                   rows_mean_rstd=True):
-    """Compare a device forward with the oracle's (same rows)."""
+    """Compare a device forward with the oracle's (same rows).
+
+    The norm output is held to the strict bound (one I/O ulp plus the fp32
+    term) on every row whose stored residual sums all equal the oracle's;
+    only on rows where a stored sum landed one ulp from the oracle's does
+    the first-order effect of that accepted difference widen the bound.
+    The norm step itself, fed the oracle's stored sums, is held to the
+    strict bound everywhere by check_norm_step."""
     dt = w.torch_dtype
     assert_close("residual_out", got["residual_out"], ref["residual_out"],
                  mag_residual_out(w, parts, bias, res), w.res_torch_dtype)
     ex_o, ex_m, ex_r = propagated_dx(w, got["residual_out"],
                                      ref["residual_out"], ref["mean"],
                                      ref["rstd"], gamma)
+    row_differs = (got["residual_out"].double() !=
+                   ref["residual_out"].double()).any(1).numpy()[:, None]
     mag = mag_norm_out(w, ref["residual_out"], ref["mean"], ref["rstd"],
                        gamma, beta)
     outs = got["gathered"] if "gathered" in got else [got["norm_out"]]
     refo = ref["gathered"][0] if "gathered" in ref else ref["norm_out"]
     for q in range(min(n_gathered, len(outs))):
         assert_close_extra(f"gathered[{q}]", outs[q], refo, mag, dt, ex_o)
+        g = outs[q].double().numpy()
+        r = refo.double().numpy()
+        strict = ulp_io(r, dt) + K_FP32 * 2.0 ** -24 * mag if \
+            dt == torch.bfloat16 else \
+            1e-5 * np.abs(r) + 1e-6 + K_FP32 * 2.0 ** -24 * mag
+        wide = ~(np.abs(g - r) <= strict)
+        assert not (wide & ~row_differs).any(), (
+            f"gathered[{q}]: {int((wide & ~row_differs).sum())} elements "
+            "need the widened bound on rows whose stored sums all match")
     if got.get("mask") is not None:
         assert np.array_equal(got["mask"], ref["mask"]), "mask bits differ"
     if got.get("rstd") is not None and rows_mean_rstd:
@@ -320,6 +338,50 @@ def check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered=1,
             gm = np.asarray(got["mean"], np.float64)
             bad = np.abs(gm - ref["mean"]) > 1e-5 * rms + ex_m
             assert not bad.any(), f"mean: {int(bad.sum())} rows outside"
+
+
+def gpu_norm_step(w, x_d, gamma_d, beta_d):
+    """The fused forward kernel's norm step alone, on the device sums x_d
+    ([rows, h] in the residual stream's dtype): the same forward call with
+    one partial sum of zeros, no bias and p = 0, so the stored sum is x_d
+    itself (x + 0 is exact) and the norm reads exactly x_d.  Returns
+    (stored sum, norm output, mean, rstd) on the device."""
+    N, h = x_d.shape
+    dt = w.torch_dtype
+    zero = torch.zeros((N, h), dtype=dt, device=x_d.device)
+    rout = torch.empty_like(x_d)
+    out = torch.empty((N, h), dtype=dt, device=x_d.device)
+    mean = torch.empty(N, dtype=torch.float32, device=x_d.device)
+    rstd = torch.empty(N, dtype=torch.float32, device=x_d.device)
+    cfg = sp.make_cfg(N, 1, h, 1, dtype=w.dtype, norm=w.norm, eps=w.eps,
+                      p_drop=0.0, res_f32=w.res != w.dtype)
+    sp.sp_rs_bias_dropout_add_norm_fwd(cfg, [zero], None, x_d, gamma_d,
+                                       beta_d, rout, [out], None, mean, rstd)
+    torch.cuda.synchronize()
+    assert sp.sp_device_error() == 0
+    return rout, out, mean, rstd
+
+
+def check_norm_step(w, got, x_ref, ref_out, ref_mean, ref_rstd, gamma, beta):
+    """gpu_norm_step's outputs (host tensors in ``got``) against the oracle's
+    norm of its own stored sums x_ref: the stored sum bit for bit, the norm
+    output within one I/O ulp plus the fp32 term, mean and rstd within 1e-5
+    relative -- no allowance for a differing input."""
+    assert torch.equal(got["residual_out"].view(torch.int16 if
+                       got["residual_out"].dtype == torch.bfloat16
+                       else torch.int32),
+                       x_ref.view(torch.int16 if x_ref.dtype == torch.bfloat16
+                                  else torch.int32)), "x + 0 changed x"
+    mag = mag_norm_out(w, x_ref, ref_mean, ref_rstd, gamma, beta)
+    assert_close("norm step", got["norm_out"], ref_out, mag, w.torch_dtype)
+    gr = np.asarray(got["rstd"], np.float64)
+    rr = np.asarray(ref_rstd, np.float64)
+    assert not (np.abs(gr - rr) > 1e-5 * rr).any(), "norm step rstd"
+    if w.norm == "layernorm":
+        rms = x_ref.double().pow(2).mean(1).sqrt().numpy()
+        gm = np.asarray(got["mean"], np.float64)
+        assert not (np.abs(gm - ref_mean) > 1e-5 * rms).any(), \
+            "norm step mean"
 
 
 def mags_backward(w, dparts, drnext, x, gamma, mean, rstd):
