@@ -95,6 +95,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         tmem_fence_before_sync();
     }
     init_ring(tail, S, C / 32);
+    grid_dep_launch();
+    grid_dep_wait();   // the previous kernel's outputs are visible
 
     if (tid >= G * C) {
         if (tid == G * C)
@@ -501,6 +503,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
 template <typename T, bool LN>
 __global__ void __launch_bounds__(1024) k_bwd_general(const __grid_constant__ BwdArgs a)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     extern __shared__ __align__(128) unsigned char smem[];
     float* dns = reinterpret_cast<float*>(smem);
     __shared__ float red[32];
@@ -578,7 +582,9 @@ static __global__ void __launch_bounds__(kColreduceWarps * 32)
     const int j = (blockIdx.x - q * tiles) * 32 + lane;
     const int w = threadIdx.x >> 5;
     float* out = q == 0 ? dgamma : (q == 1 ? dbeta : dbias);
+    grid_dep_launch();
     if (!out) return;   // uniform over the block
+    grid_dep_wait();    // the backward's slices are complete and visible
     float s = 0.f;
     if (j < h) {
         const float* p = ws + (size_t)q * h + j;

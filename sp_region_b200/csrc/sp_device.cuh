@@ -58,6 +58,26 @@ __device__ __forceinline__ void record_error(unsigned code)
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch (PTX ISA: griddepcontrol).  The library
+// launches every kernel so that the next kernel in the stream may be
+// scheduled before this one has finished; its CTAs then wait in
+// grid_dep_wait() until the kernels it depends on have completed and their
+// memory is visible.  Every kernel calls grid_dep_wait() before its first
+// global-memory access (read or write), so the early launch hides only the
+// launch and set-up latency, never a data dependence.  grid_dep_launch()
+// lets this kernel's own dependents be scheduled.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // mbarrier and bulk copy (PTX ISA: mbarrier.*, cp.async.bulk)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void* p)

@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(kEntryThreads, 1) k_norm_ag(const __grid_const
     unsigned char* sb = smem + a.param_stride;
     float* red = reinterpret_cast<float*>(smem + 2 * a.param_stride);   // [2][G][2][32]
     const bool has_beta = LN && a.beta;
+    grid_dep_launch();
+    grid_dep_wait();   // the previous kernel's outputs are visible
     for (int v = tid; v < hv; v += blockDim.x) {
         store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
         if (has_beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));

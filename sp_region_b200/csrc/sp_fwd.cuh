@@ -231,6 +231,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 
     init_ring(tail, S, C / 32);
     if (CS > 1) cluster_sync_all();   // the peer's barriers exist before any remote arrive
+    grid_dep_launch();
+    grid_dep_wait();                  // the previous kernel's outputs are visible
 
     if (tid >= G * C) {
         if (tid == G * C)
@@ -480,6 +482,8 @@ __global__ void __launch_bounds__(MAXT, 1) k_fwd_tma(const __grid_constant__ Fwd
 template <typename T, bool LN>
 __global__ void __launch_bounds__(256) k_fwd_general(const __grid_constant__ FwdArgs a)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     extern __shared__ __align__(128) unsigned char smem[];
     float* xs = reinterpret_cast<float*>(smem);
     uint32_t* mw = reinterpret_cast<uint32_t*>(xs + a.h);

@@ -23,6 +23,8 @@ struct GatherArgs {
 template <typename U>
 __global__ void __launch_bounds__(512) k_all_gather(const __grid_constant__ GatherArgs a)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     const long long total = a.shard_units * a.t;
     const long long stride = (long long)gridDim.x * blockDim.x;
     constexpr int kUnroll = 4;
@@ -51,6 +53,8 @@ __global__ void __launch_bounds__(512) k_all_gather(const __grid_constant__ Gath
 // of hanging.  Exercises the same bounded wait as the streaming kernels.
 __global__ void k_wait_selftest(unsigned long long limit_ns, int* status)
 {
+    grid_dep_launch();
+    grid_dep_wait();
     __shared__ __align__(8) uint64_t bar;
     __shared__ int abort;
     if (threadIdx.x == 0) {

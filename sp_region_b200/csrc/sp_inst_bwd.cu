@@ -36,13 +36,13 @@ constexpr bool LN = SP_LN != 0;
 template <bool EXACT>
 const void* bwd_kernel(int id)
 {
-    static_assert(kNumBwdPlans == 23, "one case per backward plan");
+    static_assert(kNumBwdPlans == 24, "one case per backward plan");
     switch (id) {
         SP_BWD_CASE(0) SP_BWD_CASE(1) SP_BWD_CASE(2) SP_BWD_CASE(3) SP_BWD_CASE(4)
         SP_BWD_CASE(5) SP_BWD_CASE(6) SP_BWD_CASE(7) SP_BWD_CASE(8) SP_BWD_CASE(9)
         SP_BWD_CASE(10) SP_BWD_CASE(11) SP_BWD_CASE(12) SP_BWD_CASE(13) SP_BWD_CASE(14)
         SP_BWD_CASE(15) SP_BWD_CASE(16) SP_BWD_CASE(17) SP_BWD_CASE(18) SP_BWD_CASE(19)
-        SP_BWD_CASE(20) SP_BWD_CASE(21) SP_BWD_CASE(22)
+        SP_BWD_CASE(20) SP_BWD_CASE(21) SP_BWD_CASE(22) SP_BWD_CASE(23)
     }
     return nullptr;
 }

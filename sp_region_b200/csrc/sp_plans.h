@@ -63,6 +63,7 @@ constexpr Plan kBwdPlans[] = {
     {2, 3, 800, 2, 1},        // 20
     {4, 1, 544, 2, 1},        // 21
     {2, 1, 544, 2, 1},        // 22
+    {4, 2, 544, 2, 1},        // 23
 };
 constexpr int kNumFwdPlans = sizeof(kFwdPlans) / sizeof(kFwdPlans[0]);
 constexpr int kNumBwdPlans = sizeof(kBwdPlans) / sizeof(kBwdPlans[0]);

@@ -122,8 +122,9 @@ constexpr int kFwdEntryOrder[] = {13, 12, 11, 10, 4, 9, 6, 8, 1, 2, 0, 3, 5, 7, 
                                   17, 18};
 // backward: tensor-memory accumulators first; they leave shared memory to the
 // ring (measured on B200 for bf16 rows of h = 12288, t = 16: 2 -> 8 stages,
-// 4.9 -> 6.6 TB/s)
-constexpr int kBwdOrder[] = {19, 15, 18, 16, 17, 21, 20, 22, 11, 8, 9, 12,
+// 4.9 -> 6.6 TB/s).  Plan 23 (two groups of 4-vector threads) tiles rows of
+// 1024 vectors exactly: h = 8192 went 5.60 -> 5.69 TB/s over plan 18.
+constexpr int kBwdOrder[] = {19, 15, 23, 18, 16, 17, 21, 20, 22, 11, 8, 9, 12,
                              2, 3, 5, 10, 6, 1, 0, 4, 7, 13, 14};
 
 int group_threads(int hv, int V)
@@ -165,8 +166,11 @@ const void* bwd_kernel_of(int dtype, bool ln, int id, bool exact)
     return ln ? bwd_kernel_f32_ln(id, exact) : bwd_kernel_f32_rms(id, exact);
 }
 
-int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream_t st,
-                  void* args)
+// Every launch allows programmatic dependent launch: the kernel may be
+// scheduled while the previous kernel in the stream is still running, and
+// waits in-kernel (griddepcontrol.wait) before touching global memory.
+int launch_kernel_args(const void* kern, int grid, int block, size_t smem, cudaStream_t st,
+                       void** params)
 {
     if (!kern) return SP_ERR_UNSUPPORTED;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -174,12 +178,28 @@ int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream
         cudaGetLastError();
         return SP_ERR_CUDA;
     }
-    void* params[] = {args};
-    if (cudaLaunchKernel(kern, dim3(grid), dim3(block), params, smem, st) != cudaSuccess) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelExC(&cfg, kern, params) != cudaSuccess) {
         cudaGetLastError();
         return SP_ERR_CUDA;
     }
     return SP_OK;
+}
+
+int launch_kernel(const void* kern, int grid, int block, size_t smem, cudaStream_t st,
+                  void* args)
+{
+    void* params[] = {args};
+    return launch_kernel_args(kern, grid, block, smem, st, params);
 }
 
 // A persistent launch of clusters of `cs` CTAs: as many clusters as fit on
@@ -194,17 +214,19 @@ int launch_clusters(const void* kern, long long rows, int cs, int block, size_t 
         cudaGetLastError();
         return SP_ERR_CUDA;
     }
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(block);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     cfg.gridDim = dim3(cs);
     int max_clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess ||
@@ -664,10 +686,12 @@ int bwd_impl(const sp_cfg* cfg, const void* const* dn_partials, const void* dR_n
             return rc;
     }
     const int tiles = (h + 31) / 32;
-    k_colreduce<<<3 * tiles, kColreduceWarps * 32, 0, st>>>(
-        a.ws, (int)ch.slices, h, dgamma, a.want_dbeta ? dbeta : nullptr,
-        a.want_dbias ? dbias : nullptr);
-    return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+    const float* ws_c = a.ws;
+    int nparts = (int)ch.slices, hh = h;
+    float* outs[3] = {dgamma, a.want_dbeta ? dbeta : nullptr, a.want_dbias ? dbias : nullptr};
+    void* params[] = {&ws_c, &nparts, &hh, &outs[0], &outs[1], &outs[2]};
+    return launch_kernel_args((const void*)k_colreduce, 3 * tiles, kColreduceWarps * 32, 0, st,
+                              params);
 }
 
 }  // namespace
@@ -809,12 +833,8 @@ int sp_debug_wait_timeout(int64_t limit_ns, int32_t* status, void* stream)
     unsigned long long lim = (unsigned long long)limit_ns;
     int* st = reinterpret_cast<int*>(status);
     void* params[] = {&lim, &st};
-    if (cudaLaunchKernel((const void*)k_wait_selftest, dim3(1), dim3(32), params, 0,
-                         static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-        cudaGetLastError();
-        return SP_ERR_CUDA;
-    }
-    return SP_OK;
+    return launch_kernel_args((const void*)k_wait_selftest, 1, 32, 0,
+                              static_cast<cudaStream_t>(stream), params);
 }
 
 }  // extern "C"
