@@ -95,6 +95,12 @@ def _lib():
         L.orc_bwd_rows.argtypes = [vp, i64, vp, vp, vp, vp, vp, dp, dp, vp, vp,
                                    dp, dp, dp]
         L.orc_bwd_rows.restype = ctypes.c_int
+        L.orc_rowpar_reduce.argtypes = [i64, i64, i64, ctypes.c_int, vp, vp, dp]
+        L.orc_linear_rs_fwd_rows.argtypes = [vp, i64, i64, vp, vp, vp, vp, vp, vp,
+                                             vp, vp, vp, vp, dp, dp]
+        L.orc_linear_rs_fwd_rows.restype = ctypes.c_int
+        L.orc_ag_colpar_fwd.argtypes = [ctypes.c_int, i64, i64, i64, vp, vp, vp]
+        L.orc_ag_colpar_fwd.restype = ctypes.c_int
         L.orc_activation_bytes.argtypes = [i64, i64, i64, i64, i32, i32,
                                            ctypes.c_double]
         L.orc_activation_bytes.restype = ctypes.c_double
@@ -358,4 +364,56 @@ def bwd_rows(cfg: Cfg, dpart_rows, drnext_rows, x_rows, gamma, mask_rows,
     out = dict(dresidual_in=dres, dY=dY)
     if with_params:
         out.update(dgamma=pg[0], dbeta=pg[1], dbias=pg[2])
+    return out
+
+
+# ----------------------------------------------------------------------------
+# tensor-parallel linears on t emulated ranks
+# ----------------------------------------------------------------------------
+
+def rowpar_reduce(x, w, t: int) -> np.ndarray:
+    """Row-parallel linear: the t ranks' partials x[:, slice k] @ w[:, slice
+    k]^T summed k ascending, in float64.  x [rows, f], w [h, f] bf16."""
+    x, w = _cpu(x, BF16), _cpu(w, BF16)
+    rows, f = x.shape
+    h = w.shape[0]
+    y = np.zeros((rows, h))
+    _lib().orc_rowpar_reduce(rows, f, h, t, _ptr(x), _ptr(w), y.ctypes.data)
+    return y
+
+
+def linear_rs_fwd_rows(cfg: Cfg, f: int, row_ids, x_rows, w, bias, residual_rows,
+                       gamma, beta) -> dict:
+    """The row-parallel linear, then the SP region, on selected global token
+    rows (x_rows [nrows, f], residual_rows [nrows, h])."""
+    ids = np.ascontiguousarray(np.asarray(row_ids, dtype=np.int64))
+    x_rows, w = _cpu(x_rows, BF16), _cpu(w, BF16)
+    bias, gamma, beta = (_cpu(v, cfg.dtype) for v in (bias, gamma, beta))
+    residual_rows = _cpu(residual_rows, cfg.res_dtype)
+    n, h = len(ids), cfg.h
+    rout = torch.empty((n, h), dtype=_torch_dtype(cfg.res_dtype))
+    out = torch.empty((n, h), dtype=_torch_dtype(cfg.dtype))
+    mask = np.zeros((n, mask_words(h)), dtype=np.uint32)
+    mean = np.zeros(n)
+    rstd = np.zeros(n)
+    rc = _lib().orc_linear_rs_fwd_rows(
+        ctypes.byref(cfg), f, n, ids.ctypes.data, _ptr(x_rows), _ptr(w), _ptr(bias),
+        _ptr(residual_rows), _ptr(gamma), _ptr(beta), _ptr(rout), _ptr(out),
+        mask.ctypes.data, mean.ctypes.data, rstd.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle linear forward rejected the configuration ({rc})")
+    return dict(residual_out=rout, norm_out=out, mask=mask,
+                mean=mean if cfg.norm == LAYERNORM else None, rstd=rstd)
+
+
+def ag_colpar_fwd(shards, w) -> torch.Tensor:
+    """All-gather of the t shards, then the column-parallel linear X @ w^T
+    rounded to bf16 (shards [rows/t, h] each, w [f_out, h])."""
+    sh = [_cpu(x, BF16) for x in shards]
+    w = _cpu(w, BF16)
+    t, (per, h), f_out = len(sh), sh[0].shape, w.shape[0]
+    out = torch.empty((t * per, f_out), dtype=torch.bfloat16)
+    rc = _lib().orc_ag_colpar_fwd(t, per, h, f_out, _ptr_array(sh), _ptr(w), _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle column-parallel forward rejected the shapes ({rc})")
     return out

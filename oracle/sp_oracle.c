@@ -583,6 +583,103 @@ int orc_bwd_rows(const orc_cfg* c, int64_t nrows, const void* const* dparts,
 }
 
 /* ------------------------------------------------------------------------- */
+/* Tensor-parallel linears on t emulated ranks                                 */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Row-parallel linear ("TP and SP explained with pictures", section "Tensor
+ * parallelism, take two: split the inner dimension"; "Chapter 6: TP and SP",
+ * section 3): rank k holds columns [k*f/t, (k+1)*f/t) of the input x and the
+ * same slice of the inner dimension of the weight w, and computes the
+ * full-shape partial
+ *     p_k[n, j] = sum over i in slice k of x[n, i] * w[j, i];
+ * the partials are then summed across the ranks, k ascending.
+ *   x [rows][f] bf16, w [h][f] bf16 (output-by-input), y [rows][h] double.
+ * The partials are kept in double: in the fused path none of them is ever
+ * stored, so none is rounded to the I/O dtype.
+ */
+void orc_rowpar_reduce(int64_t rows, int64_t f, int64_t h, int t, const void* x,
+                       const void* w, double* y)
+{
+    const int64_t per = f / t;
+    for (int64_t n = 0; n < rows; ++n)
+        for (int64_t j = 0; j < h; ++j) {
+            double acc = 0.0;
+            for (int k = 0; k < t; ++k) {
+                double part = 0.0;
+                for (int64_t i = k * per; i < (k + 1) * per; ++i)
+                    part += ld(x, n * f + i, ORC_BF16) * ld(w, j * f + i, ORC_BF16);
+                acc += part;
+            }
+            y[n * h + j] = acc;
+        }
+}
+
+/*
+ * The forward boundary with the row-parallel linear in front, on selected
+ * token rows: y = the reduced partials of orc_rowpar_reduce, then the SP
+ * region exactly as orc_fwd_rows (bias once, dropout, residual add, norm).
+ *   row_ids[i]   global token row of sample i (the dropout counter)
+ *   x_rows       [nrows][f] bf16; residual_rows [nrows][h]; outputs
+ *                [nrows][...] in sample order
+ */
+int orc_linear_rs_fwd_rows(const orc_cfg* c, int64_t f, int64_t nrows, const int64_t* row_ids,
+                           const void* x_rows, const void* w, const void* bias,
+                           const void* residual, const void* gamma, const void* beta,
+                           void* residual_out, void* norm_out, uint32_t* mask, double* mean,
+                           double* rstd)
+{
+    if (!cfg_ok(c) || f < 1 || f % c->t) return -1;
+    const int64_t h = c->h, W = orc_mask_words(h);
+    double* y = (double*)malloc(sizeof(double) * (size_t)h);
+    double* x = (double*)malloc(sizeof(double) * (size_t)h);
+    double* o = (double*)malloc(sizeof(double) * (size_t)h);
+    if (!y || !x || !o) { free(y); free(x); free(o); return -2; }
+    for (int64_t i = 0; i < nrows; ++i) {
+        const uint16_t* xr = (const uint16_t*)x_rows + i * f;
+        orc_rowpar_reduce(1, f, h, c->t, xr, w, y);
+        region_row_fwd(c, row_ids[i], y, bias, residual, i, gamma, beta, residual_out, o,
+                       mask ? mask + i * W : NULL, mean ? mean + i : NULL,
+                       rstd ? rstd + i : NULL, x);
+        for (int64_t j = 0; j < h; ++j) st(norm_out, i * h + j, c->dtype, o[j]);
+    }
+    free(y); free(x); free(o);
+    return 0;
+}
+
+/*
+ * Column-parallel linear with the all-gather in front ("TP and SP explained
+ * with pictures", sections "Tensor parallelism, take one: split the output
+ * dimension" and "Add Sequence parallelism"; "Chapter 6: TP and SP", section
+ * 2): the t sequence shards are all-gathered into the full input X (shard 0
+ * first), then out[n, o] = sum_i X[n, i] * w[o, i], rounded once to bf16.
+ *   shards[r] [shard_rows][h] bf16, w [f_out][h] bf16, out [t*shard_rows][f_out]
+ */
+int orc_ag_colpar_fwd(int t, int64_t shard_rows, int64_t h, int64_t f_out,
+                      const void* const* shards, const void* w, void* out)
+{
+    if (t < 1 || shard_rows < 1 || h < 1 || f_out < 1) return -1;
+    const int64_t N = (int64_t)t * shard_rows;
+    double** sh = (double**)malloc(sizeof(double*) * (size_t)t);
+    double* full = (double*)malloc(sizeof(double) * (size_t)(N * h));
+    double* X = (double*)malloc(sizeof(double) * (size_t)(N * h));
+    if (!sh || !full || !X) { free(sh); free(full); free(X); return -2; }
+    for (int r = 0; r < t; ++r) {
+        sh[r] = full + (int64_t)r * shard_rows * h;
+        for (int64_t i = 0; i < shard_rows * h; ++i) sh[r][i] = ld(shards[r], i, ORC_BF16);
+    }
+    orc_all_gather(t, shard_rows, h, (const double* const*)sh, X);
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t o = 0; o < f_out; ++o) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < h; ++i) acc += X[n * h + i] * ld(w, o * h + i, ORC_BF16);
+            st(out, n * f_out + o, ORC_BF16, acc);
+        }
+    free(sh); free(full); free(X);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Activation memory per layer and device ("Sequence Parallelism math",      */
 /* equations A_layer, A_TP, A_TP+SP).  mode 0: A_layer = sbh(34 + 5as/h);    */
 /* 1: A_TP = sbh(10 + 24/t + 5as/(ht)); 2: A_TP+SP = (sbh/t)(34 + 5as/h).     */

@@ -87,6 +87,15 @@ MUTANTS = {
         "if (rstd) rstd[n] = rs;", "if (rstd) rstd[i] = rs;"),
     "row-chunk shares: dbeta reported as dgamma": (
         "if (dgamma) dgamma[j] = acc[j];", "if (dgamma) dgamma[j] = acc[h + j];"),
+    "row-parallel linear drops the last rank": (
+        "            for (int k = 0; k < t; ++k) {\n                double part = 0.0;",
+        "            for (int k = 0; k < t - 1; ++k) {\n                double part = 0.0;"),
+    "row-parallel linear reads the weight transposed": (
+        "part += ld(x, n * f + i, ORC_BF16) * ld(w, j * f + i, ORC_BF16);",
+        "part += ld(x, n * f + i, ORC_BF16) * ld(w, i * h + j, ORC_BF16);"),
+    "column-parallel linear skips the all-gather order": (
+        "orc_all_gather(t, shard_rows, h, (const double* const*)sh, X);",
+        "for (int64_t q = 0; q < N * h; ++q) X[q] = sh[0][q % (shard_rows * h)];"),
     "ring volume without (t-1)/t": (
         "double phase = (double)(t - 1) / (double)t * V;",
         "double phase = V;"),

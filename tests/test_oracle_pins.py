@@ -789,3 +789,96 @@ def test_fp32_residual_stream_entry(orc):
                        float(np.float32(w.eps))).numpy()
     got = out["gathered"][0].double().numpy()
     assert (np.abs(got - ref) <= _ulp_bf16(ref) * 0.5 + 1e-12 * np.abs(ref)).all()
+
+
+# ----------------------------------------------------------------------------
+# tensor-parallel linears: the row-parallel reduction and the all-gathered
+# column-parallel linear
+# ----------------------------------------------------------------------------
+
+def _bf16(shape, seed, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_rowpar_reduce_matches_torch_matmul(orc, t):
+    """The t ranks' partials summed equal the whole product x @ w^T, against
+    torch.matmul in float64."""
+    x, w = _bf16((5, 64), 11), _bf16((24, 64), 12)
+    y = orc.rowpar_reduce(x, w, t)
+    ref = (x.double() @ w.double().T).numpy()
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rowpar_reduce_hand_worked_2x2(orc):
+    """x = [[1, 2], [3, 4]], w = [[5, 6], [7, 8]] on t = 2 ranks: rank 0's
+    partial is x[:, 0] w[:, 0]^T = [[5, 7], [15, 21]], rank 1's is
+    [[12, 16], [24, 32]]; their sum is x w^T = [[17, 23], [39, 53]]."""
+    x = torch.tensor([[1.0, 2.0], [3.0, 4.0]]).to(torch.bfloat16)
+    w = torch.tensor([[5.0, 6.0], [7.0, 8.0]]).to(torch.bfloat16)
+    assert np.array_equal(orc.rowpar_reduce(x[:, :1], w[:, :1], 1), [[5, 7], [15, 21]])
+    assert np.array_equal(orc.rowpar_reduce(x[:, 1:], w[:, 1:], 1), [[12, 16], [24, 32]])
+    assert np.array_equal(orc.rowpar_reduce(x, w, 2), [[17, 23], [39, 53]])
+
+
+def test_rowpar_reduce_does_not_depend_on_t(orc):
+    """Small integer inputs make every partial and every sum exact, so the
+    split of the inner dimension over t ranks cannot change the result."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.randint(-3, 4, (6, 64), generator=g).to(torch.bfloat16)
+    w = torch.randint(-3, 4, (10, 64), generator=g).to(torch.bfloat16)
+    ys = [orc.rowpar_reduce(x, w, t) for t in (1, 2, 4, 8)]
+    for y in ys[1:]:
+        assert np.array_equal(y, ys[0])
+
+
+@pytest.mark.parametrize("norm", ["layernorm", "rmsnorm"])
+def test_linear_rs_equals_the_boundary_on_exact_partials(orc, norm):
+    """With inputs whose every rank partial is exact in bf16 (integers of at
+    most 64 in magnitude), the row-parallel linear followed by the SP region
+    gives exactly what the boundary gives on those partials stored as t
+    buffers: stored sum, norm output, mask and statistics, bit for bit."""
+    w_ = sp_synth.WORKLOADS["C2"].replace(s=8, b=2, h=48, t=4, norm=norm,
+                                           p_drop=0.25,
+                                           has_beta=norm == "layernorm")
+    f, t = 64, w_.t
+    g = torch.Generator().manual_seed(9)
+    x = torch.randint(-2, 3, (w_.rows, f), generator=g).to(torch.bfloat16)
+    w = torch.randint(-2, 3, (w_.h, f), generator=g).to(torch.bfloat16)
+    bias, gamma, beta = sp_synth.draw_params(w_)
+    beta = beta if norm == "layernorm" else None
+    res = sp_synth.draw_residual(w_)
+    cfg = orc.cfg_from(w_)
+    per = f // t
+    parts = [(x[:, k * per:(k + 1) * per].double() @
+              w[:, k * per:(k + 1) * per].double().T).to(torch.bfloat16)
+             for k in range(t)]
+    for p_ in parts:
+        assert p_.double().abs().max() <= 64
+    ref = orc.fwd(cfg, parts, bias, res, gamma, beta)
+    got = orc.linear_rs_fwd_rows(cfg, f, list(range(w_.rows)), x, w, bias, res,
+                                 gamma, beta)
+    assert torch.equal(got["residual_out"], ref["residual_out"])
+    assert torch.equal(got["norm_out"], ref["gathered"][0])
+    assert np.array_equal(got["mask"], ref["mask"])
+    assert np.array_equal(got["rstd"], ref["rstd"])
+    if norm == "layernorm":
+        assert np.array_equal(got["mean"], ref["mean"])
+
+
+@pytest.mark.parametrize("t", [1, 2, 4])
+def test_ag_colpar_is_the_correctly_rounded_product_of_the_gathered_input(orc, t):
+    """The shards are gathered in rank order and multiplied by w^T: every
+    output is the float64 product (torch.matmul) rounded once to bf16, so it
+    lies within half a bf16 ulp of it; and reversing the shard order changes
+    the rows."""
+    shards = [_bf16((6, 40), 20 + r) for r in range(t)]
+    w = _bf16((24, 40), 30)
+    out = orc.ag_colpar_fwd(shards, w).double().numpy()
+    ref = (torch.cat(shards).double() @ w.double().T).numpy()
+    e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126)))
+    assert (np.abs(out - ref) <= 2.0 ** (e - 8) * (1 + 1e-12)).all()
+    if t > 1:
+        rev = orc.ag_colpar_fwd(shards[::-1], w).double().numpy()
+        assert not np.array_equal(rev, out)
