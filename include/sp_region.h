@@ -286,6 +286,77 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
                            float* dbeta, float* dbias, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/*
+ * Row-parallel linear with the reduce-scatter fused into its epilogue.
+ *
+ * Defined by: "TP and SP explained with pictures", sections "Tensor
+ * parallelism, take two: split the inner dimension" (each rank computes a
+ * full-shape partial sum from its slice of the inner dimension; the partials
+ * are summed across ranks) and "Add Sequence parallelism" (with SP that sum
+ * is a reduce-scatter back to token shards, followed by the SP region);
+ * "Chapter 6: TP and SP", section 3 (Row Parallel Linear: Y_i = X_i A_i).
+ *
+ * x [rows][f] bf16 holds, for this call's token rows, the row-parallel
+ * input; rank k's slice is columns [k*f/t, (k+1)*f/t).  w [h][f] bf16 is the
+ * weight in output-by-input layout; rank k's rows of the weight are its
+ * columns [k*f/t, (k+1)*f/t).  For every row n of the call:
+ *   y[n, j] = sum_{k=0..t-1} sum_{i in slice k} x[n, i] * w[j, i]
+ *           (the t partials are summed in one fp32 accumulator in tensor
+ *            memory, slice by slice; no partial is ever stored)
+ *   then bias, inverted dropout (the forward's Philox mask) and the residual
+ *   add exactly as sp_rs_bias_dropout_add_norm_fwd: residual_out = round(
+ *   residual + dropout(y + bias)), mask_bits as there.
+ * The norm and the all-gather follow in sp_linear_rs_bias_dropout_add_norm_fwd.
+ *
+ * Requirements: cfg->dtype SP_BF16 and res_f32 = 0 (else SP_ERR_UNSUPPORTED);
+ * f % t == 0 (else SP_ERR_INVALID_ARG); f and h multiples of 8 (else
+ * SP_ERR_UNSUPPORTED); x, w, bias, residual, residual_out 16-byte aligned.
+ * The row range of cfg selects the call's rows: x, residual, residual_out
+ * and mask_bits are indexed by local row, the dropout counter by global row.
+ */
+int sp_rowpar_linear_rs_fwd(const sp_cfg* cfg, int64_t f, const void* x, const void* w,
+                            const void* bias, const void* residual, void* residual_out,
+                            uint32_t* mask_bits, void* stream);
+
+/*
+ * The forward boundary with its reduce-scatter inside the row-parallel GEMM:
+ * sp_rowpar_linear_rs_fwd, then the per-token norm of residual_out and the
+ * all-gather of the result into `gathered` (the same kernel as
+ * sp_norm_all_gather_fwd).  Outputs and their layouts are those of
+ * sp_rs_bias_dropout_add_norm_fwd; the t partials of that call are replaced
+ * by x and w.  Two launches on `stream`.
+ */
+int sp_linear_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, int64_t f, const void* x,
+                                           const void* w, const void* bias,
+                                           const void* residual, const void* gamma,
+                                           const void* beta, void* residual_out,
+                                           void* const* gathered, int32_t n_gathered,
+                                           uint32_t* mask_bits, float* mean, float* rstd,
+                                           void* stream);
+
+/*
+ * Column-parallel linear with the all-gather fused into its prologue.
+ *
+ * Defined by: "TP and SP explained with pictures", sections "Tensor
+ * parallelism, take one: split the output dimension" (every rank multiplies
+ * the full input by its slice of the weight's output columns) and "Add
+ * Sequence parallelism" (with SP the full input is all-gathered from the
+ * sequence shards first); "Chapter 6: TP and SP", section 2.
+ *
+ *   out[n, o] = round( sum_i X[n, i] * w[o, i] ),  X = concat_r shards[r]
+ * shards: HOST array of t device pointers, shard r = rows [r*N/t, (r+1)*N/t)
+ * of the SP region's output, [N/t][h] bf16 each; the GEMM reads its A tiles
+ * straight from the shards, so no gathered copy is made.  w [f_out][h] bf16
+ * (output-by-input); out [N][f_out] bf16.  fp32 accumulation in tensor
+ * memory, one rounding.
+ *
+ * Requirements: SP_BF16; t <= 16 and (t == 1 or (N/t) % 128 == 0); h and
+ * f_out multiples of 8 (else SP_ERR_UNSUPPORTED); no row range (else
+ * SP_ERR_INVALID_ARG); 16-byte aligned pointers.
+ */
+int sp_ag_colpar_linear_fwd(const sp_cfg* cfg, int64_t f_out, const void* const* shards,
+                            const void* w, void* out, void* stream);
+
 /* Bytes of device scratch sp_rs_norm_dropout_bwd needs for cfg on CUDA
  * device `device`: the slices of 3*h fp32 parameter-gradient partial sums
  * that the kernel the call picks writes, for 16-byte aligned pointers or for

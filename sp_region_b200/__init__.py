@@ -33,7 +33,9 @@ EXPORTS = ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
            "sp_rs_norm_dropout_bwd", "sp_bwd_workspace_bytes",
            "sp_activation_bytes", "sp_status_string", "sp_device_error",
            "sp_debug_wait_timeout", "sp_plan_count",
-           "sp_rs_norm_dropout_bwd_noalloc", "sp_norm_all_gather_fwd")
+           "sp_rs_norm_dropout_bwd_noalloc", "sp_norm_all_gather_fwd",
+           "sp_rowpar_linear_rs_fwd", "sp_linear_rs_bias_dropout_add_norm_fwd",
+           "sp_ag_colpar_linear_fwd")
 
 
 class SPError(RuntimeError):
@@ -81,6 +83,10 @@ def _load() -> ctypes.CDLL:
     lib.sp_plan_count.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.sp_rs_norm_dropout_bwd_noalloc.argtypes = [
         cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sp_rowpar_linear_rs_fwd.argtypes = [cfgp, i64, vp, vp, vp, vp, vp, vp, vp]
+    lib.sp_linear_rs_bias_dropout_add_norm_fwd.argtypes = [
+        cfgp, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
+    lib.sp_ag_colpar_linear_fwd.argtypes = [cfgp, i64, vp, vp, vp, vp]
     for f in EXPORTS:
         getattr(lib, f).restype = (ctypes.c_char_p if f == "sp_status_string"
                                    else ctypes.c_int)
@@ -205,6 +211,43 @@ def sp_rs_norm_dropout_bwd_noalloc(cfg: sp_cfg, dn_partials, dR_next,
                _p(residual_out), _p(gamma), _p(mask_bits), _p(mean), _p(rstd),
                _p(dresidual_in), _p(dY), _p(dgamma), _p(dbeta), _p(dbias),
                _stream(stream, residual_out)))
+
+
+def sp_rowpar_linear_rs_fwd(cfg: sp_cfg, f: int, x, w, bias, residual,
+                            residual_out, mask_bits=None, stream=None) -> None:
+    """Row-parallel linear x [rows, f] @ w [h, f]^T whose t rank partials
+    are reduced in the GEMM's accumulator, then bias, dropout and the
+    residual add into residual_out (and mask_bits)."""
+    _check("sp_rowpar_linear_rs_fwd",
+           _lib.sp_rowpar_linear_rs_fwd(
+               ctypes.byref(cfg), f, _p(x), _p(w), _p(bias), _p(residual),
+               _p(residual_out), _p(mask_bits), _stream(stream, x)))
+
+
+def sp_linear_rs_bias_dropout_add_norm_fwd(cfg: sp_cfg, f: int, x, w, bias,
+                                           residual, gamma, beta,
+                                           residual_out, gathered,
+                                           mask_bits=None, mean=None,
+                                           rstd=None, stream=None) -> None:
+    """The forward boundary with its reduce-scatter in the row-parallel
+    GEMM: sp_rowpar_linear_rs_fwd, then the norm and the all-gather."""
+    gathered = list(gathered)
+    _check("sp_linear_rs_bias_dropout_add_norm_fwd",
+           _lib.sp_linear_rs_bias_dropout_add_norm_fwd(
+               ctypes.byref(cfg), f, _p(x), _p(w), _p(bias), _p(residual),
+               _p(gamma), _p(beta), _p(residual_out), _ptrs(gathered),
+               len(gathered), _p(mask_bits), _p(mean), _p(rstd),
+               _stream(stream, x)))
+
+
+def sp_ag_colpar_linear_fwd(cfg: sp_cfg, f_out: int, shards, w, out,
+                            stream=None) -> None:
+    """Column-parallel linear on the all-gathered shards: out [N, f_out] =
+    concat(shards) @ w [f_out, h]^T, reading the shards directly."""
+    _check("sp_ag_colpar_linear_fwd",
+           _lib.sp_ag_colpar_linear_fwd(
+               ctypes.byref(cfg), f_out, _ptrs(shards), _p(w), _p(out),
+               _stream(stream, out)))
 
 
 def sp_activation_bytes(s: int, b: int, h: int, a: int, t: int, mode: int,

@@ -7,9 +7,10 @@ importing the package loads the library that this script builds.
 The library is compiled for sm_100a only and links the CUDA runtime
 statically, so it loads next to any PyTorch build.  Its translation units are
 compiled in parallel: the host entry points with the small kernels
-(``sp_region.cu``), and one unit per (I/O dtype, norm) pair for each of the
-two fast streaming kernels, whose plan tables make up most of the device code
-(``sp_inst_fwd.cu`` / ``sp_inst_bwd.cu`` with ``-DSP_T_BF16 -DSP_LN``).
+(``sp_region.cu``), the tensor-core linears (``sp_gemm.cu``), and one unit
+per (I/O dtype, norm) pair for each of the two fast streaming kernels, whose
+plan tables make up most of the device code (``sp_inst_fwd.cu`` /
+``sp_inst_bwd.cu`` with ``-DSP_T_BF16 -DSP_LN``).
 """
 import concurrent.futures
 import os
@@ -34,7 +35,9 @@ FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a",
 def units():
     """(object path, source path, extra flags) of every translation unit."""
     out = [(os.path.join(OBJDIR, "sp_region.o"),
-            os.path.join(CSRC, "sp_region.cu"), [])]
+            os.path.join(CSRC, "sp_region.cu"), []),
+           (os.path.join(OBJDIR, "sp_gemm.o"),
+            os.path.join(CSRC, "sp_gemm.cu"), [])]
     for kind in ("fwd", "bwd"):
         for tb, tname in ((1, "bf16"), (0, "f32")):
             for ln, nname in ((1, "ln"), (0, "rms")):

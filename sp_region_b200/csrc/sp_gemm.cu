@@ -1,0 +1,213 @@
+// C-ABI entry points of the tensor-parallel linears with the SP collectives
+// fused into them (declared in sp_region.h): the row-parallel linear whose
+// reduce-scatter is the GEMM's own accumulation, with the SP region's bias,
+// dropout and residual add in its epilogue, and the column-parallel linear
+// whose all-gather is its A-operand prologue.  Argument validation, tensor
+// maps and launch; the arithmetic is in sp_gemm.cuh.
+#include <cuda.h>
+#include <math.h>
+#include <string.h>
+
+#include "sp_gemm.cuh"
+#include "sp_host.h"
+#include "sp_plans.h"
+#include "sp_region.h"
+
+using namespace spk;
+using namespace spk_host;
+
+namespace spk {
+SPK_ERROR_WORD_ACCESSOR(error_word_gemm)
+}  // namespace spk
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver, found once through the runtime
+// (the library links no driver library of its own)
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// Map of a bf16 matrix [rows][cols] (row stride ld elements), boxes of 64
+// columns x box_rows rows, 128-byte swizzle, zero fill outside the matrix.
+bool make_map(CUtensorMap* m, const void* base, long long rows, long long cols, long long ld,
+              int box_rows)
+{
+    EncodeTiledFn f = encode_tiled();
+    if (!f) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t tail_bytes() { return (sizeof(GemmTail) + 127) & ~(size_t)127; }
+
+template <int BN, int EPI>
+int launch_gemm(GemmArgs a, const GemmMaps& maps, const DevInfo& dev, cudaStream_t st)
+{
+    constexpr size_t kStage = (size_t)kGemmBM * kGemmBK * 2 + (size_t)BN * kGemmBK * 2;
+    const size_t fixed = 1024 + tail_bytes();   // alignment slack, barriers
+    if ((size_t)dev.smem_optin <= fixed + 2 * kStage) return SP_ERR_UNSUPPORTED;
+    int S = (int)(((size_t)dev.smem_optin - fixed) / kStage);
+    if (S > 16) S = 16;
+    a.stages = S;
+    a.tmem_cols = BN <= 128 ? 128 : 256;
+    const size_t smem = fixed + (size_t)S * kStage;
+    const void* kern = (const void*)k_tp_gemm<BN, EPI>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + kGemmBM - 1) / kGemmBM));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* params[] = {&a, const_cast<GemmMaps*>(&maps)};
+    if (cudaLaunchKernelExC(&cfg, kern, params) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
+}
+
+template <int EPI>
+int launch_gemm_bn(const GemmArgs& a, const GemmMaps& maps, const DevInfo& dev, cudaStream_t st,
+                   int bn)
+{
+    return bn == 256 ? launch_gemm<256, EPI>(a, maps, dev, st)
+                     : launch_gemm<128, EPI>(a, maps, dev, st);
+}
+
+// output features per tile: 256 unless the output is narrower
+int pick_bn(long long n) { return n >= 256 ? 256 : 128; }
+
+int check_gemm_cfg(const sp_cfg* cfg)
+{
+    int rc = check_cfg(cfg);
+    if (rc) return rc;
+    if (cfg->dtype != SP_BF16 || cfg->res_f32) return SP_ERR_UNSUPPORTED;
+    return SP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sp_rowpar_linear_rs_fwd(const sp_cfg* cfg, int64_t f, const void* x, const void* w,
+                            const void* bias, const void* residual, void* residual_out,
+                            uint32_t* mask_bits, void* stream)
+{
+    int rc = check_gemm_cfg(cfg);
+    if (rc) return rc;
+    if (!x || !w || !residual || !residual_out) return SP_ERR_INVALID_ARG;
+    if (f < 1 || f % cfg->t) return SP_ERR_INVALID_ARG;
+    if (f % 8 || cfg->h % 8 || f > (1LL << 31) - 64) return SP_ERR_UNSUPPORTED;
+    if (!mask_bits && cfg->p_drop > 0.0f) return SP_ERR_INVALID_ARG;
+    for (const void* p : {x, w, bias, residual, (const void*)residual_out})
+        if (p && !aligned(p, 16)) return SP_ERR_INVALID_ARG;
+    if (mask_bits && !aligned(mask_bits, 4)) return SP_ERR_INVALID_ARG;
+    DevInfo dev;
+    if ((rc = use_device_of(residual_out, &dev))) return rc;
+
+    long long row0 = 0, rows = 0;
+    call_rows(cfg, &row0, &rows);
+    const long long h = cfg->h;
+    const int bn = pick_bn(h);
+    GemmMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    // x: this call's rows [rows][f]; the t ranks' slices are its column
+    // blocks, so one map covers every rank
+    if (!make_map(&maps.a[0], x, rows, f, f, kGemmBM) || !make_map(&maps.b, w, h, f, f, bn))
+        return SP_ERR_INVALID_ARG;
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = rows;
+    a.N = (int)h;
+    a.K = (int)f;
+    a.rows_per_shard = (int)(rows > 0x7FFFFFFF ? 0x7FFFFFFF : rows);
+    a.nmaps = 1;
+    a.out = residual_out;
+    a.bias = bias;
+    a.residual = residual;
+    a.mask = reinterpret_cast<uint8_t*>(mask_bits);
+    a.mask_row_bytes = (int)(4 * ((h + 31) / 32));
+    a.row0 = row0;
+    a.scale = 1.0f / (1.0f - cfg->p_drop);
+    a.thr = drop_threshold(cfg->p_drop);
+    a.off_lo = (uint32_t)cfg->offset;
+    a.off_hi = (uint32_t)(cfg->offset >> 32);
+    const uint32_t seed_lo = (uint32_t)cfg->seed, seed_hi = (uint32_t)(cfg->seed >> 32);
+    for (int r = 0; r < 10; ++r) {   // Philox key schedule: Weyl increments per round
+        a.keys[r][0] = seed_lo + (uint32_t)r * 0x9E3779B9u;
+        a.keys[r][1] = seed_hi + (uint32_t)r * 0xBB67AE85u;
+    }
+    a.dropout = cfg->p_drop > 0.0f ? 1 : 0;
+    return launch_gemm_bn<0>(a, maps, dev, static_cast<cudaStream_t>(stream), bn);
+}
+
+int sp_ag_colpar_linear_fwd(const sp_cfg* cfg, int64_t f_out, const void* const* shards,
+                            const void* w, void* out, void* stream)
+{
+    int rc = check_gemm_cfg(cfg);
+    if (rc) return rc;
+    if (!shards || !w || !out || f_out < 1) return SP_ERR_INVALID_ARG;
+    if (!(cfg->row_begin == 0 && cfg->row_end == 0)) return SP_ERR_INVALID_ARG;
+    const int t = cfg->t;
+    const long long N = cfg->s * cfg->b, per = N / t, h = cfg->h;
+    if (t > kGemmMaxShards) return SP_ERR_UNSUPPORTED;
+    if (t > 1 && per % kGemmBM) return SP_ERR_UNSUPPORTED;   // a tile lies in one shard
+    if (h % 8 || f_out % 8 || h > (1LL << 31) - 64 || f_out > (1LL << 31) - 256)
+        return SP_ERR_UNSUPPORTED;
+    for (int r = 0; r < t; ++r)
+        if (!shards[r] || !aligned(shards[r], 16)) return SP_ERR_INVALID_ARG;
+    if (!aligned(w, 16) || !aligned(out, 16)) return SP_ERR_INVALID_ARG;
+    DevInfo dev;
+    if ((rc = use_device_of(out, &dev))) return rc;
+
+    const int bn = pick_bn(f_out);
+    GemmMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    for (int r = 0; r < t; ++r)
+        if (!make_map(&maps.a[r], shards[r], per, h, h, kGemmBM)) return SP_ERR_INVALID_ARG;
+    if (!make_map(&maps.b, w, f_out, h, h, bn)) return SP_ERR_INVALID_ARG;
+    GemmArgs a;
+    memset(&a, 0, sizeof(a));
+    a.M = N;
+    a.N = (int)f_out;
+    a.K = (int)h;
+    a.rows_per_shard = (int)per;
+    a.nmaps = t;
+    a.out = out;
+    return launch_gemm_bn<1>(a, maps, dev, static_cast<cudaStream_t>(stream), bn);
+}
+
+}  // extern "C"

@@ -1,0 +1,355 @@
+// Tensor-parallel linears on sm_100a tensor cores (tcgen05), with the
+// sequence-parallel collectives fused into them.
+//
+// "TP and SP explained with pictures", sections "Tensor parallelism, take
+// two: split the inner dimension" and "Add Sequence parallelism": a
+// row-parallel linear gives every rank a full-shape partial sum of its slice
+// of the inner dimension, and with SP those partials are reduce-scattered
+// into token shards; a column-parallel linear needs the full input, which SP
+// all-gathers from the shards ("Chapter 6: TP and SP", sections 2 and 3).
+//
+// On one GPU the t ranks' slices of the inner dimension are consecutive
+// column blocks of x and of the weight, so the reduce-scatter of the t
+// partials IS the K loop of one GEMM: the tensor cores accumulate every
+// rank's contribution into the same fp32 accumulator in tensor memory, rank
+// by rank, and the partials never exist in HBM.  The epilogue then applies
+// the SP region (bias, dropout, residual) to the reduced tile.  For the
+// column-parallel linear the all-gather becomes the prologue: the A-operand
+// tiles are loaded straight from the t shard buffers.
+//
+// k_tp_gemm: one 128 x BN output tile per CTA.
+//   warp 0 (one lane)  TMA producer: A and B tiles (K-major, 128-byte
+//                      swizzle, 64 K-elements per stage) into an S-stage ring
+//   warp 1 (one lane)  MMA issuer: tcgen05.mma kind::f16, M = 128, N = BN,
+//                      K = 16, bf16 x bf16 -> fp32 in tensor memory;
+//                      tcgen05.commit frees each stage and finally signals
+//                      the accumulator
+//   warps 2..5         epilogue: tcgen05.ld of the accumulator rows (warp w
+//                      reads lanes 32 (w % 4) .. +32, one row per thread)
+// Every wait is bounded in time; a wait that runs out records an error and
+// the CTA drains what it issued, frees its tensor memory and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "sp_device.cuh"
+#include "sp_fwd.cuh"
+
+namespace spk {
+
+constexpr int kGemmBM = 128;           // rows per tile (tcgen05 M)
+constexpr int kGemmBK = 64;            // K elements per stage: one 128-byte row
+constexpr int kGemmThreads = 192;      // producer, MMA, 4 epilogue warps
+constexpr int kGemmMaxShards = 16;      // A tensor maps (sequence shards)
+
+struct GemmArgs {
+    // epilogue kind 0: row-parallel SP (bias, dropout, residual, mask)
+    // epilogue kind 1: plain bf16 store
+    long long M;              // output rows (tokens)
+    int N;                    // output features
+    int K;                    // inner dimension
+    int stages;
+    int rows_per_shard;       // A rows per tensor map (shards: M / nmaps)
+    int nmaps;                // A tensor maps (1, or t shards)
+    // epilogue
+    void* out;                // kind 0: residual_out [M][N]; kind 1: out [M][N]
+    const void* bias;         // [N] or NULL (kind 0)
+    const void* residual;     // [M][N] (kind 0)
+    uint8_t* mask;            // [M][mask_row_bytes] or NULL (kind 0)
+    int mask_row_bytes;
+    long long row0;           // global token row of output row 0 (Philox counter)
+    float scale;              // 1 / (1 - p)
+    uint32_t thr;
+    uint32_t off_lo, off_hi;
+    uint32_t keys[10][2];
+    int dropout;
+    uint32_t tmem_cols;
+};
+
+// Tensor maps (built on the host with cuTensorMapEncodeTiled): B = the
+// weight [N][K]; A = the input rows, either one map of [M][K] or one map per
+// sequence shard ([rows_per_shard][K] each).
+struct GemmMaps {
+    CUtensorMap b;
+    CUtensorMap a[kGemmMaxShards];
+};
+
+// Shared memory of k_tp_gemm after the 1024-aligned stages: barriers.
+struct GemmTail {
+    uint64_t full[16];
+    uint64_t empty[16];
+    uint64_t accum;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMA wrappers (PTX ISA: tcgen05.mma, tcgen05.commit, tcgen05.ld,
+// cp.async.bulk.tensor)
+// ---------------------------------------------------------------------------
+
+// Shared-memory matrix descriptor of a K-major tile with 128-byte swizzle:
+// rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), the
+// leading byte offset unused for this layout (1), descriptor version 1,
+// swizzle mode 2.  The tile base must be 1024-byte aligned.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr)
+{
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when every tcgen05.mma this thread issued so far has
+// completed (and its shared-memory operands may be overwritten).
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+
+// 2-D tiled bulk tensor load into this CTA's shared memory; x (the inner
+// coordinate, in elements) is always a multiple of 64, so x * 2 bytes is a
+// multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar, uint64_t policy)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map)
+{
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// 32 consecutive accumulator columns of this thread's lane (one fp32 each).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t r[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// The kernel.  BN: output features per tile (a multiple of 32, <= 256).
+// EPI 0: row-parallel linear + SP epilogue; EPI 1: plain store.
+// Grid: x = column tiles (ceil(N / BN)), y = row tiles (ceil(M / 128)).
+// Dynamic shared memory: 1024 bytes of alignment slack, stages * (16 KB +
+// BN * 128 B), then GemmTail.  A tile's rows lie in one A map
+// (rows_per_shard is a multiple of 128, or the whole of M).
+// ---------------------------------------------------------------------------
+template <int BN, int EPI>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_tp_gemm(const __grid_constant__ GemmArgs a, const __grid_constant__ GemmMaps maps)
+{
+    constexpr uint32_t kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
+    constexpr uint32_t kBBytes = BN * kGemmBK * 2;
+    constexpr uint32_t kStage = kABytes + kBBytes;
+    extern __shared__ __align__(1024) unsigned char gsm_raw[];
+    // the stages need 1024-byte alignment (128-byte swizzle atoms)
+    unsigned char* gsm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~(uintptr_t)1023);
+    const int S = a.stages;
+    GemmTail* tail = reinterpret_cast<GemmTail*>(gsm + (size_t)S * kStage);
+    volatile int* abort = &tail->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = blockIdx.x * BN;
+    const long long m0 = (long long)blockIdx.y * kGemmBM;
+    const int KB = (a.K + kGemmBK - 1) / kGemmBK;
+    // A rows of this tile come from one shard (rows_per_shard % 128 == 0)
+    const int map_id = (int)(m0 / a.rows_per_shard);
+    const int a_row = (int)(m0 - (long long)map_id * a.rows_per_shard);
+    const CUtensorMap* amap = &maps.a[map_id];
+    const CUtensorMap* bmap = &maps.b;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_addr(&tail->full[s]), 1);
+            mbar_init(smem_addr(&tail->empty[s]), 1);
+        }
+        mbar_init(smem_addr(&tail->accum), 1);
+        tail->abort = 0;
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&tail->tmem_base), a.tmem_cols);
+        tmem_fence_before_sync();
+    }
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(bmap);
+        tma_prefetch_desc(amap);
+    }
+    __syncthreads();
+    tmem_fence_after_sync();
+    const uint32_t tbase = tail->tmem_base;
+    grid_dep_launch();
+    grid_dep_wait();   // inputs written by the previous kernel are visible
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer: A (x rows) read by every column tile, kept in L2;
+            // B (weight rows) likewise shared by every row tile
+            const uint64_t pol = policy_evict_last();
+            int issued = 0;
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % S;
+                if (kb >= S &&
+                    !mbar_wait(smem_addr(&tail->empty[s]), (uint32_t)(((kb / S) - 1) & 1), abort,
+                               ERR_WAIT_EMPTY))
+                    break;
+                const uint32_t bar = smem_addr(&tail->full[s]);
+                mbar_arrive_expect_tx(bar, kStage);
+                const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
+                tma_load_2d(sa, amap, kb * kGemmBK, a_row, bar, pol);
+                tma_load_2d(sa + kABytes, bmap, kb * kGemmBK, n0, bar, pol);
+                ++issued;
+            }
+            if (*abort) {
+                // let every issued copy land before the CTA's memory goes away
+                const int first = issued > S ? issued - S : 0;
+                for (int i = first; i < issued; ++i) {
+                    volatile int no_abort = 0;
+                    if (!mbar_wait(smem_addr(&tail->full[i % S]), (uint32_t)((i / S) & 1),
+                                   &no_abort, ERR_DRAIN))
+                        break;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_bf16(kGemmBM, BN);
+            bool ok = true;
+            int kb = 0;
+            for (; kb < KB; ++kb) {
+                const int s = kb % S;
+                if (!mbar_wait(smem_addr(&tail->full[s]), (uint32_t)((kb / S) & 1), abort,
+                               ERR_WAIT_FULL)) {
+                    ok = false;
+                    break;
+                }
+                tmem_fence_after_sync();
+                const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
+                const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + kABytes);
+#pragma unroll
+                for (int k = 0; k < kGemmBK / 16; ++k)
+                    // +32 bytes of K per step: +2 in the start-address field
+                    umma_bf16(tbase, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                umma_commit(smem_addr(&tail->empty[s]));   // stage s may be refilled
+            }
+            // the accumulator is complete (or, on abort, every issued MMA
+            // has finished reading shared memory)
+            umma_commit(smem_addr(&tail->accum));
+            (void)ok;
+        }
+    } else {
+        // epilogue warps 2..5: warp w owns accumulator lanes 32 (w % 4) ..
+        const int q = warp & 3;
+        const long long m = m0 + 32 * q + lane;   // output row of this thread
+        const bool done = mbar_wait(smem_addr(&tail->accum), 0u, abort, ERR_WAIT_FULL);
+        tmem_fence_after_sync();
+        const bool row_ok = done && !*abort && m < a.M;
+        const uint32_t trow = tbase + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(trow + (uint32_t)c0, r);   // warp-wide, outside per-thread branches
+            if (!row_ok) continue;
+#pragma unroll
+            for (int v8 = 0; v8 < 4; ++v8) {
+                const int col = n0 + c0 + 8 * v8;   // first feature of this 8-vector
+                if (col >= a.N) continue;           // N % 8 == 0: vectors are whole
+                F2 y[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+                    y[p] = f2(__uint_as_float(r[8 * v8 + 2 * p]),
+                              __uint_as_float(r[8 * v8 + 2 * p + 1]));
+                if (EPI == 0) {
+                    const long long n = a.row0 + m;   // global token row
+                    if (a.bias) {
+                        F2 b[4];
+                        IO<__nv_bfloat16>::unpack2(load_vec<__nv_bfloat16>(a.bias, col / 8), b);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) y[p] = add2(y[p], b[p]);
+                    }
+                    uint32_t kb8 = 0xFFu;
+                    if (a.dropout) {
+                        kb8 = keep_bits8((uint32_t)(col / 8), (uint32_t)n, a.off_lo, a.off_hi,
+                                         a.keys, a.thr);
+                        const F2 sc2 = f2(a.scale);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p)
+                            y[p] = keep2(mul2(y[p], sc2), (kb8 >> (2 * p)) & 1u,
+                                         (kb8 >> (2 * p + 1)) & 1u);
+                    }
+                    if (a.mask) a.mask[(size_t)m * a.mask_row_bytes + col / 8] = (uint8_t)kb8;
+                    F2 rs[4];
+                    const unsigned char* rrow =
+                        static_cast<const unsigned char*>(a.residual) + (size_t)m * a.N * 2;
+                    IO<__nv_bfloat16>::unpack2(load_vec<__nv_bfloat16>(rrow, col / 8), rs);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) y[p] = add2(rs[p], y[p]);
+                }
+                unsigned char* orow = static_cast<unsigned char*>(a.out) + (size_t)m * a.N * 2;
+                store_vec<__nv_bfloat16>(orow, col / 8, IO<__nv_bfloat16>::pack2v(y));
+            }
+            if (EPI == 0 && a.mask && n0 + c0 + 32 >= a.N && n0 + c0 < a.N) {
+                // the row's last features: zero the mask's padding bytes
+                for (int pb = a.N / 8; pb < a.mask_row_bytes; ++pb)
+                    a.mask[(size_t)m * a.mask_row_bytes + pb] = 0;
+            }
+        }
+    }
+    // every tensor-memory read is done before warp 1 frees the columns
+    tmem_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_fence_after_sync();
+        tmem_dealloc(tbase, a.tmem_cols);
+    }
+}
+
+}  // namespace spk

@@ -83,6 +83,7 @@ const void* bwd_kernel_f32_rms(int id, bool exact);
 // Every translation unit with kernels has its own device error word; these
 // read (and optionally clear) the word of one unit.  0 on success.
 int error_word_host(unsigned* v, int clear);
+int error_word_gemm(unsigned* v, int clear);
 int error_word_fwd_bf16_ln(unsigned* v, int clear);
 int error_word_fwd_bf16_rms(unsigned* v, int clear);
 int error_word_fwd_f32_ln(unsigned* v, int clear);

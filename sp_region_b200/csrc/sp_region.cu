@@ -13,23 +13,17 @@
 #include "sp_entry.cuh"
 #include "sp_fwd.cuh"
 #include "sp_gather.cuh"
+#include "sp_host.h"
 #include "sp_plans.h"
 
 using namespace spk;
+using namespace spk_host;
 
 namespace spk {
 SPK_ERROR_WORD_ACCESSOR(error_word_host)
 }  // namespace spk
 
-namespace {
-
-constexpr int kGeneralThreads = 256;
-
-struct DevInfo {
-    int id;
-    int sms;
-    int smem_optin;
-};
+namespace spk_host {
 
 // Make the device that owns `p` current for this library's CUDA runtime and
 // read its limits.  The caller's framework may have another device current,
@@ -95,6 +89,12 @@ int res_elem_bytes(const sp_cfg* c) { return c->res_f32 ? 4 : elem_bytes(c); }
 bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 uint32_t drop_threshold(float p) { return (uint32_t)floor((double)p * 4294967296.0); }
+
+}  // namespace spk_host
+
+namespace {
+
+constexpr int kGeneralThreads = 256;
 
 size_t round128(size_t x) { return (x + 127) & ~(size_t)127; }
 
@@ -720,6 +720,27 @@ int sp_norm_all_gather_fwd(const sp_cfg* cfg, const void* x, const void* gamma,
                     nullptr, mean, rstd, stream);
 }
 
+int sp_linear_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, int64_t f, const void* x,
+                                           const void* w, const void* bias,
+                                           const void* residual, const void* gamma,
+                                           const void* beta, void* residual_out,
+                                           void* const* gathered, int32_t n_gathered,
+                                           uint32_t* mask_bits, float* mean, float* rstd,
+                                           void* stream)
+{
+    if (!cfg || !gamma || !gathered || n_gathered < 1 || n_gathered > SP_MAX_T)
+        return SP_ERR_INVALID_ARG;
+    int rc = sp_rowpar_linear_rs_fwd(cfg, f, x, w, bias, residual, residual_out, mask_bits,
+                                     stream);
+    if (rc) return rc;
+    // the stored residual sum is the norm's input; the entry kernel
+    // normalises each row and writes it to every gathered buffer
+    sp_cfg c = *cfg;
+    c.fwd_plan = 0;
+    return sp_norm_all_gather_fwd(&c, residual_out, gamma, beta, gathered, n_gathered, mean,
+                                  rstd, stream);
+}
+
 int sp_all_gather(const sp_cfg* cfg, const void* const* shards, void* const* outs,
                   int32_t n_out, void* stream)
 {
@@ -810,7 +831,8 @@ int sp_device_error(int32_t device, int32_t* code, int32_t clear)
     int (*const words[])(unsigned*, int) = {
         error_word_host,         error_word_fwd_bf16_ln, error_word_fwd_bf16_rms,
         error_word_fwd_f32_ln,   error_word_fwd_f32_rms, error_word_bwd_bf16_ln,
-        error_word_bwd_bf16_rms, error_word_bwd_f32_ln,  error_word_bwd_f32_rms};
+        error_word_bwd_bf16_rms, error_word_bwd_f32_ln,  error_word_bwd_f32_rms,
+        error_word_gemm};
     unsigned first = 0;
     for (auto fn : words) {
         unsigned v = 0;

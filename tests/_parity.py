@@ -293,7 +293,7 @@ def assert_close_extra(name, gpu, ref, mag, dtype, extra, k=K_FP32):
 
 
 def check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered=1,
-                  rows_mean_rstd=True):
+                  rows_mean_rstd=True, mag_rout=None):
     """Compare a device forward with the oracle's (same rows).
 
     The norm output is held to the strict bound (one I/O ulp plus the fp32
@@ -303,8 +303,10 @@ def check_forward(w, got, ref, parts, bias, res, gamma, beta, n_gathered=1,
     The norm step itself, fed the oracle's stored sums, is held to the
     strict bound everywhere by check_norm_step."""
     dt = w.torch_dtype
+    if mag_rout is None:
+        mag_rout = mag_residual_out(w, parts, bias, res)
     assert_close("residual_out", got["residual_out"], ref["residual_out"],
-                 mag_residual_out(w, parts, bias, res), w.res_torch_dtype)
+                 mag_rout, w.res_torch_dtype)
     ex_o, ex_m, ex_r = propagated_dx(w, got["residual_out"],
                                      ref["residual_out"], ref["mean"],
                                      ref["rstd"], gamma)
@@ -407,3 +409,25 @@ def mags_backward(w, dparts, drnext, x, gamma, mean, rstd):
                 dgamma_terms=(dn.abs() * xh.abs()).sum(0).numpy(),
                 dbeta_terms=dn.abs().sum(0).numpy(),
                 dbias_terms=(scale * m).sum(0).numpy())
+
+
+def mag_linear_rout(w, x, wt, bias, res, y_ref):
+    """Magnitude term for residual_out of the row-parallel linear: the
+    epilogue's fp32 terms, plus the tensor-core accumulation of K products.
+    Each of the K / 16 accumulator updates (one per tcgen05.mma of K = 16)
+    can move the fp32 sum by at most 2^-23 of its magnitude, bounded by
+    M = sum_i |x_i w_i|; the bound (K/16 + 16) 2^-23 M is expressed in units
+    of assert_close's 16 * 2^-24 term."""
+    K = x.shape[1]
+    scale = 1.0 / (1.0 - float(np.float32(w.p_drop)))
+    gm = (x.double().abs() @ wt.double().abs().T)
+    m = res.double().abs() + scale * torch.as_tensor(np.abs(y_ref))
+    if bias is not None:
+        m = m + scale * bias.double().abs()
+    return (m + ((K / 16 + 16) / 8.0) * scale * gm).numpy()
+
+
+def mag_linear_out(x, wt):
+    """The same accumulation bound for a plain linear's output."""
+    K = x.shape[1]
+    return (((K / 16 + 16) / 8.0) * (x.double().abs() @ wt.double().abs().T)).numpy()
