@@ -101,6 +101,12 @@ def _lib():
         L.orc_linear_rs_fwd_rows.restype = ctypes.c_int
         L.orc_ag_colpar_fwd.argtypes = [ctypes.c_int, i64, i64, i64, vp, vp, vp]
         L.orc_ag_colpar_fwd.restype = ctypes.c_int
+        L.orc_ring_attention.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_double,
+                                         vp, vp, vp, vp, dp]
+        L.orc_ring_attention.restype = ctypes.c_int
+        L.orc_ring_attention_rows.argtypes = [i64, i64, ctypes.c_int, ctypes.c_double,
+                                              vp, vp, i64, vp, vp, vp, dp]
+        L.orc_ring_attention_rows.restype = ctypes.c_int
         L.orc_activation_bytes.argtypes = [i64, i64, i64, i64, i32, i32,
                                            ctypes.c_double]
         L.orc_activation_bytes.restype = ctypes.c_double
@@ -417,3 +423,37 @@ def ag_colpar_fwd(shards, w) -> torch.Tensor:
     if rc != 0:
         raise ValueError(f"oracle column-parallel forward rejected the shapes ({rc})")
     return out
+
+
+# ----------------------------------------------------------------------------
+# context parallelism: ring attention
+# ----------------------------------------------------------------------------
+
+def ring_attention(q, k, v, t: int, scale: float):
+    """Ring attention over t ranks; q, k, v [bh, s, d] bf16.  Returns
+    (out [bh, s, d] bf16, lse [bh, s] float64)."""
+    q, k, v = (_cpu(x, BF16) for x in (q, k, v))
+    bh, s, d = q.shape
+    out = torch.empty((bh, s, d), dtype=torch.bfloat16)
+    lse = np.zeros((bh, s))
+    rc = _lib().orc_ring_attention(bh, s, d, t, scale, _ptr(q), _ptr(k), _ptr(v),
+                                   _ptr(out), lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle ring attention rejected the shapes ({rc})")
+    return out, lse
+
+
+def ring_attention_rows(q_rows, rows, k, v, t: int, scale: float):
+    """Ring attention of one head on selected query rows: q_rows [n, d]
+    (the queries of tokens rows[i]), k, v [s, d]."""
+    q_rows, k, v = (_cpu(x, BF16) for x in (q_rows, k, v))
+    ids = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    s, d = k.shape
+    out = torch.empty((len(ids), d), dtype=torch.bfloat16)
+    lse = np.zeros(len(ids))
+    rc = _lib().orc_ring_attention_rows(s, d, t, scale, _ptr(q_rows), ids.ctypes.data,
+                                        len(ids), _ptr(k), _ptr(v), _ptr(out),
+                                        lse.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle ring attention rejected the shapes ({rc})")
+    return out, lse

@@ -680,6 +680,118 @@ int orc_ag_colpar_fwd(int t, int64_t shard_rows, int64_t h, int64_t f_out,
 }
 
 /* ------------------------------------------------------------------------- */
+/* Context parallelism: ring attention                                         */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * Ring attention ("Sequence Parallelism math", section "Context parallelism
+ * and ring attention"): Q, K and V are sharded along the sequence, rank r
+ * holding the contiguous block r of s/t tokens.  The ranks form a ring; at
+ * step i (0 .. t-1) rank r holds K/V block (r - i) mod t (each step every
+ * rank passes its block to the next rank), attends its queries against it
+ * and folds the result into an online softmax: for each query the running
+ * maximum m of its scores so far, the sum l of exp(score - m) and the
+ * exp(score - m)-weighted sum o of the values.  When a block raises the
+ * maximum, l and o are rescaled by exp(m_old - m_new).  After the t steps
+ * every query has seen every key and the output is o / l.
+ *   score(n, j) = scale * sum_c q[n, c] * k[j, c]
+ *   q, k, v  [bh][s][d] bf16 (bh = batch * heads, each head its own problem)
+ *   out      [bh][s][d] bf16, rounded once
+ *   lse      [bh][s] double, m + log(l) (the log-sum-exp of the scores), or NULL
+ */
+int orc_ring_attention(int64_t bh, int64_t s, int64_t d, int t, double scale, const void* q,
+                       const void* k, const void* v, void* out, double* lse)
+{
+    if (bh < 1 || s < 1 || d < 1 || t < 1 || s % t) return -1;
+    const int64_t per = s / t;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)per);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!sc || !o) { free(sc); free(o); return -2; }
+    for (int64_t g = 0; g < bh; ++g) {
+        const int64_t base = g * s * d;
+        for (int64_t n = 0; n < s; ++n) {
+            const int r = (int)(n / per);
+            double m = -INFINITY, l = 0.0;
+            for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+            for (int i = 0; i < t; ++i) {
+                const int64_t blk = ((int64_t)r - i + t) % t;
+                /* the block's scores and their maximum */
+                double bmax = -INFINITY;
+                for (int64_t jj = 0; jj < per; ++jj) {
+                    const int64_t j = blk * per + jj;
+                    double acc = 0.0;
+                    for (int64_t c = 0; c < d; ++c)
+                        acc += ld(q, base + n * d + c, ORC_BF16) * ld(k, base + j * d + c, ORC_BF16);
+                    sc[jj] = scale * acc;
+                    if (sc[jj] > bmax) bmax = sc[jj];
+                }
+                /* fold the block into the running softmax */
+                const double mnew = bmax > m ? bmax : m;
+                const double alpha = exp(m - mnew);   /* exp(-inf) = 0 at the first step */
+                l *= alpha;
+                for (int64_t c = 0; c < d; ++c) o[c] *= alpha;
+                for (int64_t jj = 0; jj < per; ++jj) {
+                    const int64_t j = blk * per + jj;
+                    const double p = exp(sc[jj] - mnew);
+                    l += p;
+                    for (int64_t c = 0; c < d; ++c) o[c] += p * ld(v, base + j * d + c, ORC_BF16);
+                }
+                m = mnew;
+            }
+            for (int64_t c = 0; c < d; ++c) st(out, base + n * d + c, ORC_BF16, o[c] / l);
+            if (lse) lse[g * s + n] = m + log(l);
+        }
+    }
+    free(sc); free(o);
+    return 0;
+}
+
+/* The same on selected query rows of one head g: rows[i] is a token index;
+ * out [nrows][d], lse [nrows]. */
+int orc_ring_attention_rows(int64_t s, int64_t d, int t, double scale, const void* q_rows,
+                            const int64_t* rows, int64_t nrows, const void* k, const void* v,
+                            void* out, double* lse)
+{
+    if (s < 1 || d < 1 || t < 1 || s % t) return -1;
+    const int64_t per = s / t;
+    double* sc = (double*)malloc(sizeof(double) * (size_t)per);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!sc || !o) { free(sc); free(o); return -2; }
+    for (int64_t i0 = 0; i0 < nrows; ++i0) {
+        const int r = (int)(rows[i0] / per);
+        double m = -INFINITY, l = 0.0;
+        for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+        for (int i = 0; i < t; ++i) {
+            const int64_t blk = ((int64_t)r - i + t) % t;
+            double bmax = -INFINITY;
+            for (int64_t jj = 0; jj < per; ++jj) {
+                const int64_t j = blk * per + jj;
+                double acc = 0.0;
+                for (int64_t c = 0; c < d; ++c)
+                    acc += ld(q_rows, i0 * d + c, ORC_BF16) * ld(k, j * d + c, ORC_BF16);
+                sc[jj] = scale * acc;
+                if (sc[jj] > bmax) bmax = sc[jj];
+            }
+            const double mnew = bmax > m ? bmax : m;
+            const double alpha = exp(m - mnew);
+            l *= alpha;
+            for (int64_t c = 0; c < d; ++c) o[c] *= alpha;
+            for (int64_t jj = 0; jj < per; ++jj) {
+                const int64_t j = blk * per + jj;
+                const double p = exp(sc[jj] - mnew);
+                l += p;
+                for (int64_t c = 0; c < d; ++c) o[c] += p * ld(v, j * d + c, ORC_BF16);
+            }
+            m = mnew;
+        }
+        for (int64_t c = 0; c < d; ++c) st(out, i0 * d + c, ORC_BF16, o[c] / l);
+        if (lse) lse[i0] = m + log(l);
+    }
+    free(sc); free(o);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Activation memory per layer and device ("Sequence Parallelism math",      */
 /* equations A_layer, A_TP, A_TP+SP).  mode 0: A_layer = sbh(34 + 5as/h);    */
 /* 1: A_TP = sbh(10 + 24/t + 5as/(ht)); 2: A_TP+SP = (sbh/t)(34 + 5as/h).     */

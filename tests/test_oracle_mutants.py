@@ -96,6 +96,15 @@ MUTANTS = {
     "column-parallel linear skips the all-gather order": (
         "orc_all_gather(t, shard_rows, h, (const double* const*)sh, X);",
         "for (int64_t q = 0; q < N * h; ++q) X[q] = sh[0][q % (shard_rows * h)];"),
+    "ring attention skips the last ring step": (
+        "            for (int i = 0; i < t; ++i) {\n                const int64_t blk = ((int64_t)r - i + t) % t;\n                /* the block's scores",
+        "            for (int i = 0; i < t - 1; ++i) {\n                const int64_t blk = ((int64_t)r - i + t) % t;\n                /* the block's scores"),
+    "ring attention does not rescale the values when the maximum grows": (
+        "                l *= alpha;\n                for (int64_t c = 0; c < d; ++c) o[c] *= alpha;\n                for (int64_t jj = 0; jj < per; ++jj) {\n                    const int64_t j = blk * per + jj;\n                    const double p = exp(sc[jj] - mnew);\n                    l += p;\n                    for (int64_t c = 0; c < d; ++c) o[c] += p * ld(v, base",
+        "                l *= alpha;\n                for (int64_t jj = 0; jj < per; ++jj) {\n                    const int64_t j = blk * per + jj;\n                    const double p = exp(sc[jj] - mnew);\n                    l += p;\n                    for (int64_t c = 0; c < d; ++c) o[c] += p * ld(v, base"),
+    "ring attention ignores the scale": (
+        "                    sc[jj] = scale * acc;\n                    if (sc[jj] > bmax) bmax = sc[jj];\n                }\n                /* fold",
+        "                    sc[jj] = acc;\n                    if (sc[jj] > bmax) bmax = sc[jj];\n                }\n                /* fold"),
     "ring volume without (t-1)/t": (
         "double phase = (double)(t - 1) / (double)t * V;",
         "double phase = V;"),

@@ -882,3 +882,55 @@ def test_ag_colpar_is_the_correctly_rounded_product_of_the_gathered_input(orc, t
     if t > 1:
         rev = orc.ag_colpar_fwd(shards[::-1], w).double().numpy()
         assert not np.array_equal(rev, out)
+
+
+# ----------------------------------------------------------------------------
+# context parallelism: ring attention with an online softmax
+# ----------------------------------------------------------------------------
+
+def _attn_ref(q, k, v, scale):
+    """softmax(q k^T * scale) v and the log-sum-exp, float64 (torch)."""
+    sc = (q.double() @ k.double().transpose(-1, -2)) * scale
+    return torch.softmax(sc, -1) @ v.double(), torch.logsumexp(sc, -1)
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 8])
+def test_ring_attention_equals_plain_attention(orc, t):
+    """After the t ring steps the online softmax has reached the plain
+    softmax attention over all keys: the output is its bf16 rounding and the
+    log-sum-exp matches torch.logsumexp (float64)."""
+    bh, s, d = 2, 32, 16
+    q, k, v = (_bf16((bh, s, d), 40 + i) for i in range(3))
+    scale = d ** -0.5
+    out, lse = orc.ring_attention(q, k, v, t, scale)
+    ref, ref_lse = _attn_ref(q, k, v, scale)
+    e = np.floor(np.log2(np.maximum(np.abs(ref.numpy()), 2.0 ** -126)))
+    assert (np.abs(out.double().numpy() - ref.numpy()) <= 2.0 ** (e - 8) * 1.001 + 1e-12).all()
+    assert np.allclose(lse, ref_lse.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_ring_attention_special_cases(orc):
+    """All scores equal (q = 0): every query averages all values.  One key
+    far above the rest: the output is that key's value (to the bf16 ulp)."""
+    bh, s, d, t = 1, 16, 8, 4
+    k, v = _bf16((bh, s, d), 50), _bf16((bh, s, d), 51)
+    q = torch.zeros((bh, s, d), dtype=torch.bfloat16)
+    out, lse = orc.ring_attention(q, k, v, t, 1.0)
+    mean = v.double().mean(1, keepdim=True).expand(bh, s, d)
+    assert torch.allclose(out.double(), mean, rtol=2 ** -8, atol=1e-6)
+    assert np.allclose(lse, np.log(s))
+    k2 = torch.zeros((bh, s, d), dtype=torch.bfloat16)
+    k2[0, 11] = 8.0                      # key 11 in rank 2's block
+    q2 = torch.ones((bh, s, d), dtype=torch.bfloat16)
+    out2, _ = orc.ring_attention(q2, k2, v, t, 1.0)
+    assert torch.equal(out2[0], v[0, 11].expand(s, d))
+
+
+def test_ring_attention_rows_agree_with_the_whole(orc):
+    bh, s, d, t = 1, 64, 16, 4
+    q, k, v = (_bf16((bh, s, d), 60 + i) for i in range(3))
+    out, lse = orc.ring_attention(q, k, v, t, 0.25)
+    rows = [0, 15, 16, 47, 63]
+    o2, l2 = orc.ring_attention_rows(q[0, rows], rows, k[0], v[0], t, 0.25)
+    assert torch.equal(o2, out[0, rows])
+    assert np.array_equal(l2, lse[0, rows])
