@@ -40,6 +40,7 @@ sys.path.insert(0, ROOT)
 METRIC = "SP-boundary fwd+bwd achieved HBM GB/s (% of B200 peak); tokens/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 # ----------------------------------------------------------------------------
@@ -112,6 +113,17 @@ def measured_peak():
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback (no MEASURED_PEAKS.json)"
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s for a kernel timed on its own (the burst figure)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback (no MEASURED_PEAKS.json)"
 
 
 def kernel_sources_sha():
@@ -385,10 +397,15 @@ def run_ours(args):
     e2e = None
     cpu = None
     workloads = None
+    linears = None
+    attention = None
     if args.op == "boundary":
         e2e = run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world)
         if world == 1 and args.workloads:
             workloads = time_workloads(args, sp, torch, dev, peak)
+        if world == 1 and not args.skip_linears:
+            linears = time_linears(args, sp, torch, dev)
+            attention = time_ring_attention(args, sp, torch, dev)
         if rank == 0 and world == 1 and not args.skip_cpu_baseline:
             cpu = cpu_baseline(w, fb, bb, budget_s=args.cpu_seconds)
 
@@ -420,6 +437,8 @@ def run_ours(args):
         "roofline": roofline,
         "kernels": kern,
         "workloads": workloads,
+        "tp_linears": linears,
+        "ring_attention": attention,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": 3 * K,
@@ -539,6 +558,125 @@ def time_workloads(args, sp, torch, dev, peak):
         torch.cuda.empty_cache()
     assert sp.sp_device_error(dev.index) == 0, "device-side wait timed out"
     return out
+
+
+def time_linears(args, sp, torch, dev):
+    """The tensor-parallel linears around the boundary at the C2 layer shape
+    (s=2048, b=4, h=6144, t=8), the FFN down-projection f = 4h = 24576 as
+    the row-parallel linear and the up-projection h -> 4h as the
+    column-parallel one, synthetic bf16 inputs:
+
+      fused      sp_linear_rs_bias_dropout_add_norm_fwd: the GEMM whose
+                 accumulator reduces the t partials, with bias / dropout /
+                 residual in its epilogue, then norm + all-gather
+      gemm       sp_rowpar_linear_rs_fwd alone (tensor roofline)
+      unfused    t GEMMs each writing its partial [N, h] to HBM, then
+                 sp_rs_bias_dropout_add_norm_fwd on the t partials
+      colpar     sp_ag_colpar_linear_fwd reading the t shards directly
+    """
+    import gc
+    import sp_synth
+    w = sp_synth.WORKLOADS["C2"]
+    N, h, t = w.rows, w.h, w.t
+    f = 4 * h
+    per = f // t
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_src = measured_tensor_peak()
+    g = torch.Generator(device=dev).manual_seed(4242)
+    x = (torch.randn((N, f), generator=g, device=dev) * f ** -0.5).to(torch.bfloat16)
+    wt = torch.randn((h, f), generator=g, device=dev).to(torch.bfloat16)
+    bias, gamma, beta = sp_synth.draw_params(w, dev)
+    res = sp_synth.draw_residual(w, dev)
+    rout = torch.empty((N, h), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((N, h), dtype=torch.bfloat16, device=dev)
+    mask = torch.empty((N, (h + 31) // 32), dtype=torch.int32, device=dev)
+    mean = torch.empty(N, dtype=torch.float32, device=dev)
+    rstd = torch.empty(N, dtype=torch.float32, device=dev)
+    cfg = sp.make_cfg(w.s, w.b, h, t, dtype="bf16", norm=w.norm, eps=w.eps,
+                      p_drop=w.p_drop, seed=w.drop_seed, offset=w.drop_offset)
+    flops = 2.0 * N * f * h
+    K = 10
+
+    def rec(kernel, ms, nflops=flops):
+        tf = nflops / (ms * 1e-3) / 1e12
+        return {"kernel": kernel, "avg_ms": round(ms, 4), "tflops": round(tf, 1),
+                "frac": round(tf / peak, 4), "flops_per_launch": nflops}
+
+    fused_ms = time_launches(torch, stream, lambda: sp.sp_linear_rs_bias_dropout_add_norm_fwd(
+        cfg, f, x, wt, bias, res, gamma, beta, rout, [out], mask, mean, rstd,
+        stream=stream), K, 3)
+    gemm_ms = time_launches(torch, stream, lambda: sp.sp_rowpar_linear_rs_fwd(
+        cfg, f, x, wt, bias, res, rout, mask, stream=stream), K, 3)
+    # the unfused path: each rank's slice in its own buffers, its partial
+    # written to HBM, then the boundary on the t partials
+    xs = [x[:, k * per:(k + 1) * per].contiguous() for k in range(t)]
+    ws = [wt[:, k * per:(k + 1) * per].contiguous() for k in range(t)]
+    parts = [torch.empty((N, h), dtype=torch.bfloat16, device=dev) for _ in range(t)]
+    cfg1 = sp.make_cfg(N, 1, per, 1, dtype="bf16")
+
+    def unfused():
+        for k in range(t):
+            sp.sp_ag_colpar_linear_fwd(cfg1, h, [xs[k]], ws[k], parts[k], stream=stream)
+        sp.sp_rs_bias_dropout_add_norm_fwd(cfg, parts, bias, res, gamma, beta, rout,
+                                           [out], mask, mean, rstd, stream=stream)
+    unfused_ms = time_launches(torch, stream, unfused, K, 3)
+    del xs, ws, parts, x, wt
+    gc.collect()
+    torch.cuda.empty_cache()
+    # the column-parallel up-projection from the t shards of the norm output
+    fo = 4 * h
+    w_in = (torch.randn((fo, h), generator=g, device=dev) * h ** -0.5).to(torch.bfloat16)
+    z = torch.empty((N, fo), dtype=torch.bfloat16, device=dev)
+    shards = [out[r * (N // t):(r + 1) * (N // t)] for r in range(t)]
+    cfg_c = sp.make_cfg(w.s, w.b, h, t, dtype="bf16")
+    col_ms = time_launches(torch, stream, lambda: sp.sp_ag_colpar_linear_fwd(
+        cfg_c, fo, shards, w_in, z, stream=stream), K, 3)
+    assert sp.sp_device_error(dev.index) == 0, "device-side wait timed out"
+    r = {
+        "workload": (f"C2 layer: s={w.s} b={w.b} h={h} t={t}; row-parallel FFN "
+                     f"down-projection f={f} -> h, then the SP boundary (LN, p=0.1, "
+                     f"bias); column-parallel up-projection h -> {fo}; bf16"),
+        "peak_tflops": peak, "peak_source": peak_src,
+        "fused": rec("k_tp_gemm (SP epilogue) + k_norm_ag", fused_ms),
+        "gemm": rec("k_tp_gemm (SP epilogue)", gemm_ms),
+        "unfused": rec(f"{t} x k_tp_gemm (partials to HBM) + k_fwd_tma", unfused_ms),
+        "colpar": rec("k_tp_gemm (all-gather prologue)", col_ms, 2.0 * N * h * fo),
+        "fused_speedup": round(unfused_ms / fused_ms, 3),
+    }
+    del w_in, z, out, rout, res
+    gc.collect()
+    torch.cuda.empty_cache()
+    return r
+
+
+def time_ring_attention(args, sp, torch, dev):
+    """Ring attention over t = 16 context-parallel ranks at the long-sequence
+    workload's length (s = 32768, head dimension 128 = 12288 / 96), two of its
+    96 heads, b = 1, synthetic bf16 q, k, v ~ N(0, 1), scale 1/sqrt(128).
+    FLOPs per call: 4 s^2 d per head (Q K^T and P V)."""
+    import gc
+    b, heads, s, t, d = 1, 2, 32768, 16, 128
+    peak, peak_src = measured_tensor_peak()
+    g = torch.Generator(device=dev).manual_seed(99)
+    q, k, v = (torch.randn((b, heads, s, d), generator=g, device=dev).to(torch.bfloat16)
+               for _ in range(3))
+    out = torch.empty_like(q)
+    lse = torch.empty((b, heads, s), dtype=torch.float32, device=dev)
+    cfg = sp.make_cfg(s, b, heads * d, t, dtype="bf16")
+    stream = torch.cuda.current_stream(dev)
+    ms = time_launches(torch, stream, lambda: sp.sp_ring_attention_fwd(
+        cfg, heads, d ** -0.5, q, k, v, out, lse, stream=stream), 3, 3)
+    assert sp.sp_device_error(dev.index) == 0, "device-side wait timed out"
+    flops = 4.0 * s * s * d * heads * b
+    tf = flops / (ms * 1e-3) / 1e12
+    del q, k, v, out, lse
+    gc.collect()
+    torch.cuda.empty_cache()
+    return {"workload": (f"C5 attention core: s={s}, t={t} ranks of {s // t} tokens, "
+                         f"head dim {d}, {heads} heads, b={b}, bf16, full attention"),
+            "kernel": "k_ring_attn", "avg_ms": round(ms, 3), "tflops": round(tf, 1),
+            "frac": round(tf / peak, 4), "peak_tflops": peak, "peak_source": peak_src,
+            "flops_per_launch": flops}
 
 
 def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
@@ -854,6 +992,9 @@ def main():
     ap.add_argument("--reference-cores", type=int, default=0,
                     help="processes for --impl reference (0: every core, up to 64)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-linears", action="store_true",
+                    help="skip timing the tensor-parallel linears and the ring "
+                         "attention (N = 1)")
     ap.add_argument("--workloads", default="C2,C3,C4,C5",
                     help="after the timed steps, time the forward and backward "
                          "of these workloads one by one (N = 1; '' for none)")

@@ -357,6 +357,56 @@ int sp_linear_rs_bias_dropout_add_norm_fwd(const sp_cfg* cfg, int64_t f, const v
 int sp_ag_colpar_linear_fwd(const sp_cfg* cfg, int64_t f_out, const void* const* shards,
                             const void* w, void* out, void* stream);
 
+/*
+ * The backward with dY written to n_dY full buffers: each row of the
+ * dropout gradient goes to every buffer, as the forward writes its
+ * normalised rows to every gathered buffer.  With t real ranks, rank r runs
+ * its row range (cfg->row_begin/row_end) and passes the t ranks' dY buffers
+ * (peers' through peer pointers): the all-gather of dY, the reduce-scatter's
+ * backward ("Sequence Parallelism math", section "The collective
+ * substitution"), is then done by the kernels' own stores, and every rank's
+ * copy is complete once every rank's call has finished.  Arguments are
+ * those of sp_rs_norm_dropout_bwd with dY replaced by a HOST array of n_dY
+ * (1 .. SP_MAX_T) device pointers, each [s,b,h] indexed by global row.
+ */
+int sp_rs_norm_dropout_bwd_ag(const sp_cfg* cfg, const void* const* dn_partials,
+                              const void* dR_next, const void* residual_out,
+                              const void* gamma, const uint32_t* mask_bits,
+                              const float* mean, const float* rstd, void* dresidual_in,
+                              void* const* dY, int32_t n_dY, float* dgamma, float* dbeta,
+                              float* dbias, void* workspace, size_t workspace_bytes,
+                              void* stream);
+
+/*
+ * Ring attention (context parallelism) over t ranks, forward.
+ *
+ * Defined by: "Sequence Parallelism math", sections "Where SP stops: the
+ * attention core and long sequences" and "Context parallelism and ring
+ * attention": Q, K and V are sharded along the sequence, rank r holding the
+ * contiguous block r of s/t tokens; at step i rank r attends its queries
+ * against K/V block (r - i) mod t and folds the scores into an online
+ * softmax (running maximum m, sum l of exp(score - m), weighted values o),
+ * so after t steps every query has seen every key.
+ *
+ * For every batch b, head, and query n (its rank r = n / (s/t)):
+ *   score(n, j) = scale * sum_c q[n, c] * k[j, c]   over all s keys j,
+ *   visited block by block in ring order (block r first), 128 keys a tile
+ *   out[n, :] = round( sum_j exp(score(n, j) - m) v[j, :] / l )
+ *   lse[n]    = m + log(l)  (natural log; NULL: not written)
+ * Attention is full (every query sees every key), as on the page.
+ *
+ * cfg: s = sequence length, b = batch, t = ranks of the ring, dtype SP_BF16,
+ * h = heads * 128 (head dimension 128), no row range.  q, k, v, out:
+ * [b][heads][s][128] bf16, 16-byte aligned; lse [b][heads][s] fp32 or NULL.
+ * Requirements: s % 128 == 0 and (s / t) % 128 == 0, b * heads * s < 2^31
+ * (else SP_ERR_UNSUPPORTED); scale > 0 (else SP_ERR_INVALID_ARG).  The
+ * probabilities enter the second product as bf16; both products accumulate
+ * in fp32 in tensor memory.
+ */
+int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const void* q,
+                          const void* k, const void* v, void* out, float* lse,
+                          void* stream);
+
 /* Bytes of device scratch sp_rs_norm_dropout_bwd needs for cfg on CUDA
  * device `device`: the slices of 3*h fp32 parameter-gradient partial sums
  * that the kernel the call picks writes, for 16-byte aligned pointers or for

@@ -35,7 +35,8 @@ EXPORTS = ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
            "sp_debug_wait_timeout", "sp_plan_count",
            "sp_rs_norm_dropout_bwd_noalloc", "sp_norm_all_gather_fwd",
            "sp_rowpar_linear_rs_fwd", "sp_linear_rs_bias_dropout_add_norm_fwd",
-           "sp_ag_colpar_linear_fwd")
+           "sp_ag_colpar_linear_fwd", "sp_rs_norm_dropout_bwd_ag",
+           "sp_ring_attention_fwd")
 
 
 class SPError(RuntimeError):
@@ -83,10 +84,15 @@ def _load() -> ctypes.CDLL:
     lib.sp_plan_count.argtypes = [ctypes.POINTER(i32), ctypes.POINTER(i32)]
     lib.sp_rs_norm_dropout_bwd_noalloc.argtypes = [
         cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.sp_rs_norm_dropout_bwd_ag.argtypes = [
+        cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp,
+        ctypes.c_size_t, vp]
     lib.sp_rowpar_linear_rs_fwd.argtypes = [cfgp, i64, vp, vp, vp, vp, vp, vp, vp]
     lib.sp_linear_rs_bias_dropout_add_norm_fwd.argtypes = [
         cfgp, i64, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, vp, vp, vp]
     lib.sp_ag_colpar_linear_fwd.argtypes = [cfgp, i64, vp, vp, vp, vp]
+    lib.sp_ring_attention_fwd.argtypes = [cfgp, i32, ctypes.c_float, vp, vp, vp,
+                                          vp, vp, vp]
     for f in EXPORTS:
         getattr(lib, f).restype = (ctypes.c_char_p if f == "sp_status_string"
                                    else ctypes.c_int)
@@ -196,6 +202,23 @@ def sp_rs_norm_dropout_bwd(cfg: sp_cfg, dn_partials, dR_next, residual_out,
                _stream(stream, residual_out)))
 
 
+def sp_rs_norm_dropout_bwd_ag(cfg: sp_cfg, dn_partials, dR_next, residual_out,
+                              gamma, mask_bits, mean, rstd, dresidual_in, dY,
+                              dgamma, dbeta, dbias, workspace,
+                              stream=None) -> None:
+    """The backward with every row of dY written to each buffer in ``dY``
+    (every rank's copy: the all-gather done by the kernel's stores)."""
+    dY = list(dY)
+    _check("sp_rs_norm_dropout_bwd_ag",
+           _lib.sp_rs_norm_dropout_bwd_ag(
+               ctypes.byref(cfg), _ptrs(dn_partials), _p(dR_next),
+               _p(residual_out), _p(gamma), _p(mask_bits), _p(mean), _p(rstd),
+               _p(dresidual_in), _ptrs(dY), len(dY), _p(dgamma), _p(dbeta),
+               _p(dbias), _p(workspace),
+               workspace.numel() * workspace.element_size(),
+               _stream(stream, residual_out)))
+
+
 def sp_rs_norm_dropout_bwd_noalloc(cfg: sp_cfg, dn_partials, dR_next,
                                    residual_out, gamma, mask_bits, mean, rstd,
                                    dresidual_in, dY, dgamma, dbeta, dbias,
@@ -248,6 +271,16 @@ def sp_ag_colpar_linear_fwd(cfg: sp_cfg, f_out: int, shards, w, out,
            _lib.sp_ag_colpar_linear_fwd(
                ctypes.byref(cfg), f_out, _ptrs(shards), _p(w), _p(out),
                _stream(stream, out)))
+
+
+def sp_ring_attention_fwd(cfg: sp_cfg, heads: int, scale: float, q, k, v, out,
+                          lse=None, stream=None) -> None:
+    """Ring attention over cfg.t context-parallel ranks: q, k, v, out
+    [b, heads, s, 128] bf16, lse [b, heads, s] fp32 or None."""
+    _check("sp_ring_attention_fwd",
+           _lib.sp_ring_attention_fwd(ctypes.byref(cfg), heads, scale, _p(q),
+                                      _p(k), _p(v), _p(out), _p(lse),
+                                      _stream(stream, out)))
 
 
 def sp_activation_bytes(s: int, b: int, h: int, a: int, t: int, mode: int,

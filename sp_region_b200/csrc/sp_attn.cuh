@@ -1,0 +1,367 @@
+// Ring attention (context parallelism) on sm_100a tensor cores.
+//
+// "Sequence Parallelism math", section "Context parallelism and ring
+// attention": Q, K and V are sharded along the sequence, rank r holding the
+// contiguous block r of s/t tokens; at step i rank r attends its queries
+// against K/V block (r - i) mod t and folds the result into an online
+// softmax, so after t steps every query has seen every key and no rank ever
+// holds more than an (s/t) x (s/t) tile of scores.
+//
+// On one GPU the t ranks' blocks are consecutive key ranges of one K/V
+// tensor, and a CTA whose queries lie in rank r's block visits the key tiles
+// in ring order: block r first, then r-1, r-2, ... (mod t), 128 keys per
+// tile.
+//
+// k_ring_attn: one CTA per (128-query tile, head); head dimension 128.
+//   warp 0 (one lane)  TMA producer: Q once, K and V tiles (2 stages each)
+//   warp 1 (one lane)  MMA issuer: S = Q K^T (tcgen05 kind::f16, M = N = 128,
+//                      two tensor-memory score buffers, so the next tile's
+//                      scores are computed while this one's softmax runs)
+//                      and O += P V (V read as an MN-major operand)
+//   warps 2..5         softmax: one query row per thread; running maximum and
+//                      sum in registers, O rescaled in tensor memory when the
+//                      maximum grows, P written to shared memory in the
+//                      operand layout (K-major, 128-byte swizzle); at the end
+//                      O / l to global memory and the log-sum-exp
+// Tensor memory: S0 columns [0, 128), S1 [128, 256), O [256, 384).
+#pragma once
+
+#include "sp_gemm.cuh"
+
+namespace spk {
+
+constexpr int kAttnBM = 128;        // queries per CTA
+constexpr int kAttnBN = 128;        // keys per tile
+constexpr int kAttnD = 128;         // head dimension
+constexpr int kAttnThreads = 192;
+constexpr uint32_t kAttnTile = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column chunks)
+
+struct AttnArgs {
+    long long s;              // sequence length
+    int t;                    // ranks of the ring
+    int tiles_per_block;      // (s / t) / 128
+    float scale_log2;         // score scale * log2(e)
+    void* out;                // [bh][s][128] bf16
+    float* lse;               // [bh][s] natural-log sum of exp(scores), or NULL
+};
+
+struct AttnMaps {
+    CUtensorMap q, k, v;      // [bh * s][128] bf16, boxes of 64 x 128
+};
+
+struct AttnTail {
+    uint64_t q_full;
+    uint64_t k_full[2], k_empty[2];
+    uint64_t v_full[2], v_empty[2];
+    uint64_t s_full[2], s_free[2];
+    uint64_t p_full, o_done, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Shared-memory descriptor of an MN-major tile with 128-byte swizzle: 64
+// MN-elements per 128-byte row, 8 K-rows per 1024-byte group (stride byte
+// offset, between K groups) and mn_stride bytes between 64-element MN atoms
+// (leading byte offset).
+__device__ __forceinline__ uint64_t sw128_desc_mn(uint32_t saddr, uint32_t mn_stride)
+{
+    uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
+    d |= (uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)(1024 >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+        "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+        "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+        "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+        "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+// Generic-proxy writes to shared memory become visible to the tensor cores.
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+    k_ring_attn(const __grid_constant__ AttnArgs a, const __grid_constant__ AttnMaps maps)
+{
+    extern __shared__ __align__(1024) unsigned char asm_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(asm_raw) + 1023) & ~(uintptr_t)1023);
+    unsigned char* sq = sm;                                 // Q: 2 chunks of 16 KB
+    unsigned char* sk = sm + kAttnTile;                     // K: 2 stages
+    unsigned char* sv = sm + 3 * kAttnTile;                 // V: 2 stages
+    unsigned char* sp = sm + 5 * kAttnTile;                 // P
+    AttnTail* tail = reinterpret_cast<AttnTail*>(sm + 6 * kAttnTile);
+    volatile int* abort = &tail->abort;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long q0 = (long long)blockIdx.x * kAttnBM;   // first query row
+    const long long g = blockIdx.y;                          // batch * head index
+    const long long per = a.s / a.t;
+    const int rank = (int)(q0 / per);                        // the queries' rank
+    const int T = a.tiles_per_block;
+    const int n_tiles = a.t * T;
+    // first key row of tile j: block (rank - j / T) mod t, its (j % T)-th tile
+    auto kv_row = [&](int j) -> long long {
+        const int blk = ((rank - j / T) % a.t + a.t) % a.t;
+        return (long long)blk * per + (long long)(j % T) * kAttnBN;
+    };
+
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&tail->q_full), 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_addr(&tail->k_full[i]), 1);
+            mbar_init(smem_addr(&tail->k_empty[i]), 1);
+            mbar_init(smem_addr(&tail->v_full[i]), 1);
+            mbar_init(smem_addr(&tail->v_empty[i]), 1);
+            mbar_init(smem_addr(&tail->s_full[i]), 1);
+            mbar_init(smem_addr(&tail->s_free[i]), 4);
+        }
+        mbar_init(smem_addr(&tail->p_full), 4);
+        mbar_init(smem_addr(&tail->o_done), 1);
+        mbar_init(smem_addr(&tail->drain), 1);
+        tail->abort = 0;
+        mbar_init_fence();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_addr(&tail->tmem_base), 512);
+        tmem_fence_before_sync();
+    }
+    if (threadIdx.x == 0) {
+        tma_prefetch_desc(&maps.q);
+        tma_prefetch_desc(&maps.k);
+        tma_prefetch_desc(&maps.v);
+    }
+    __syncthreads();
+    tmem_fence_after_sync();
+    const uint32_t tbase = tail->tmem_base;
+    grid_dep_launch();
+    grid_dep_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_last();
+            const int qrow = (int)(g * a.s + q0);
+            const uint32_t qb = smem_addr(&tail->q_full);
+            mbar_arrive_expect_tx(qb, kAttnTile);
+            tma_load_2d(smem_addr(sq), &maps.q, 0, qrow, qb, pol);
+            tma_load_2d(smem_addr(sq) + kAttnTile / 2, &maps.q, 64, qrow, qb, pol);
+            int issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int st = j & 1;
+                const int krow = (int)(g * a.s + kv_row(j));
+                if (j >= 2 && !mbar_wait(smem_addr(&tail->k_empty[st]),
+                                         (uint32_t)(((j >> 1) - 1) & 1), abort, ERR_WAIT_EMPTY))
+                    break;
+                const uint32_t kb = smem_addr(&tail->k_full[st]);
+                const uint32_t kd = smem_addr(sk + (size_t)st * kAttnTile);
+                mbar_arrive_expect_tx(kb, kAttnTile);
+                tma_load_2d(kd, &maps.k, 0, krow, kb, pol);
+                tma_load_2d(kd + kAttnTile / 2, &maps.k, 64, krow, kb, pol);
+                if (j >= 2 && !mbar_wait(smem_addr(&tail->v_empty[st]),
+                                         (uint32_t)(((j >> 1) - 1) & 1), abort, ERR_WAIT_EMPTY)) {
+                    ++issued;   // the K copies of this tile are in flight
+                    break;
+                }
+                const uint32_t vb = smem_addr(&tail->v_full[st]);
+                const uint32_t vd = smem_addr(sv + (size_t)st * kAttnTile);
+                mbar_arrive_expect_tx(vb, kAttnTile);
+                tma_load_2d(vd, &maps.v, 0, krow, vb, pol);
+                tma_load_2d(vd + kAttnTile / 2, &maps.v, 64, krow, vb, pol);
+                ++issued;
+            }
+            if (*abort) {
+                // every issued copy lands before the CTA's memory goes away
+                volatile int no_abort = 0;
+                mbar_wait(smem_addr(&tail->q_full), 0u, &no_abort, ERR_DRAIN);
+                const int first = issued > 2 ? issued - 2 : 0;
+                for (int i = first; i < issued; ++i) {
+                    mbar_wait(smem_addr(&tail->k_full[i & 1]), (uint32_t)((i >> 1) & 1),
+                              &no_abort, ERR_DRAIN);
+                    mbar_wait(smem_addr(&tail->v_full[i & 1]), (uint32_t)((i >> 1) & 1),
+                              &no_abort, ERR_DRAIN);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16(kAttnBM, kAttnBN);
+            constexpr uint32_t idesc_o = idesc_bf16(kAttnBM, kAttnD) | (1u << 16);  // B MN-major
+            const uint32_t q_s = smem_addr(sq), p_s = smem_addr(sp);
+            bool ok = mbar_wait(smem_addr(&tail->q_full), 0u, abort, ERR_WAIT_FULL);
+            // S_j = Q K_j^T into score buffer j & 1
+            auto issue_s = [&](int j) -> bool {
+                const int b = j & 1;
+                if (j >= 2 && !mbar_wait(smem_addr(&tail->s_free[b]),
+                                         (uint32_t)(((j >> 1) - 1) & 1), abort, ERR_WAIT_FULL))
+                    return false;
+                if (!mbar_wait(smem_addr(&tail->k_full[j & 1]), (uint32_t)((j >> 1) & 1), abort,
+                               ERR_WAIT_FULL))
+                    return false;
+                tmem_fence_after_sync();
+                const uint32_t k_s = smem_addr(sk + (size_t)(j & 1) * kAttnTile);
+#pragma unroll
+                for (int kk = 0; kk < kAttnD / 16; ++kk) {
+                    // 16 of the 128 head features: chunk kk / 4, 32 bytes each
+                    const uint32_t off = (uint32_t)(kk >> 2) * (kAttnTile / 2) + (uint32_t)(kk & 3) * 32;
+                    umma_bf16(tbase + (uint32_t)(b * kAttnBN), sw128_desc(q_s + off),
+                              sw128_desc(k_s + off), idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(smem_addr(&tail->k_empty[j & 1]));
+                umma_commit(smem_addr(&tail->s_full[b]));
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                if (j + 1 < n_tiles && !issue_s(j + 1)) {
+                    ok = false;
+                    break;
+                }
+                if (!mbar_wait(smem_addr(&tail->p_full), (uint32_t)(j & 1), abort,
+                               ERR_WAIT_FULL) ||
+                    !mbar_wait(smem_addr(&tail->v_full[j & 1]), (uint32_t)((j >> 1) & 1), abort,
+                               ERR_WAIT_FULL)) {
+                    ok = false;
+                    break;
+                }
+                tmem_fence_after_sync();
+                const uint32_t v_s = smem_addr(sv + (size_t)(j & 1) * kAttnTile);
+#pragma unroll
+                for (int kk = 0; kk < kAttnBN / 16; ++kk) {
+                    // keys 16 kk .. 16 kk + 15: P chunk kk / 4 (K-major), V rows
+                    // 16 kk .. (two 8-row groups of 1024 bytes, MN-major)
+                    const uint32_t poff = (uint32_t)(kk >> 2) * (kAttnTile / 2) + (uint32_t)(kk & 3) * 32;
+                    umma_bf16(tbase + 256, sw128_desc(p_s + poff),
+                              sw128_desc_mn(v_s + (uint32_t)kk * 2048, kAttnTile / 2), idesc_o,
+                              (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(smem_addr(&tail->v_empty[j & 1]));
+                umma_commit(smem_addr(&tail->o_done));
+            }
+            // every issued MMA has finished before the CTA tears down
+            umma_commit(smem_addr(&tail->drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_addr(&tail->drain), 0u, &no_abort, ERR_DRAIN);
+        }
+    } else {
+        // softmax warps 2..5: thread = query row 32 (warp % 4) + lane
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        const uint32_t tlane = (uint32_t)(32 * q) << 16;
+        float m = -INFINITY, l = 0.f;   // running maximum (log2 units) and sum
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int b = j & 1;
+            if (!mbar_wait(smem_addr(&tail->s_full[b]), (uint32_t)((j >> 1) & 1), abort,
+                           ERR_WAIT_FULL)) {
+                ok = false;
+                break;
+            }
+            tmem_fence_after_sync();
+            uint32_t sc[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * c), sc + 32 * c);
+            // the score buffer may be overwritten by tile j + 2
+            tmem_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->s_free[b]));
+            float mx = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sc[i]));
+            const float m_new = fmaxf(m, mx * a.scale_log2);
+            const float alpha = exp2f(m - m_new);   // 0 at the first tile
+            float lsum = 0.f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                const float p0 = exp2f(fmaf(__uint_as_float(sc[2 * i]), a.scale_log2, -m_new));
+                const float p1 = exp2f(fmaf(__uint_as_float(sc[2 * i + 1]), a.scale_log2, -m_new));
+                lsum += p0 + p1;
+                pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
+            }
+            l = l * alpha + lsum;
+            m = m_new;
+            if (j > 0) {
+                // O of the previous tiles is complete and P may be reused
+                if (!mbar_wait(smem_addr(&tail->o_done), (uint32_t)((j - 1) & 1), abort,
+                               ERR_WAIT_FULL)) {
+                    ok = false;
+                    break;
+                }
+                tmem_fence_after_sync();
+                if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tbase + tlane + 256 + 32 * c, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tbase + tlane + 256 + 32 * c, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row into the operand layout: chunk c holds keys 64c .. 64c+63,
+            // 16-byte unit u of row r at (u ^ (r % 8)) within its 128-byte row
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint32_t off = (uint32_t)c * (kAttnTile / 2) + (uint32_t)(row >> 3) * 1024 +
+                                         (uint32_t)(row & 7) * 128 + (uint32_t)((u ^ (row & 7)) << 4);
+                    const uint4 val = make_uint4(pk[32 * c + 4 * u], pk[32 * c + 4 * u + 1],
+                                                 pk[32 * c + 4 * u + 2], pk[32 * c + 4 * u + 3]);
+                    *reinterpret_cast<uint4*>(sp + off) = val;
+                }
+            fence_async_smem();
+            tmem_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->p_full));
+        }
+        if (ok && mbar_wait(smem_addr(&tail->o_done), (uint32_t)((n_tiles - 1) & 1), abort,
+                            ERR_WAIT_FULL)) {
+            tmem_fence_after_sync();
+            const float inv = 1.0f / l;
+            unsigned char* orow = static_cast<unsigned char*>(a.out) +
+                                  ((size_t)g * a.s + q0 + row) * (kAttnD * 2);
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tbase + tlane + 256 + 32 * c, o);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    F2 f[4];
+#pragma unroll
+                    for (int p = 0; p < 4; ++p)
+                        f[p] = f2(__uint_as_float(o[8 * u + 2 * p]) * inv,
+                                  __uint_as_float(o[8 * u + 2 * p + 1]) * inv);
+                    store_vec<__nv_bfloat16>(orow, 4 * c + u, IO<__nv_bfloat16>::pack2v(f));
+                }
+            }
+            if (a.lse) a.lse[(size_t)g * a.s + q0 + row] = (m + log2f(l)) * 0.69314718055994531f;
+        } else {
+            // warp-wide tensor-memory reads must still be matched: nothing
+            // more to read on the abort path
+        }
+    }
+    tmem_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_fence_after_sync();
+        tmem_dealloc(tbase, 512);
+    }
+}
+
+}  // namespace spk

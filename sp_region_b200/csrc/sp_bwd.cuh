@@ -39,7 +39,8 @@ struct BwdArgs {
     const float* mean;
     const float* rstd;
     void* dres;
-    void* dY;
+    void* dY[kMaxT];         // n_dY full [s,b,h] buffers, indexed by global row
+    int n_dY;                // 0: no dY; t: every rank's copy (the all-gather)
     float* ws;               // [gridDim.x][3][h] per-CTA partial sums
     long long rows;          // token rows of this call (local index i)
     long long row0;          // global index of local row 0: n = row0 + i
@@ -335,8 +336,7 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
         take_turn(1, j);
         unsigned char* dres =
             static_cast<unsigned char*>(a.dres) + (size_t)i_row * a.res_seg_bytes;   // shard
-        unsigned char* dy =
-            static_cast<unsigned char*>(a.dY) + (size_t)n * a.seg_bytes;       // gathered
+        const size_t dy_off = (size_t)n * a.seg_bytes;   // gathered: global row
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             const int v = c + i * C;
@@ -367,7 +367,12 @@ __global__ void __launch_bounds__(MAXT, 1) k_bwd_tma(const __grid_constant__ Bwd
                     store_vec<float>(dres, v, IO<float>::pack2v(dr));
                 else
                     store_vec<T>(dres, v, IO<T>::pack2v(dr));
-                if (a.dY) store_vec<T>(dy, v, IO<T>::pack2v(dz));
+                if (a.n_dY) {
+                    // the all-gather of dY: this row into every rank's copy
+                    const Vec dzv = IO<T>::pack2v(dz);
+                    for (int q = 0; q < a.n_dY; ++q)
+                        store_vec<T>(static_cast<unsigned char*>(a.dY[q]) + dy_off, v, dzv);
+                }
                 if (a.want_dbias) {
                     if (ACC_SMEM) {
                         acc_add(2, v, dz);
@@ -553,7 +558,7 @@ __global__ void __launch_bounds__(1024) k_bwd_general(const __grid_constant__ Bw
             uint32_t keep = 1u;
             if (a.mask) keep = (a.mask[(size_t)i_row * a.mask_row_bytes + (j >> 3)] >> (j & 7)) & 1u;
             const float dz = keep ? dr * a.scale : 0.f;
-            if (a.dY) IO<T>::store1(a.dY, base + j, dz);
+            for (int q = 0; q < a.n_dY; ++q) IO<T>::store1(a.dY[q], base + j, dz);
             if (a.want_dbias) ws[2 * h + j] += dz;
         }
         __syncthreads();   // dns is rewritten by the next row

@@ -1,13 +1,15 @@
-// C-ABI entry points of the tensor-parallel linears with the SP collectives
-// fused into them (declared in sp_region.h): the row-parallel linear whose
-// reduce-scatter is the GEMM's own accumulation, with the SP region's bias,
-// dropout and residual add in its epilogue, and the column-parallel linear
-// whose all-gather is its A-operand prologue.  Argument validation, tensor
-// maps and launch; the arithmetic is in sp_gemm.cuh.
+// C-ABI entry points of the tensor-core kernels (declared in sp_region.h):
+// the row-parallel linear whose reduce-scatter is the GEMM's own
+// accumulation, with the SP region's bias, dropout and residual add in its
+// epilogue; the column-parallel linear whose all-gather is its A-operand
+// prologue; and ring attention over the context-parallel ranks.  Argument
+// validation, tensor maps and launch; the arithmetic is in sp_gemm.cuh and
+// sp_attn.cuh.
 #include <cuda.h>
 #include <math.h>
 #include <string.h>
 
+#include "sp_attn.cuh"
 #include "sp_gemm.cuh"
 #include "sp_host.h"
 #include "sp_plans.h"
@@ -208,6 +210,65 @@ int sp_ag_colpar_linear_fwd(const sp_cfg* cfg, int64_t f_out, const void* const*
     a.nmaps = t;
     a.out = out;
     return launch_gemm_bn<1>(a, maps, dev, static_cast<cudaStream_t>(stream), bn);
+}
+
+int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const void* q,
+                          const void* k, const void* v, void* out, float* lse, void* stream)
+{
+    int rc = check_gemm_cfg(cfg);
+    if (rc) return rc;
+    if (!q || !k || !v || !out || heads < 1 || !(scale > 0.0f) || !isfinite(scale))
+        return SP_ERR_INVALID_ARG;
+    if (!(cfg->row_begin == 0 && cfg->row_end == 0)) return SP_ERR_INVALID_ARG;
+    if (cfg->h != (int64_t)heads * kAttnD) return SP_ERR_UNSUPPORTED;   // head dim 128
+    const long long S = cfg->s, per = S / cfg->t;
+    if (S % kAttnBM || per % kAttnBN) return SP_ERR_UNSUPPORTED;
+    const long long bh = cfg->b * (long long)heads;
+    if (bh * S >= (1LL << 31) || bh > 65535) return SP_ERR_UNSUPPORTED;
+    for (const void* p : {q, k, v, (const void*)out})
+        if (!aligned(p, 16)) return SP_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return SP_ERR_INVALID_ARG;
+    DevInfo dev;
+    if ((rc = use_device_of(out, &dev))) return rc;
+
+    AttnMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!make_map(&maps.q, q, bh * S, kAttnD, kAttnD, kAttnBM) ||
+        !make_map(&maps.k, k, bh * S, kAttnD, kAttnD, kAttnBN) ||
+        !make_map(&maps.v, v, bh * S, kAttnD, kAttnD, kAttnBN))
+        return SP_ERR_INVALID_ARG;
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.s = S;
+    a.t = cfg->t;
+    a.tiles_per_block = (int)(per / kAttnBN);
+    a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    a.out = out;
+    a.lse = lse;
+    const size_t smem = 1024 + 6 * (size_t)kAttnTile + ((sizeof(AttnTail) + 127) & ~(size_t)127);
+    if (smem > (size_t)dev.smem_optin) return SP_ERR_UNSUPPORTED;
+    const void* kern = (const void*)k_ring_attn;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)(S / kAttnBM), (unsigned)bh);
+    lc.blockDim = dim3(kAttnThreads);
+    lc.dynamicSmemBytes = smem;
+    lc.stream = static_cast<cudaStream_t>(stream);
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    void* params[] = {&a, &maps};
+    if (cudaLaunchKernelExC(&lc, kern, params) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
 }
 
 }  // extern "C"

@@ -40,7 +40,8 @@ namespace spk {
 constexpr int kGemmBM = 128;           // rows per tile (tcgen05 M)
 constexpr int kGemmBK = 64;            // K elements per stage: one 128-byte row
 constexpr int kGemmThreads = 192;      // producer, MMA, 4 epilogue warps
-constexpr int kGemmMaxShards = 16;      // A tensor maps (sequence shards)
+constexpr int kGemmMaxShards = 16;     // A tensor maps (sequence shards)
+constexpr int kGemmGroup = 16;         // row tiles per group of the tile order
 
 struct GemmArgs {
     // epilogue kind 0: row-parallel SP (bias, dropout, residual, mask)
@@ -196,8 +197,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     GemmTail* tail = reinterpret_cast<GemmTail*>(gsm + (size_t)S * kStage);
     volatile int* abort = &tail->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = blockIdx.x * BN;
-    const long long m0 = (long long)blockIdx.y * kGemmBM;
+    // tile order: the CTAs that run at the same time cover a block of
+    // kGemmGroup row tiles by a few column tiles, so the A and B slabs they
+    // stream (in near lock-step along K) are each read from HBM once and
+    // shared through L2
+    const int ncol = gridDim.x, nrow = gridDim.y;
+    const long long lin = (long long)blockIdx.y * ncol + blockIdx.x;
+    const long long per_group = (long long)kGemmGroup * ncol;
+    const int grp = (int)(lin / per_group);
+    const int in_grp = (int)(lin - (long long)grp * per_group);
+    const int rows_in_grp = min(kGemmGroup, nrow - grp * kGemmGroup);
+    const int tile_row = grp * kGemmGroup + in_grp % rows_in_grp;
+    const int tile_col = in_grp / rows_in_grp;
+    const int n0 = tile_col * BN;
+    const long long m0 = (long long)tile_row * kGemmBM;
     const int KB = (a.K + kGemmBK - 1) / kGemmBK;
     // A rows of this tile come from one shard (rows_per_shard % 128 == 0)
     const int map_id = (int)(m0 / a.rows_per_shard);

@@ -611,8 +611,9 @@ int noalloc_scratch(int dev, size_t need, void** out);
 // fixed device array (sp_rs_norm_dropout_bwd_noalloc).
 int bwd_impl(const sp_cfg* cfg, const void* const* dn_partials, const void* dR_next,
              const void* residual_out, const void* gamma, const uint32_t* mask_bits,
-             const float* mean, const float* rstd, void* dresidual_in, void* dY, float* dgamma,
-             float* dbeta, float* dbias, void* workspace, size_t workspace_bytes, void* stream)
+             const float* mean, const float* rstd, void* dresidual_in, void* const* dY,
+             int n_dY, float* dgamma, float* dbeta, float* dbias, void* workspace,
+             size_t workspace_bytes, void* stream)
 {
     int rc = check_cfg(cfg);
     if (rc) return rc;
@@ -628,11 +629,13 @@ int bwd_impl(const sp_cfg* cfg, const void* const* dn_partials, const void* dR_n
         all16 = all16 && aligned(dn_partials[k], 16);
     }
     const int Er = res_elem_bytes(cfg);
-    const void* elem_ptrs[] = {gamma, dY};
-    for (const void* p : elem_ptrs) {
-        if (p && !aligned(p, E)) return SP_ERR_INVALID_ARG;
-        all16 = all16 && (!p || aligned(p, 16));
+    if (n_dY < 0 || n_dY > SP_MAX_T || (n_dY > 0 && !dY)) return SP_ERR_INVALID_ARG;
+    for (int q = 0; q < n_dY; ++q) {
+        if (!dY[q] || !aligned(dY[q], E)) return SP_ERR_INVALID_ARG;
+        all16 = all16 && aligned(dY[q], 16);
     }
+    if (!aligned(gamma, E)) return SP_ERR_INVALID_ARG;
+    all16 = all16 && aligned(gamma, 16);
     for (const void* p : {dR_next, residual_out, (const void*)dresidual_in}) {   // residual stream
         if (p && !aligned(p, Er)) return SP_ERR_INVALID_ARG;
         all16 = all16 && (!p || aligned(p, 16));
@@ -664,7 +667,8 @@ int bwd_impl(const sp_cfg* cfg, const void* const* dn_partials, const void* dR_n
     a.mean = ln ? mean : nullptr;
     a.rstd = rstd;
     a.dres = dresidual_in;
-    a.dY = dY;
+    for (int q = 0; q < n_dY; ++q) a.dY[q] = dY[q];
+    a.n_dY = n_dY;
     a.ws = static_cast<float*>(workspace);
     a.want_dbeta = (ln && dbeta) ? 1 : 0;
     a.want_dbias = dbias ? 1 : 0;
@@ -817,7 +821,21 @@ int sp_rs_norm_dropout_bwd(const sp_cfg* cfg, const void* const* dn_partials,
 {
     if (!workspace) return SP_ERR_INVALID_ARG;
     return bwd_impl(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits, mean, rstd,
-                    dresidual_in, dY, dgamma, dbeta, dbias, workspace, workspace_bytes, stream);
+                    dresidual_in, &dY, dY ? 1 : 0, dgamma, dbeta, dbias, workspace,
+                    workspace_bytes, stream);
+}
+
+int sp_rs_norm_dropout_bwd_ag(const sp_cfg* cfg, const void* const* dn_partials,
+                              const void* dR_next, const void* residual_out, const void* gamma,
+                              const uint32_t* mask_bits, const float* mean, const float* rstd,
+                              void* dresidual_in, void* const* dY, int32_t n_dY, float* dgamma,
+                              float* dbeta, float* dbias, void* workspace,
+                              size_t workspace_bytes, void* stream)
+{
+    if (!workspace || n_dY < 1) return SP_ERR_INVALID_ARG;
+    return bwd_impl(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits, mean, rstd,
+                    dresidual_in, dY, n_dY, dgamma, dbeta, dbias, workspace, workspace_bytes,
+                    stream);
 }
 
 int sp_device_error(int32_t device, int32_t* code, int32_t clear)
@@ -913,5 +931,5 @@ extern "C" int sp_rs_norm_dropout_bwd_noalloc(
     // the backward picks its kernel for the actual pointers, then checks that
     // the slices that kernel writes fit the array
     return bwd_impl(cfg, dn_partials, dR_next, residual_out, gamma, mask_bits, mean, rstd,
-                    dresidual_in, dY, dgamma, dbeta, dbias, nullptr, 0, stream);
+                    dresidual_in, &dY, dY ? 1 : 0, dgamma, dbeta, dbias, nullptr, 0, stream);
 }

@@ -6,11 +6,11 @@ partial-sum buffer (the peers' through peer-mapped memory; that read is the
 reduce-scatter) and pushes its normalised rows into every rank's gathered
 buffer (the all-gather) -- "Sequence Parallelism math", section "The
 collective substitution".  The backward is the same with the upstream
-gradients, except that the library writes dY (the all-gather of the dropout
-gradient, the reduce-scatter's backward) into one buffer: each rank writes
-its own rows of its full-size dY and an in-place all-gather of the row blocks
-completes every rank's copy.  Last, the replicated parameters' gradients
-(gamma, beta and the bias live on every rank) are summed over the ranks.
+gradients: it reads its rows of every rank's gradient partials and pushes
+its rows of dY (the all-gather of the dropout gradient, the reduce-scatter's
+backward) into every rank's dY buffer.  Last, the replicated parameters'
+gradients (gamma, beta and the bias live on every rank) are summed over the
+ranks.
 
 The kernels never wait on another rank.  Ordering between ranks is kept on
 the host: every rank's inputs are written before any rank's kernel reads
@@ -105,10 +105,10 @@ class LibraryOps:
 
     def backward(self, cfg, dparts, drnext, residual_out, gamma, mask, mean, rstd,
                  dres, dY, dgamma, dbeta, dbias, workspace, stream):
-        from sp_region_b200 import sp_rs_norm_dropout_bwd
-        sp_rs_norm_dropout_bwd(cfg, dparts, drnext, residual_out, gamma, mask, mean,
-                               rstd, dres, dY, dgamma, dbeta, dbias, workspace,
-                               stream=stream)
+        from sp_region_b200 import sp_rs_norm_dropout_bwd_ag
+        sp_rs_norm_dropout_bwd_ag(cfg, dparts, drnext, residual_out, gamma, mask, mean,
+                                  rstd, dres, dY, dgamma, dbeta, dbias, workspace,
+                                  stream=stream)
 
     def synchronize(self, stream):
         (stream or torch.cuda.current_stream()).synchronize()
@@ -185,22 +185,21 @@ class SPBoundary:
 
     def backward(self, cfg, dparts, drnext, residual_out, gamma, mask, mean, rstd,
                  dres, dY, dgamma, dbeta, dbias, workspace, stream=None):
-        """dparts: the world's gradient partials in rank order (peer_buffers).
-        dY: this rank's full [N, h] buffer, complete on return.  The rest are
-        this rank's shard.  dgamma / dbeta / dbias come back summed over the
-        ranks."""
-        if len(dparts) != self.world:
-            raise ValueError("one gradient partial buffer per rank")
+        """dparts, dY: the world's gradient partials and dY buffers in rank
+        order (peer_buffers); every rank's dY is complete on return.  The rest
+        are this rank's shard.  dgamma / dbeta / dbias come back summed over
+        the ranks."""
+        if len(dparts) != self.world or len(dY) != self.world:
+            raise ValueError("one gradient partial and one dY buffer per rank")
         c = self._cfg(cfg)
-        r0, r1 = c.row_begin, c.row_end
         self._inputs_written("backward inputs written", stream)
-        self._run("backward outputs written",
+        # each rank pushes its dY rows into every rank's dY; once all have
+        # arrived, every copy is complete
+        self._run("backward outputs pushed",
                   lambda: self.ops.backward(c, dparts, drnext, residual_out, gamma,
                                             mask, mean, rstd, dres, dY, dgamma, dbeta,
                                             dbias, workspace, stream),
                   stream)
-        # every rank's dY rows, in rank order, into every rank's dY
-        dist.all_gather_into_tensor(dY, dY[r0:r1], group=self.group)
         # gamma, beta and bias are replicated: sum their gradients over ranks
         for g in (dgamma, dbeta, dbias):
             if g is not None:

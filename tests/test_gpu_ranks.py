@@ -5,7 +5,8 @@ its rows of every rank's partial sum (on a multi-GPU system, peers' buffers
 through peer pointers), keeps its residual / stored outputs / mask /
 statistics as a shard indexed from 0, and writes its normalised rows into
 every rank's gathered buffer (the all-gather, pushed).  The backward does the
-same with the upstream partials and dY.  Run rank by rank on one GPU, the t
+same with the upstream partials, pushing its dY rows into every rank's dY
+buffer.  Run rank by rank on one GPU, the t
 calls must reproduce the single whole-tensor call bit for bit (the dropout
 counter uses the global row), and the per-rank parameter gradients must sum
 to the whole call's ("Sequence Parallelism math", section "The collective
@@ -113,7 +114,9 @@ def test_ranks_reproduce_the_whole_call(name, over):
     sp.sp_rs_norm_dropout_bwd(_cfg(w), dparts, None, whole["rout"], gamma,
                               whole["mask"], whole["mean"], whole["rstd"],
                               dres, dY, *g0, ws)
-    dY_r = torch.full((N, h), float("nan"), dtype=dt, device="cuda")
+    # every rank's dY copy, each filled by the t range calls' pushes
+    dY_r = [torch.full((N, h), float("nan"), dtype=dt, device="cuda")
+            for _ in range(t)]
     dres_r = []
     gsum = [np.zeros(h), np.zeros(h), np.zeros(h)]
     for r in range(t):
@@ -121,9 +124,9 @@ def test_ranks_reproduce_the_whole_call(name, over):
         o = shards[r]
         dr = torch.empty((per, h), dtype=dt, device="cuda")
         gr = grads()
-        sp.sp_rs_norm_dropout_bwd(_cfg(w, r * per, (r + 1) * per), dparts,
-                                  None, o["rout"], gamma, o["mask"],
-                                  o["mean"], o["rstd"], dr, dY_r, *gr, ws)
+        sp.sp_rs_norm_dropout_bwd_ag(_cfg(w, r * per, (r + 1) * per), dparts,
+                                     None, o["rout"], gamma, o["mask"],
+                                     o["mean"], o["rstd"], dr, dY_r, *gr, ws)
         torch.cuda.synchronize()
         dres_r.append(dr)
         for q in range(3):
@@ -131,7 +134,8 @@ def test_ranks_reproduce_the_whole_call(name, over):
                 gsum[q] += gr[q].cpu().double().numpy()
     assert sp.sp_device_error() == 0
     assert torch.equal(bits(torch.cat(dres_r)), bits(dres))
-    assert torch.equal(bits(dY_r), bits(dY))
+    for q in range(t):
+        assert torch.equal(bits(dY_r[q]), bits(dY)), q
     # replicated parameters: the per-rank partial gradients sum to the whole
     dn_abs = sum(d.double().abs() for d in dparts).sum(0).cpu().numpy()
     for q in range(3):

@@ -1,7 +1,7 @@
 """sp_region_b200.ranks with the real library calls, on a one-rank NCCL group
 (the one GPU here): SPBoundary's forward and backward, with their row range,
-rendezvous, dY all-gather and gradient all-reduce, must give the bits of the
-direct library calls.  Peer-mapped buffers (several GPUs) are not exercised."""
+rendezvous, dY pushed by the kernel and gradient all-reduce, must give the
+bits of the direct library calls.  Peer-mapped buffers (several GPUs) are not exercised."""
 import socket
 
 import pytest
@@ -81,7 +81,7 @@ def test_one_rank_boundary_gives_the_direct_calls_bits(one_rank_group):
                               a["db"], a["dc"], ws)
     b = bwd_bufs()
     sb.backward(cfg, dparts, None, d["rout"], gamma, d["mask"], d["mean"], d["rstd"],
-                b["dres"], b["dY"], b["dg"], b["db"], b["dc"], ws)
+                b["dres"], [b["dY"]], b["dg"], b["db"], b["dc"], ws)
     torch.cuda.synchronize()
     assert sp.sp_device_error() == 0
     for k in ("dres", "dY"):

@@ -3,7 +3,8 @@ gloo ranks on the CPU.
 
 The library calls are replaced by a stand-in that moves data the way the
 kernels do: rank r reads its rows of every rank's partial buffer and pushes
-its result rows into every rank's gathered buffer.  The buffers are shared
+its result rows into every rank's gathered buffer (forward) and every rank's
+dY buffer (backward).  The buffers are shared
 host tensors, standing in for peer-mapped GPU memory.  Rank 1 is made slow at
 each step, so a missing rendezvous would show up as a wrong value on rank 0.
 Failures are made on the host, as the failure-detection tests require: a
@@ -53,7 +54,8 @@ class _Ops:
         if self.rank == 1:
             time.sleep(0.3)
         dres.copy_(dz)
-        dY[r0:r1] = dz
+        for d in dY:                 # pushed into every rank's dY
+            d[r0:r1] = dz
         dgamma.fill_(self.rank + 1.0)
         dbeta.fill_(10.0 * (self.rank + 1))
 
@@ -100,7 +102,7 @@ def _worker(rank, port, scenario, bufs, q):
         dres = torch.empty(N // WORLD, H)
         dg, db = torch.empty(H), torch.empty(H)
         sb.backward(cfg, bufs["dparts"], None, rout, None, None, None, None, dres,
-                    dY, dg, db, None, None)
+                    bufs["dY"], dg, db, None, None)
         # the store keeps only each rank's key of the latest rendezvous
         rdv = sb.rdv
         old_keys = [rdv._key(q_, tag, rank) for q_, tag in
