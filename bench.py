@@ -18,8 +18,11 @@ The metric is achieved HBM bandwidth on the algorithmic bytes of both calls
 
 With N > 1 (launched by torch.distributed.run) every rank runs an independent
 replica on its own GPU (weak scaling; the path has no exchange between
-replicas); the time is the maximum over ranks.  ``--impl reference`` times the
-CPU oracle on the host cores instead.
+replicas); the time is the maximum over ranks.  ``--mode ranks`` instead runs
+the boundary itself on t = N ranks, the partial sums, gathered outputs and
+gradients in symmetric memory reached by the kernels over NVLink, beside
+NCCL's all-reduce and reduce-scatter + all-gather on the same bytes.
+``--impl reference`` times the CPU oracle on the host cores instead.
 """
 from __future__ import annotations
 
@@ -679,6 +682,144 @@ def time_ring_attention(args, sp, torch, dev):
             "flops_per_launch": flops}
 
 
+def collective_record(nbytes, ar_ms, rs_ag_ms, world, device=None):
+    """The NCCL arm on the same bytes: one all-reduce against a
+    reduce-scatter plus an all-gather, each timed per call on every rank and
+    taken at the slowest rank.  Per-rank wire volume of either: 2 (t-1)/t of
+    the tensor ("Sequence Parallelism math", section "Why the byte count is
+    identical")."""
+    ar = max_over_ranks(ar_ms, device)
+    rs_ag = max_over_ranks(rs_ag_ms, device)
+    wire = 2.0 * (world - 1) / world * nbytes
+    return {"bytes": nbytes, "all_reduce_ms": round(ar, 4), "rs_ag_ms": round(rs_ag, 4),
+            "rs_ag_over_all_reduce": round(rs_ag / ar, 4) if ar > 0 else None,
+            "wire_bytes_per_rank": wire,
+            "all_reduce_busbw_gbs": round(wire / (ar * 1e-3) / 1e9, 1) if ar > 0 else None}
+
+
+def run_ranks(args):
+    """The boundary on t = N real ranks, one GPU each, through peer memory:
+    rank r runs the fused forward on its token rows, pulling its rows of every
+    rank's partial sum (the reduce-scatter) and pushing its normalised rows
+    into every rank's gathered buffer (the all-gather); the backward pulls the
+    gradient partials and pushes dY the same way, then the replicated
+    parameters' gradients are all-reduced.  Beside it, NCCL's all-reduce and
+    reduce-scatter + all-gather on one partial-sum tensor."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import torch.distributed._symmetric_memory as symm_mem
+    import sp_synth
+    import sp_region_b200 as sp
+    from sp_region_b200.ranks import peer_buffers
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    w = workload_of(args).replace(t=world)
+    N, h, t = w.rows, w.h, world
+    per = N // t
+    r0, r1 = rank * per, (rank + 1) * per
+    dt = w.torch_dtype
+    cfg = sp.make_cfg(w.s, w.b, h, t, dtype=w.dtype, norm=w.norm, eps=w.eps,
+                      p_drop=w.p_drop, seed=w.drop_seed, offset=w.drop_offset,
+                      row_begin=r0, row_end=r1)
+
+    def shared(x):
+        buf = symm_mem.empty(tuple(x.shape), dtype=x.dtype, device=dev)
+        buf.copy_(x)
+        return buf
+    part = shared(sp_synth.draw_partials(w, dev)[rank])
+    dpart = shared(sp_synth.draw_grad_partials(w, dev)[rank])
+    out = shared(torch.zeros((N, h), dtype=dt, device=dev))
+    dy = shared(torch.zeros((N, h), dtype=dt, device=dev))
+    parts, gathered = peer_buffers(part), peer_buffers(out)
+    dparts, dys = peer_buffers(dpart), peer_buffers(dy)
+    bias, gamma, beta = sp_synth.draw_params(w, dev)
+    res = sp_synth.draw_residual(w, dev)[r0:r1].contiguous()
+    rout = torch.empty((per, h), dtype=dt, device=dev)
+    mask = torch.empty((per, (h + 31) // 32), dtype=torch.int32, device=dev)
+    mean = torch.empty(per, dtype=torch.float32, device=dev)
+    rstd = torch.empty(per, dtype=torch.float32, device=dev)
+    dres = torch.empty((per, h), dtype=dt, device=dev)
+    grads = [torch.empty(h, dtype=torch.float32, device=dev) for _ in range(3)]
+    ws = torch.empty(sp.sp_bwd_workspace_bytes(cfg, local) // 4, dtype=torch.float32,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        sp.sp_rs_bias_dropout_add_norm_fwd(cfg, parts, bias, res, gamma, beta, rout,
+                                           gathered, mask, mean, rstd, stream=stream)
+        sp.sp_rs_norm_dropout_bwd_ag(cfg, dparts, None, rout, gamma, mask, mean, rstd,
+                                     dres, dys, *grads, ws, stream=stream)
+        for g_ in grads:        # replicated parameters: sum over the ranks
+            dist.all_reduce(g_)
+
+    # every rank's inputs are written before any rank's kernel reads them
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    K = args.steps
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    assert sp.sp_device_error(local) == 0, "device-side wait timed out"
+    total_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    step_bytes = fwd_bytes(w) + bwd_bytes(w)
+    value = step_bytes * K / (total_ms * 1e-3) / 1e9
+
+    # NCCL on one partial-sum tensor: all-reduce vs reduce-scatter + all-gather
+    x = part.clone()
+    shard = torch.empty((per, h), dtype=dt, device=dev)
+    KC = 20
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(KC):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / KC
+    ar_ms = timed(lambda: dist.all_reduce(x))
+    rs_ag_ms = timed(lambda: (dist.reduce_scatter_tensor(shard, x),
+                              dist.all_gather_into_tensor(x, shard)))
+    coll = collective_record(N * h * w.elem_bytes, ar_ms, rs_ag_ms, world, dev)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "f32", "io_dtype": w.dtype, "data": "synthetic", "mode": "ranks",
+        "config": {"workload": (f"{w.name} shape on t={t} real ranks, one GPU each: rank r "
+                                f"owns token rows [r*{per}, (r+1)*{per}); partials, gathered "
+                                "outputs, gradient partials and dY in symmetric memory, "
+                                "reached by the kernels over peer memory"),
+                   "s": w.s, "b": w.b, "h": h, "t": t, "parallelism": f"sp{t}"},
+        "nccl": coll,
+        "gpu_launches": 3 * K,
+    }
+    for b_ in (out, dy, part, dpart):
+        del b_
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def run_e2e(args, w, cfg, sp, torch, dev, step_bytes, world):
     """Same metric through the public API with host buffers: every step
     copies its inputs from pinned host memory, runs forward and backward, and
@@ -992,6 +1133,11 @@ def main():
     ap.add_argument("--reference-cores", type=int, default=0,
                     help="processes for --impl reference (0: every core, up to 64)")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "ranks"],
+                    help="replicas: N independent copies of the boundary (weak "
+                         "scaling); ranks: the boundary on t = N ranks over peer "
+                         "memory, with NCCL all-reduce vs reduce-scatter + "
+                         "all-gather beside it")
     ap.add_argument("--skip-linears", action="store_true",
                     help="skip timing the tensor-parallel linears and the ring "
                          "attention (N = 1)")
@@ -1009,6 +1155,8 @@ def main():
         ap.error("at least 3 warm-up steps")
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "ranks":
+        run_ranks(args)
     else:
         run_ours(args)
 

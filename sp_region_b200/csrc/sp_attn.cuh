@@ -18,11 +18,16 @@
 //                      two tensor-memory score buffers, so the next tile's
 //                      scores are computed while this one's softmax runs)
 //                      and O += P V (V read as an MN-major operand)
-//   warps 2..5         softmax: one query row per thread; running maximum and
-//                      sum in registers, O rescaled in tensor memory when the
-//                      maximum grows, P written to shared memory in the
-//                      operand layout (K-major, 128-byte swizzle); at the end
-//                      O / l to global memory and the log-sum-exp
+//   warps 2..9         softmax: each query row is shared by two warps of the
+//                      same sub-partition (warps w and w + 4 read the same
+//                      tensor-memory lanes), one taking score columns 0..63,
+//                      the other 64..127.  The pair exchanges its halves'
+//                      maxima once per tile; both keep the same running
+//                      maximum, so their partial sums add up at the end.  O
+//                      is rescaled in tensor memory when the maximum grows,
+//                      P written to shared memory in the operand layout
+//                      (K-major, 128-byte swizzle); at the end O / l to
+//                      global memory and the log-sum-exp
 // Tensor memory: S0 columns [0, 128), S1 [128, 256), O [256, 384).
 #pragma once
 
@@ -33,7 +38,7 @@ namespace spk {
 constexpr int kAttnBM = 128;        // queries per CTA
 constexpr int kAttnBN = 128;        // keys per tile
 constexpr int kAttnD = 128;         // head dimension
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;   // producer, MMA, 8 softmax warps
 constexpr uint32_t kAttnTile = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column chunks)
 
 struct AttnArgs {
@@ -57,6 +62,10 @@ struct AttnTail {
     uint64_t p_full, o_done, drain;
     uint32_t tmem_base;
     int abort;
+    uint64_t pair[4][2];         // per row quarter and tile parity: both halves' maxima posted
+    uint64_t pair_fin[4];        // per row quarter: both halves' sums posted
+    float xmax[2][2][kAttnBM];   // [tile parity][half][row]: the halves' maxima
+    float xsum[2][kAttnBM];      // [half][row]: the halves' sums at the end
 };
 
 // Shared-memory descriptor of an MN-major tile with 128-byte swizzle: 64
@@ -126,11 +135,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(smem_addr(&tail->v_full[i]), 1);
             mbar_init(smem_addr(&tail->v_empty[i]), 1);
             mbar_init(smem_addr(&tail->s_full[i]), 1);
-            mbar_init(smem_addr(&tail->s_free[i]), 4);
+            mbar_init(smem_addr(&tail->s_free[i]), 8);
         }
-        mbar_init(smem_addr(&tail->p_full), 4);
+        mbar_init(smem_addr(&tail->p_full), 8);
         mbar_init(smem_addr(&tail->o_done), 1);
         mbar_init(smem_addr(&tail->drain), 1);
+        for (int qq = 0; qq < 4; ++qq) {   // every thread of the two warps arrives
+            mbar_init(smem_addr(&tail->pair[qq][0]), 64);
+            mbar_init(smem_addr(&tail->pair[qq][1]), 64);
+            mbar_init(smem_addr(&tail->pair_fin[qq]), 64);
+        }
         tail->abort = 0;
         mbar_init_fence();
     }
@@ -255,36 +269,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_wait(smem_addr(&tail->drain), 0u, &no_abort, ERR_DRAIN);
         }
     } else {
-        // softmax warps 2..5: thread = query row 32 (warp % 4) + lane
+        // softmax warps 2..9: query row 32 (warp % 4) + lane; half hf of the
+        // score columns (and of O's columns); the pair (w, w + 4) shares rows
         const int q = warp & 3;
+        const int hf = (warp - 2) >> 2;
         const int row = 32 * q + lane;
         const uint32_t tlane = (uint32_t)(32 * q) << 16;
-        float m = -INFINITY, l = 0.f;   // running maximum (log2 units) and sum
+        // a bounded wait whose outcome is the same in every lane of the warp,
+        // so the warp-collective tensor-memory accesses after it are uniform
+        auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+            const bool w = mbar_wait(bar, parity, abort, ERR_WAIT_FULL);
+            return __all_sync(0xFFFFFFFFu, w) != 0;
+        };
+        float m = -INFINITY, l = 0.f;   // running maximum (log2 units), this half's sum
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int b = j & 1;
-            if (!mbar_wait(smem_addr(&tail->s_full[b]), (uint32_t)((j >> 1) & 1), abort,
-                           ERR_WAIT_FULL)) {
+            if (!wait_all(smem_addr(&tail->s_full[b]), (uint32_t)((j >> 1) & 1))) {
                 ok = false;
                 break;
             }
             tmem_fence_after_sync();
-            uint32_t sc[128];
+            uint32_t sc[64];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * c), sc + 32 * c);
+            for (int c = 0; c < 2; ++c)
+                tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + 64 * hf + 32 * c), sc + 32 * c);
             // the score buffer may be overwritten by tile j + 2
             tmem_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&tail->s_free[b]));
             float mx = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sc[i]));
+            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sc[i]));
+            tail->xmax[b][hf][row] = mx;
+            mbar_arrive(smem_addr(&tail->pair[q][b]));
+            if (!wait_all(smem_addr(&tail->pair[q][b]), (uint32_t)((j >> 1) & 1))) {
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, tail->xmax[b][hf ^ 1][row]);   // the row's maximum
             const float m_new = fmaxf(m, mx * a.scale_log2);
             const float alpha = exp2f(m - m_new);   // 0 at the first tile
             float lsum = 0.f;
-            uint32_t pk[64];
+            uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
+            for (int i = 0; i < 32; ++i) {
                 const float p0 = exp2f(fmaf(__uint_as_float(sc[2 * i]), a.scale_log2, -m_new));
                 const float p1 = exp2f(fmaf(__uint_as_float(sc[2 * i + 1]), a.scale_log2, -m_new));
                 lsum += p0 + p1;
@@ -294,51 +323,53 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             m = m_new;
             if (j > 0) {
                 // O of the previous tiles is complete and P may be reused
-                if (!mbar_wait(smem_addr(&tail->o_done), (uint32_t)((j - 1) & 1), abort,
-                               ERR_WAIT_FULL)) {
+                if (!wait_all(smem_addr(&tail->o_done), (uint32_t)((j - 1) & 1))) {
                     ok = false;
                     break;
                 }
                 tmem_fence_after_sync();
                 if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(tbase + tlane + 256 + 32 * c, o);
+                        const uint32_t oc = tbase + tlane + 256 + (uint32_t)(64 * hf + 32 * c);
+                        tmem_ld32(oc, o);
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tbase + tlane + 256 + 32 * c, o);
+                        tmem_st32(oc, o);
                     }
                     tmem_wait_st();
                 }
             }
-            // P row into the operand layout: chunk c holds keys 64c .. 64c+63,
+            // this half of the P row into chunk hf of the operand layout:
             // 16-byte unit u of row r at (u ^ (r % 8)) within its 128-byte row
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const uint32_t off = (uint32_t)c * (kAttnTile / 2) + (uint32_t)(row >> 3) * 1024 +
-                                         (uint32_t)(row & 7) * 128 + (uint32_t)((u ^ (row & 7)) << 4);
-                    const uint4 val = make_uint4(pk[32 * c + 4 * u], pk[32 * c + 4 * u + 1],
-                                                 pk[32 * c + 4 * u + 2], pk[32 * c + 4 * u + 3]);
-                    *reinterpret_cast<uint4*>(sp + off) = val;
-                }
+            for (int u = 0; u < 8; ++u) {
+                const uint32_t off = (uint32_t)hf * (kAttnTile / 2) + (uint32_t)(row >> 3) * 1024 +
+                                     (uint32_t)(row & 7) * 128 + (uint32_t)((u ^ (row & 7)) << 4);
+                *reinterpret_cast<uint4*>(sp + off) =
+                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            }
             fence_async_smem();
             tmem_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&tail->p_full));
         }
-        if (ok && mbar_wait(smem_addr(&tail->o_done), (uint32_t)((n_tiles - 1) & 1), abort,
-                            ERR_WAIT_FULL)) {
+        // the row's sum: both halves post theirs (a half that left the loop
+        // early makes the other's bounded wait run out, never hang)
+        tail->xsum[hf][row] = l;
+        mbar_arrive(smem_addr(&tail->pair_fin[q]));
+        if (ok && !wait_all(smem_addr(&tail->pair_fin[q]), 0u)) ok = false;
+        const float lt = tail->xsum[0][row] + tail->xsum[1][row];   // same bits in both warps
+        if (ok && wait_all(smem_addr(&tail->o_done), (uint32_t)((n_tiles - 1) & 1))) {
             tmem_fence_after_sync();
-            const float inv = 1.0f / l;
+            const float inv = 1.0f / lt;
             unsigned char* orow = static_cast<unsigned char*>(a.out) +
                                   ((size_t)g * a.s + q0 + row) * (kAttnD * 2);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tbase + tlane + 256 + 32 * c, o);
+                tmem_ld32(tbase + tlane + 256 + (uint32_t)(64 * hf + 32 * c), o);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     F2 f[4];
@@ -346,13 +377,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int p = 0; p < 4; ++p)
                         f[p] = f2(__uint_as_float(o[8 * u + 2 * p]) * inv,
                                   __uint_as_float(o[8 * u + 2 * p + 1]) * inv);
-                    store_vec<__nv_bfloat16>(orow, 4 * c + u, IO<__nv_bfloat16>::pack2v(f));
+                    store_vec<__nv_bfloat16>(orow, 8 * hf + 4 * c + u, IO<__nv_bfloat16>::pack2v(f));
                 }
             }
-            if (a.lse) a.lse[(size_t)g * a.s + q0 + row] = (m + log2f(l)) * 0.69314718055994531f;
-        } else {
-            // warp-wide tensor-memory reads must still be matched: nothing
-            // more to read on the abort path
+            if (a.lse && hf == 0)
+                a.lse[(size_t)g * a.s + q0 + row] = (m + log2f(lt)) * 0.69314718055994531f;
         }
     }
     tmem_fence_before_sync();

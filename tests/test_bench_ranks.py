@@ -31,8 +31,11 @@ def _worker(rank, world, port, q):
         local = [12.5, 20.0][rank]          # rank 1 is the slow one
         mx = bench.max_over_ranks(local, "cpu")
         v = bench.job_throughput(1e9, 10, world, mx)
+        # the NCCL arm's record: each collective at its slowest rank
+        coll = bench.collective_record(1 << 20, [0.5, 0.75][rank], [0.9, 0.6][rank],
+                                       world, "cpu")
         dist.barrier()
-        q.put((rank, mx, v))
+        q.put((rank, mx, v, coll))
     finally:
         dist.destroy_process_group()
 
@@ -48,10 +51,14 @@ def test_two_ranks_take_the_slowest_time_and_count_every_rank():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, mx, v in out:
+    for rank, mx, v, coll in out:
         assert mx == 20.0
         # 2 ranks x 10 steps x 1 GB in 20 ms
         assert v == pytest.approx(2 * 10 * 1e9 / 0.020 / 1e9)
+        assert coll["all_reduce_ms"] == 0.75 and coll["rs_ag_ms"] == 0.9
+        assert coll["rs_ag_over_all_reduce"] == pytest.approx(1.2)
+        # 2 (t-1)/t of the tensor per rank: the whole tensor at t = 2
+        assert coll["wire_bytes_per_rank"] == float(1 << 20)
 
 
 def test_single_process_needs_no_group():
