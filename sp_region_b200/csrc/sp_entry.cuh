@@ -7,11 +7,13 @@
 // k_norm_ag streams one row segment per token and has no partial sums to
 // reduce, so it needs no staging ring: each thread loads its vectors of the
 // row straight into registers (read-only, not kept in L1) and prefetches the
-// same vectors of its group's next row while it normalises this one.  G
-// consumer groups per CTA take every G-th row of the CTA; gamma / beta are
-// copied to shared memory once.  The two row reductions (mean, then the
-// centred second moment) are warp butterflies plus one value per warp
-// through shared memory, double-buffered by row parity.
+// same vectors of its group's next row while it normalises this one (the
+// first row's loads are issued before gamma / beta are staged).  G consumer
+// groups per CTA take every G-th row of the CTA; gamma / beta are copied to
+// shared memory once.  The two row reductions (mean, then the centred second
+// moment) are warp butterflies plus one value per warp through shared
+// memory, double-buffered by row parity; the row is centred in place, so the
+// output pass scales it directly.
 #pragma once
 
 #include "sp_device.cuh"
@@ -66,14 +68,6 @@ __global__ void __launch_bounds__(kEntryThreads, 1) k_norm_ag(const __grid_const
     unsigned char* sb = smem + a.param_stride;
     float* red = reinterpret_cast<float*>(smem + 2 * a.param_stride);   // [2][G][2][32]
     const bool has_beta = LN && a.beta;
-    grid_dep_launch();
-    grid_dep_wait();   // the previous kernel's outputs are visible
-    for (int v = tid; v < hv; v += blockDim.x) {
-        store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
-        if (has_beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));
-    }
-    __syncthreads();
-
     auto valid = [&](int k) { return EXACT || c + k * C < hv; };
     const long long step = (long long)G * gridDim.x;
     long long i = blockIdx.x + (long long)g * gridDim.x;   // local row
@@ -84,7 +78,14 @@ __global__ void __launch_bounds__(kEntryThreads, 1) k_norm_ag(const __grid_const
         for (int k = 0; k < V; ++k)
             if (valid(k)) nxt[k] = ld_stream_vec<T>(src, c + k * C);
     };
-    if (i < a.rows) fetch(i);
+    grid_dep_launch();
+    grid_dep_wait();   // the previous kernel's outputs are visible
+    if (i < a.rows) fetch(i);   // in flight while the parameters are staged
+    for (int v = tid; v < hv; v += blockDim.x) {
+        store_vec<T>(sg, v, load_vec<T>(a.gamma, v));
+        if (has_beta) store_vec<T>(sb, v, load_vec<T>(a.beta, v));
+    }
+    __syncthreads();
     auto group_sum = [&](float x, float* slot) {
         x = warp_sum(x);
         if (lane == 0) slot[c >> 5] = x;
@@ -115,8 +116,8 @@ __global__ void __launch_bounds__(kEntryThreads, 1) k_norm_ag(const __grid_const
                 if (valid(k))
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
-                        const F2 d = sub2(acc[k][p], mean2);
-                        q2 = fma2(d, d, q2);
+                        acc[k][p] = sub2(acc[k][p], mean2);   // centred in place
+                        q2 = fma2(acc[k][p], acc[k][p], q2);
                     }
             rstd = rsqrtf(group_sum(hsum(q2), slots + 32) * a.inv_h + a.eps);
         } else {
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kEntryThreads, 1) k_norm_ag(const __grid_const
             rstd = rsqrtf(group_sum(hsum(q2), slots) * a.inv_h + a.eps);
         }
 
-        const F2 mean2 = f2(mean), rstd2 = f2(rstd);
+        const F2 rstd2 = f2(rstd);
         const size_t orow = (size_t)(a.row0 + i) * a.seg_bytes;   // gathered: global row
 #pragma unroll
         for (int k = 0; k < V; ++k) {
@@ -141,15 +142,14 @@ __global__ void __launch_bounds__(kEntryThreads, 1) k_norm_ag(const __grid_const
                 F2 b[4];
                 IO<T>::unpack2(load_vec<T>(sb, v), b);
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    o[p] = fma2(mul2(sub2(acc[k][p], mean2), rstd2), gm[p], b[p]);
+                for (int p = 0; p < 4; ++p) o[p] = fma2(mul2(acc[k][p], rstd2), gm[p], b[p]);
             } else {
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    o[p] = mul2(mul2(LN ? sub2(acc[k][p], mean2) : acc[k][p], rstd2), gm[p]);
+                for (int p = 0; p < 4; ++p) o[p] = mul2(mul2(acc[k][p], rstd2), gm[p]);
             }
             const Vec ov = IO<T>::pack2v(o);
-            for (int q = 0; q < a.n_gathered; ++q)
+            store_vec<T>(static_cast<unsigned char*>(a.gathered[0]) + orow, v, ov);
+            for (int q = 1; q < a.n_gathered; ++q)
                 store_vec<T>(static_cast<unsigned char*>(a.gathered[q]) + orow, v, ov);
         }
         if (c == 0) {

@@ -28,6 +28,11 @@ CASES = {
     "ln_h1000_ragged": dict(base="C2", s=64, b=2, h=1000, t=4),
     "f32_rms_h520_ragged": dict(base="C3", s=48, b=2, h=520, t=2, dtype="f32"),
     "ln_h2048_no_beta": dict(base="C2", s=64, b=2, h=2048, t=4, has_beta=False),
+    # many rows per consumer group (the prefetch runs across every row)
+    "ln_h6144_many_rows": dict(base="C2", s=1024, b=2),
+    "rms_h4096_many_rows": dict(base="C3", s=4096, b=1, h=4096, t=4),
+    # one-warp consumer groups
+    "ln_h1024_t2": dict(base="C2", s=512, b=1, h=1024, t=2),
 }
 
 
@@ -79,7 +84,8 @@ def test_entry_forward_matches_oracle(name, plan):
         assert (np.abs(mean.t.cpu().numpy() - ref["mean"]) <= 1e-5 * rms).all()
 
 
-@pytest.mark.parametrize("name", ["ln_h6144_t8", "ln_general_h100"])
+@pytest.mark.parametrize("name", ["ln_h6144_t8", "ln_general_h100", "rms_h4096_many_rows",
+                                  "ln_h1000_ragged"])
 def test_entry_as_ranks(name):
     """t row-range calls, each normalising its own shard and pushing into
     every rank's gathered buffer, reproduce the whole call bit for bit."""
