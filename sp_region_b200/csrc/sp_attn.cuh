@@ -14,21 +14,28 @@
 //
 // k_ring_attn: one CTA per (128-query tile, head); head dimension 128.
 //   warp 0 (one lane)  TMA producer: Q once, K and V tiles (2 stages each)
-//   warp 1 (one lane)  MMA issuer: S = Q K^T (tcgen05 kind::f16, M = N = 128,
-//                      two tensor-memory score buffers, so the next tile's
-//                      scores are computed while this one's softmax runs)
-//                      and O += P V (V read as an MN-major operand)
+//   warp 1 (one lane)  MMA issuer, in the order S0, S1, PV0, S2, PV1, S3, ...:
+//                      S_j = Q K_j^T (tcgen05 kind::f16, M = N = 128) into
+//                      tensor-memory buffer j % 2, and O += P_j V_j with P_j
+//                      read from tensor memory (where the softmax wrote it
+//                      over S_j) and V read as an MN-major operand.  The
+//                      tensor cores run one CTA's MMAs in issue order, so
+//                      S_{j+2} overwrites buffer j % 2 only after PV_j has
+//                      read P_j from it.
 //   warps 2..9         softmax: each query row is shared by two warps of the
 //                      same sub-partition (warps w and w + 4 read the same
 //                      tensor-memory lanes), one taking score columns 0..63,
 //                      the other 64..127.  The pair exchanges its halves'
 //                      maxima once per tile; both keep the same running
-//                      maximum, so their partial sums add up at the end.  O
-//                      is rescaled in tensor memory when the maximum grows,
-//                      P written to shared memory in the operand layout
-//                      (K-major, 128-byte swizzle); at the end O / l to
-//                      global memory and the log-sum-exp
-// Tensor memory: S0 columns [0, 128), S1 [128, 256), O [256, 384).
+//                      maximum, so their partial sums add up at the end.  The
+//                      maximum used for the exponentials moves only when a
+//                      row's true maximum exceeds it by more than 8 (log2
+//                      units): the probabilities then stay below 2^8, and O is
+//                      rescaled in tensor memory only on those tiles, so in
+//                      most tiles the softmax never waits for the previous
+//                      PV.  P goes to tensor memory as bf16 pairs; at the end
+//                      O / l to global memory and the log-sum-exp
+// Tensor memory: S0/P0 columns [0, 128), S1/P1 [128, 256), O [256, 384).
 #pragma once
 
 #include "sp_gemm.cuh"
@@ -58,8 +65,10 @@ struct AttnTail {
     uint64_t q_full;
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2], s_free[2];
-    uint64_t p_full, o_done, drain;
+    uint64_t s_full[2];          // S_j in buffer j % 2
+    uint64_t p_full[2];          // P_j in buffer j % 2 (and O rescaled for tile j)
+    uint64_t o_done[2];          // PV_j complete, by tile parity
+    uint64_t drain;
     uint32_t tmem_base;
     int abort;
     uint64_t pair[4][2];         // per row quarter and tile parity: both halves' maxima posted
@@ -96,11 +105,21 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t r[32])
         : "memory");
 }
 
-// Generic-proxy writes to shared memory become visible to the tensor cores.
-__device__ __forceinline__ void fence_async_smem()
+// D (+)= A B with A (M x K, K-major) in tensor memory, B in shared memory.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t accumulate)
 {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
+
+// The running maximum (log2 units) moves only when the tile's exceeds it by
+// more than this, bounding the probabilities by 2^8.
+constexpr float kAttnMaxSlack = 8.0f;
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_ring_attn(const __grid_constant__ AttnArgs a, const __grid_constant__ AttnMaps maps)
@@ -111,8 +130,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     unsigned char* sq = sm;                                 // Q: 2 chunks of 16 KB
     unsigned char* sk = sm + kAttnTile;                     // K: 2 stages
     unsigned char* sv = sm + 3 * kAttnTile;                 // V: 2 stages
-    unsigned char* sp = sm + 5 * kAttnTile;                 // P
-    AttnTail* tail = reinterpret_cast<AttnTail*>(sm + 6 * kAttnTile);
+    AttnTail* tail = reinterpret_cast<AttnTail*>(sm + 5 * kAttnTile);
     volatile int* abort = &tail->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long q0 = (long long)blockIdx.x * kAttnBM;   // first query row
@@ -135,10 +153,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(smem_addr(&tail->v_full[i]), 1);
             mbar_init(smem_addr(&tail->v_empty[i]), 1);
             mbar_init(smem_addr(&tail->s_full[i]), 1);
-            mbar_init(smem_addr(&tail->s_free[i]), 8);
+            mbar_init(smem_addr(&tail->p_full[i]), 8);
+            mbar_init(smem_addr(&tail->o_done[i]), 1);
         }
-        mbar_init(smem_addr(&tail->p_full), 8);
-        mbar_init(smem_addr(&tail->o_done), 1);
         mbar_init(smem_addr(&tail->drain), 1);
         for (int qq = 0; qq < 4; ++qq) {   // every thread of the two warps arrives
             mbar_init(smem_addr(&tail->pair[qq][0]), 64);
@@ -212,19 +229,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(kAttnBM, kAttnBN);
             constexpr uint32_t idesc_o = idesc_bf16(kAttnBM, kAttnD) | (1u << 16);  // B MN-major
-            const uint32_t q_s = smem_addr(sq), p_s = smem_addr(sp);
+            const uint32_t q_s = smem_addr(sq);
             bool ok = mbar_wait(smem_addr(&tail->q_full), 0u, abort, ERR_WAIT_FULL);
-            // S_j = Q K_j^T into score buffer j & 1
+            // S_j = Q K_j^T into buffer j % 2 (after PV_{j-2}, which read P_{j-2} there)
             auto issue_s = [&](int j) -> bool {
                 const int b = j & 1;
-                if (j >= 2 && !mbar_wait(smem_addr(&tail->s_free[b]),
-                                         (uint32_t)(((j >> 1) - 1) & 1), abort, ERR_WAIT_FULL))
-                    return false;
-                if (!mbar_wait(smem_addr(&tail->k_full[j & 1]), (uint32_t)((j >> 1) & 1), abort,
+                if (!mbar_wait(smem_addr(&tail->k_full[b]), (uint32_t)((j >> 1) & 1), abort,
                                ERR_WAIT_FULL))
                     return false;
                 tmem_fence_after_sync();
-                const uint32_t k_s = smem_addr(sk + (size_t)(j & 1) * kAttnTile);
+                const uint32_t k_s = smem_addr(sk + (size_t)b * kAttnTile);
 #pragma unroll
                 for (int kk = 0; kk < kAttnD / 16; ++kk) {
                     // 16 of the 128 head features: chunk kk / 4, 32 bytes each
@@ -232,36 +246,38 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     umma_bf16(tbase + (uint32_t)(b * kAttnBN), sw128_desc(q_s + off),
                               sw128_desc(k_s + off), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(smem_addr(&tail->k_empty[j & 1]));
+                umma_commit(smem_addr(&tail->k_empty[b]));
                 umma_commit(smem_addr(&tail->s_full[b]));
                 return true;
             };
             if (ok) ok = issue_s(0);
+            if (ok && n_tiles > 1) ok = issue_s(1);
             for (int j = 0; ok && j < n_tiles; ++j) {
-                if (j + 1 < n_tiles && !issue_s(j + 1)) {
-                    ok = false;
-                    break;
-                }
-                if (!mbar_wait(smem_addr(&tail->p_full), (uint32_t)(j & 1), abort,
+                const int b = j & 1;
+                if (!mbar_wait(smem_addr(&tail->p_full[b]), (uint32_t)((j >> 1) & 1), abort,
                                ERR_WAIT_FULL) ||
-                    !mbar_wait(smem_addr(&tail->v_full[j & 1]), (uint32_t)((j >> 1) & 1), abort,
+                    !mbar_wait(smem_addr(&tail->v_full[b]), (uint32_t)((j >> 1) & 1), abort,
                                ERR_WAIT_FULL)) {
                     ok = false;
                     break;
                 }
                 tmem_fence_after_sync();
-                const uint32_t v_s = smem_addr(sv + (size_t)(j & 1) * kAttnTile);
+                const uint32_t v_s = smem_addr(sv + (size_t)b * kAttnTile);
 #pragma unroll
                 for (int kk = 0; kk < kAttnBN / 16; ++kk) {
-                    // keys 16 kk .. 16 kk + 15: P chunk kk / 4 (K-major), V rows
-                    // 16 kk .. (two 8-row groups of 1024 bytes, MN-major)
-                    const uint32_t poff = (uint32_t)(kk >> 2) * (kAttnTile / 2) + (uint32_t)(kk & 3) * 32;
-                    umma_bf16(tbase + 256, sw128_desc(p_s + poff),
-                              sw128_desc_mn(v_s + (uint32_t)kk * 2048, kAttnTile / 2), idesc_o,
-                              (j > 0 || kk > 0) ? 1u : 0u);
+                    // keys 16 kk .. 16 kk + 15: P columns 8 kk .. (two bf16 a
+                    // column), V rows 16 kk .. (two 8-row groups of 1024
+                    // bytes, MN-major)
+                    umma_bf16_ts(tbase + 256, tbase + (uint32_t)(b * kAttnBN + 8 * kk),
+                                 sw128_desc_mn(v_s + (uint32_t)kk * 2048, kAttnTile / 2), idesc_o,
+                                 (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(smem_addr(&tail->v_empty[j & 1]));
-                umma_commit(smem_addr(&tail->o_done));
+                umma_commit(smem_addr(&tail->v_empty[b]));
+                umma_commit(smem_addr(&tail->o_done[b]));
+                if (j + 2 < n_tiles && !issue_s(j + 2)) {
+                    ok = false;
+                    break;
+                }
             }
             // every issued MMA has finished before the CTA tears down
             umma_commit(smem_addr(&tail->drain));
@@ -281,7 +297,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const bool w = mbar_wait(bar, parity, abort, ERR_WAIT_FULL);
             return __all_sync(0xFFFFFFFFu, w) != 0;
         };
-        float m = -INFINITY, l = 0.f;   // running maximum (log2 units), this half's sum
+        float m = -INFINITY, l = 0.f;   // maximum in use (log2 units), this half's sum
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int b = j & 1;
@@ -294,66 +310,57 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
                 tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + 64 * hf + 32 * c), sc + 32 * c);
-            // the score buffer may be overwritten by tile j + 2
-            tmem_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&tail->s_free[b]));
             float mx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sc[i]));
             tail->xmax[b][hf][row] = mx;
+            // past this barrier both warps of the row have read their scores,
+            // so either may write P over them
+            tmem_fence_before_sync();
             mbar_arrive(smem_addr(&tail->pair[q][b]));
             if (!wait_all(smem_addr(&tail->pair[q][b]), (uint32_t)((j >> 1) & 1))) {
                 ok = false;
                 break;
             }
-            mx = fmaxf(mx, tail->xmax[b][hf ^ 1][row]);   // the row's maximum
-            const float m_new = fmaxf(m, mx * a.scale_log2);
-            const float alpha = exp2f(m - m_new);   // 0 at the first tile
+            tmem_fence_after_sync();
+            mx = fmaxf(mx, tail->xmax[b][hf ^ 1][row]) * a.scale_log2;   // the row's maximum
+            const bool bump = mx > m + kAttnMaxSlack;   // first tile: m = -inf
+            const float alpha = bump ? exp2f(m - mx) : 1.0f;   // 0 at the first tile
+            if (bump) m = mx;
             float lsum = 0.f;
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float p0 = exp2f(fmaf(__uint_as_float(sc[2 * i]), a.scale_log2, -m_new));
-                const float p1 = exp2f(fmaf(__uint_as_float(sc[2 * i + 1]), a.scale_log2, -m_new));
+                const float p0 = exp2f(fmaf(__uint_as_float(sc[2 * i]), a.scale_log2, -m));
+                const float p1 = exp2f(fmaf(__uint_as_float(sc[2 * i + 1]), a.scale_log2, -m));
                 lsum += p0 + p1;
                 pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
             }
             l = l * alpha + lsum;
-            m = m_new;
-            if (j > 0) {
-                // O of the previous tiles is complete and P may be reused
-                if (!wait_all(smem_addr(&tail->o_done), (uint32_t)((j - 1) & 1))) {
+            // this half of the P row: keys 64 hf .. as bf16 pairs, columns
+            // 32 hf .. of buffer b
+            tmem_st32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * hf), pk);
+            if (j > 0 && __any_sync(0xFFFFFFFFu, bump)) {
+                // O of the previous tiles is complete: rescale this half
+                if (!wait_all(smem_addr(&tail->o_done[b ^ 1]), (uint32_t)(((j - 1) >> 1) & 1))) {
                     ok = false;
                     break;
                 }
                 tmem_fence_after_sync();
-                if (__any_sync(0xFFFFFFFFu, alpha != 1.0f)) {
 #pragma unroll 1
-                    for (int c = 0; c < 2; ++c) {
-                        uint32_t o[32];
-                        const uint32_t oc = tbase + tlane + 256 + (uint32_t)(64 * hf + 32 * c);
-                        tmem_ld32(oc, o);
+                for (int c = 0; c < 2; ++c) {
+                    uint32_t o[32];
+                    const uint32_t oc = tbase + tlane + 256 + (uint32_t)(64 * hf + 32 * c);
+                    tmem_ld32(oc, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(oc, o);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(oc, o);
                 }
             }
-            // this half of the P row into chunk hf of the operand layout:
-            // 16-byte unit u of row r at (u ^ (r % 8)) within its 128-byte row
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint32_t off = (uint32_t)hf * (kAttnTile / 2) + (uint32_t)(row >> 3) * 1024 +
-                                     (uint32_t)(row & 7) * 128 + (uint32_t)((u ^ (row & 7)) << 4);
-                *reinterpret_cast<uint4*>(sp + off) =
-                    make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            }
-            fence_async_smem();
+            tmem_wait_st();
             tmem_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&tail->p_full));
+            if (lane == 0) mbar_arrive(smem_addr(&tail->p_full[b]));
         }
         // the row's sum: both halves post theirs (a half that left the loop
         // early makes the other's bounded wait run out, never hang)
@@ -361,7 +368,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(smem_addr(&tail->pair_fin[q]));
         if (ok && !wait_all(smem_addr(&tail->pair_fin[q]), 0u)) ok = false;
         const float lt = tail->xsum[0][row] + tail->xsum[1][row];   // same bits in both warps
-        if (ok && wait_all(smem_addr(&tail->o_done), (uint32_t)((n_tiles - 1) & 1))) {
+        if (ok && wait_all(smem_addr(&tail->o_done[(n_tiles - 1) & 1]),
+                           (uint32_t)(((n_tiles - 1) >> 1) & 1))) {
             tmem_fence_after_sync();
             const float inv = 1.0f / lt;
             unsigned char* orow = static_cast<unsigned char*>(a.out) +

@@ -245,7 +245,7 @@ int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const v
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
     a.out = out;
     a.lse = lse;
-    const size_t smem = 1024 + 6 * (size_t)kAttnTile + ((sizeof(AttnTail) + 127) & ~(size_t)127);
+    const size_t smem = 1024 + 5 * (size_t)kAttnTile + ((sizeof(AttnTail) + 127) & ~(size_t)127);
     if (smem > (size_t)dev.smem_optin) return SP_ERR_UNSUPPORTED;
     const void* kern = (const void*)k_ring_attn;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
