@@ -117,6 +117,22 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, u
         : "memory");
 }
 
+// 2^x by the transcendental unit's approximation (PTX ex2.approx.ftz: at most
+// 2 ulp; results below 2^-126 flush to zero).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // The running maximum (log2 units) moves only when the tile's exceeds it by
 // more than this, bounding the probabilities by 2^8.
 constexpr float kAttnMaxSlack = 8.0f;
@@ -310,9 +326,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
                 tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + 64 * hf + 32 * c), sc + 32 * c);
-            float mx = -INFINITY;
+            float mx;
+            {
+                // two independent chains of three-input maxima
+                float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-            for (int i = 0; i < 64; ++i) mx = fmaxf(mx, __uint_as_float(sc[i]));
+                for (int i = 0; i < 64; i += 4) {
+                    m0 = max3f(m0, __uint_as_float(sc[i]), __uint_as_float(sc[i + 1]));
+                    m1 = max3f(m1, __uint_as_float(sc[i + 2]), __uint_as_float(sc[i + 3]));
+                }
+                mx = fmaxf(m0, m1);
+            }
             tail->xmax[b][hf][row] = mx;
             // past this barrier both warps of the row have read their scores,
             // so either may write P over them
@@ -325,18 +349,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_fence_after_sync();
             mx = fmaxf(mx, tail->xmax[b][hf ^ 1][row]) * a.scale_log2;   // the row's maximum
             const bool bump = mx > m + kAttnMaxSlack;   // first tile: m = -inf
-            const float alpha = bump ? exp2f(m - mx) : 1.0f;   // 0 at the first tile
+            const float alpha = bump ? ex2_approx(m - mx) : 1.0f;   // 0 at the first tile
             if (bump) m = mx;
-            float lsum = 0.f;
+            // p = 2^(s * scale - m): the scaling as paired fused multiply-adds,
+            // the sum in two pair lanes
+            const F2 scale2 = f2(a.scale_log2), negm2 = f2(-m);
+            F2 lsum2 = f2(0.f);
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                const float p0 = exp2f(fmaf(__uint_as_float(sc[2 * i]), a.scale_log2, -m));
-                const float p1 = exp2f(fmaf(__uint_as_float(sc[2 * i + 1]), a.scale_log2, -m));
-                lsum += p0 + p1;
+                const float2 x = halves(fma2(f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])),
+                                             scale2, negm2));
+                const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+                lsum2 = add2(lsum2, f2(p0, p1));
                 pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
             }
-            l = l * alpha + lsum;
+            l = l * alpha + hsum(lsum2);
             // this half of the P row: keys 64 hf .. as bf16 pairs, columns
             // 32 hf .. of buffer b
             tmem_st32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * hf), pk);
