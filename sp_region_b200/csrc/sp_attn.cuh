@@ -45,7 +45,9 @@ namespace spk {
 constexpr int kAttnBM = 128;        // queries per CTA
 constexpr int kAttnBN = 128;        // keys per tile
 constexpr int kAttnD = 128;         // head dimension
-constexpr int kAttnThreads = 320;   // producer, MMA, 8 softmax warps
+constexpr int kAttnSplit = 2;                      // softmax warps per query row
+constexpr int kAttnCols = 128 / kAttnSplit;        // score columns per softmax warp
+constexpr int kAttnThreads = 64 + 4 * kAttnSplit * 32;   // producer, MMA, softmax warps
 constexpr uint32_t kAttnTile = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column chunks)
 
 struct AttnArgs {
@@ -71,10 +73,10 @@ struct AttnTail {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    uint64_t pair[4][2];         // per row quarter and tile parity: both halves' maxima posted
-    uint64_t pair_fin[4];        // per row quarter: both halves' sums posted
-    float xmax[2][2][kAttnBM];   // [tile parity][half][row]: the halves' maxima
-    float xsum[2][kAttnBM];      // [half][row]: the halves' sums at the end
+    uint64_t pair[4][2];         // per row quarter and tile parity: every slice's maximum posted
+    uint64_t pair_fin[4];        // per row quarter: every slice's sum posted
+    float xmax[2][kAttnSplit][kAttnBM];   // [tile parity][column slice][row]
+    float xsum[kAttnSplit][kAttnBM];      // [column slice][row]: the slices' sums at the end
 };
 
 // Shared-memory descriptor of an MN-major tile with 128-byte swizzle: 64
@@ -169,14 +171,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(smem_addr(&tail->v_full[i]), 1);
             mbar_init(smem_addr(&tail->v_empty[i]), 1);
             mbar_init(smem_addr(&tail->s_full[i]), 1);
-            mbar_init(smem_addr(&tail->p_full[i]), 8);
+            mbar_init(smem_addr(&tail->p_full[i]), 4 * kAttnSplit);   // every softmax warp
             mbar_init(smem_addr(&tail->o_done[i]), 1);
         }
         mbar_init(smem_addr(&tail->drain), 1);
         for (int qq = 0; qq < 4; ++qq) {   // every thread of the two warps arrives
-            mbar_init(smem_addr(&tail->pair[qq][0]), 64);
-            mbar_init(smem_addr(&tail->pair[qq][1]), 64);
-            mbar_init(smem_addr(&tail->pair_fin[qq]), 64);
+            mbar_init(smem_addr(&tail->pair[qq][0]), 32 * kAttnSplit);
+            mbar_init(smem_addr(&tail->pair[qq][1]), 32 * kAttnSplit);
+            mbar_init(smem_addr(&tail->pair_fin[qq]), 32 * kAttnSplit);
         }
         tail->abort = 0;
         mbar_init_fence();
@@ -301,8 +303,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_wait(smem_addr(&tail->drain), 0u, &no_abort, ERR_DRAIN);
         }
     } else {
-        // softmax warps 2..9: query row 32 (warp % 4) + lane; half hf of the
-        // score columns (and of O's columns); the pair (w, w + 4) shares rows
+        // softmax warps 2 ..: query row 32 (warp % 4) + lane; column slice hf
+        // of the scores (and of O's columns); warps w, w + 4, ... share rows
         const int q = warp & 3;
         const int hf = (warp - 2) >> 2;
         const int row = 32 * q + lane;
@@ -322,16 +324,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 break;
             }
             tmem_fence_after_sync();
-            uint32_t sc[64];
+            uint32_t sc[kAttnCols];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + 64 * hf + 32 * c), sc + 32 * c);
+            for (int c = 0; c < kAttnCols / 32; ++c)
+                tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + kAttnCols * hf + 32 * c), sc + 32 * c);
             float mx;
             {
                 // two independent chains of three-input maxima
                 float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < 64; i += 4) {
+                for (int i = 0; i < kAttnCols; i += 4) {
                     m0 = max3f(m0, __uint_as_float(sc[i]), __uint_as_float(sc[i + 1]));
                     m1 = max3f(m1, __uint_as_float(sc[i + 2]), __uint_as_float(sc[i + 3]));
                 }
@@ -347,7 +349,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 break;
             }
             tmem_fence_after_sync();
-            mx = fmaxf(mx, tail->xmax[b][hf ^ 1][row]) * a.scale_log2;   // the row's maximum
+#pragma unroll
+            for (int h = 0; h < kAttnSplit; ++h) mx = fmaxf(mx, tail->xmax[b][h][row]);
+            mx *= a.scale_log2;   // the row's maximum
             const bool bump = mx > m + kAttnMaxSlack;   // first tile: m = -inf
             const float alpha = bump ? ex2_approx(m - mx) : 1.0f;   // 0 at the first tile
             if (bump) m = mx;
@@ -355,9 +359,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             // the sum in two pair lanes
             const F2 scale2 = f2(a.scale_log2), negm2 = f2(-m);
             F2 lsum2 = f2(0.f);
-            uint32_t pk[32];
+            uint32_t pk[kAttnCols / 2];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < kAttnCols / 2; ++i) {
                 const float2 x = halves(fma2(f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])),
                                              scale2, negm2));
                 const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
@@ -365,9 +369,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
             }
             l = l * alpha + hsum(lsum2);
-            // this half of the P row: keys 64 hf .. as bf16 pairs, columns
-            // 32 hf .. of buffer b
-            tmem_st32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * hf), pk);
+            // this slice of the P row: keys kAttnCols hf .. as bf16 pairs,
+            // columns kAttnCols / 2 hf .. of buffer b
+            if constexpr (kAttnCols == 64)
+                tmem_st32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * hf), pk);
+            else
+                tmem_st16(tbase + tlane + (uint32_t)(b * kAttnBN + 16 * hf), pk);
             if (j > 0 && __any_sync(0xFFFFFFFFu, bump)) {
                 // O of the previous tiles is complete: rescale this half
                 if (!wait_all(smem_addr(&tail->o_done[b ^ 1]), (uint32_t)(((j - 1) >> 1) & 1))) {
@@ -376,9 +383,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
                 tmem_fence_after_sync();
 #pragma unroll 1
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < kAttnCols / 32; ++c) {
                     uint32_t o[32];
-                    const uint32_t oc = tbase + tlane + 256 + (uint32_t)(64 * hf + 32 * c);
+                    const uint32_t oc = tbase + tlane + 256 + (uint32_t)(kAttnCols * hf + 32 * c);
                     tmem_ld32(oc, o);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
@@ -395,7 +402,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tail->xsum[hf][row] = l;
         mbar_arrive(smem_addr(&tail->pair_fin[q]));
         if (ok && !wait_all(smem_addr(&tail->pair_fin[q]), 0u)) ok = false;
-        const float lt = tail->xsum[0][row] + tail->xsum[1][row];   // same bits in both warps
+        float lt = tail->xsum[0][row];   // the same order, so the same bits, in every warp
+#pragma unroll
+        for (int h = 1; h < kAttnSplit; ++h) lt += tail->xsum[h][row];
         if (ok && wait_all(smem_addr(&tail->o_done[(n_tiles - 1) & 1]),
                            (uint32_t)(((n_tiles - 1) >> 1) & 1))) {
             tmem_fence_after_sync();
@@ -403,9 +412,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             unsigned char* orow = static_cast<unsigned char*>(a.out) +
                                   ((size_t)g * a.s + q0 + row) * (kAttnD * 2);
 #pragma unroll 1
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < kAttnCols / 32; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tbase + tlane + 256 + (uint32_t)(64 * hf + 32 * c), o);
+                tmem_ld32(tbase + tlane + 256 + (uint32_t)(kAttnCols * hf + 32 * c), o);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     F2 f[4];
@@ -413,7 +422,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     for (int p = 0; p < 4; ++p)
                         f[p] = f2(__uint_as_float(o[8 * u + 2 * p]) * inv,
                                   __uint_as_float(o[8 * u + 2 * p + 1]) * inv);
-                    store_vec<__nv_bfloat16>(orow, 8 * hf + 4 * c + u, IO<__nv_bfloat16>::pack2v(f));
+                    store_vec<__nv_bfloat16>(orow, (kAttnCols / 8) * hf + 4 * c + u,
+                                             IO<__nv_bfloat16>::pack2v(f));
                 }
             }
             if (a.lse && hf == 0)
