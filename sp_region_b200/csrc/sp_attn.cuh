@@ -12,18 +12,25 @@
 // in ring order: block r first, then r-1, r-2, ... (mod t), 128 keys per
 // tile.
 //
-// k_ring_attn: one CTA per (128-query tile, head); head dimension 128.
-//   warp 0 (one lane)  TMA producer: Q once, K and V tiles (2 stages each)
-//   warp 1 (one lane)  MMA issuer, in the order S0, S1, PV0, S2, PV1, S3, ...:
-//                      S_j = Q K_j^T (tcgen05 kind::f16, M = N = 128) into
-//                      tensor-memory buffer j % 2, and O += P_j V_j with P_j
-//                      read from tensor memory (where the softmax wrote it
-//                      over S_j) and V read as an MN-major operand.  The
-//                      tensor cores run one CTA's MMAs in issue order, so
-//                      S_{j+2} overwrites buffer j % 2 only after PV_j has
-//                      read P_j from it.
-//   warps 2..9         softmax: each query row is shared by two warps of the
-//                      same sub-partition (warps w and w + 4 read the same
+// k_ring_attn<QT>: one CTA per QT 128-query tiles of one head (QT = 2 when a
+// rank's block holds an even number of tiles, so both tiles visit the key
+// tiles in the same ring order and share every K / V tile); head dim 128.
+//   warp 0 (one lane)  TMA producer: the Q tiles once, K and V tiles (2
+//                      stages each)
+//   warp 1 (one lane)  MMA issuer.  S_j = Q K_j^T (tcgen05 kind::f16, M = N =
+//                      128) into a tensor-memory score buffer, and O += P_j V_j
+//                      with P_j read from tensor memory (where the softmax
+//                      wrote it over S_j) and V read as an MN-major operand.
+//                      QT = 1: two score buffers by tile parity, in the order
+//                      S0, S1, PV0, S2, PV1, ...  QT = 2: one score buffer per
+//                      query tile, in the order S_A0, S_B0, PV_A0, S_A1, PV_B0,
+//                      S_B1, ..., so the tensor cores run one query tile's PV
+//                      and next scores while the other tile's softmax runs.
+//                      The tensor cores run one CTA's MMAs in issue order, so
+//                      S overwrites a buffer only after the PV that read the
+//                      P there.
+//   softmax warps      8 per query tile: each query row is shared by two warps
+//                      of the same sub-partition (they read the same
 //                      tensor-memory lanes), one taking score columns 0..63,
 //                      the other 64..127.  The pair exchanges its halves'
 //                      maxima once per tile; both keep the same running
@@ -35,7 +42,9 @@
 //                      most tiles the softmax never waits for the previous
 //                      PV.  P goes to tensor memory as bf16 pairs; at the end
 //                      O / l to global memory and the log-sum-exp
-// Tensor memory: S0/P0 columns [0, 128), S1/P1 [128, 256), O [256, 384).
+// Tensor memory: QT = 1: S0/P0 [0, 128), S1/P1 [128, 256), O [256, 384);
+// QT = 2: S/P of tile A [0, 128), of tile B [128, 256), O_A [256, 384), O_B
+// [384, 512).
 #pragma once
 
 #include "sp_gemm.cuh"
@@ -47,7 +56,8 @@ constexpr int kAttnBN = 128;        // keys per tile
 constexpr int kAttnD = 128;         // head dimension
 constexpr int kAttnSplit = 2;                      // softmax warps per query row
 constexpr int kAttnCols = 128 / kAttnSplit;        // score columns per softmax warp
-constexpr int kAttnThreads = 64 + 4 * kAttnSplit * 32;   // producer, MMA, softmax warps
+constexpr int kAttnSoftWarps = 4 * kAttnSplit;     // softmax warps per query tile
+__host__ __device__ constexpr int attn_threads(int qt) { return 64 + qt * kAttnSoftWarps * 32; }
 constexpr uint32_t kAttnTile = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column chunks)
 
 struct AttnArgs {
@@ -63,20 +73,23 @@ struct AttnMaps {
     CUtensorMap q, k, v;      // [bh * s][128] bf16, boxes of 64 x 128
 };
 
+// Barriers and scratch after the tiles; arrays of 2 are indexed by the score
+// buffer (tile parity for QT = 1, query tile for QT = 2).
+template <int QT>
 struct AttnTail {
     uint64_t q_full;
     uint64_t k_full[2], k_empty[2];
     uint64_t v_full[2], v_empty[2];
-    uint64_t s_full[2];          // S_j in buffer j % 2
-    uint64_t p_full[2];          // P_j in buffer j % 2 (and O rescaled for tile j)
-    uint64_t o_done[2];          // PV_j complete, by tile parity
+    uint64_t s_full[2];          // S in buffer
+    uint64_t p_full[2];          // P in buffer (and O rescaled for its tile)
+    uint64_t o_done[2];          // the PV that read buffer's P complete
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    uint64_t pair[4][2];         // per row quarter and tile parity: every slice's maximum posted
-    uint64_t pair_fin[4];        // per row quarter: every slice's sum posted
-    float xmax[2][kAttnSplit][kAttnBM];   // [tile parity][column slice][row]
-    float xsum[kAttnSplit][kAttnBM];      // [column slice][row]: the slices' sums at the end
+    uint64_t pair[QT][4][2];     // per query tile, row quarter and tile parity: every slice's maximum posted
+    uint64_t pair_fin[QT][4];    // per query tile and row quarter: every slice's sum posted
+    float xmax[QT][2][kAttnSplit][kAttnBM];   // [query tile][tile parity][column slice][row]
+    float xsum[QT][kAttnSplit][kAttnBM];      // [query tile][column slice][row]
 };
 
 // Shared-memory descriptor of an MN-major tile with 128-byte swizzle: 64
@@ -139,22 +152,23 @@ __device__ __forceinline__ float max3f(float a, float b, float c)
 // more than this, bounding the probabilities by 2^8.
 constexpr float kAttnMaxSlack = 8.0f;
 
-__global__ void __launch_bounds__(kAttnThreads, 1)
+template <int QT>
+__global__ void __launch_bounds__(attn_threads(QT), 1)
     k_ring_attn(const __grid_constant__ AttnArgs a, const __grid_constant__ AttnMaps maps)
 {
     extern __shared__ __align__(1024) unsigned char asm_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(asm_raw) + 1023) & ~(uintptr_t)1023);
-    unsigned char* sq = sm;                                 // Q: 2 chunks of 16 KB
-    unsigned char* sk = sm + kAttnTile;                     // K: 2 stages
-    unsigned char* sv = sm + 3 * kAttnTile;                 // V: 2 stages
-    AttnTail* tail = reinterpret_cast<AttnTail*>(sm + 5 * kAttnTile);
+    unsigned char* sq = sm;                                   // Q: QT tiles of 2 chunks
+    unsigned char* sk = sm + QT * kAttnTile;                  // K: 2 stages
+    unsigned char* sv = sm + (QT + 2) * kAttnTile;            // V: 2 stages
+    AttnTail<QT>* tail = reinterpret_cast<AttnTail<QT>*>(sm + (QT + 4) * kAttnTile);
     volatile int* abort = &tail->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long q0 = (long long)blockIdx.x * kAttnBM;   // first query row
-    const long long g = blockIdx.y;                          // batch * head index
+    const long long q0 = (long long)blockIdx.x * (QT * kAttnBM);   // first query row
+    const long long g = blockIdx.y;                                 // batch * head index
     const long long per = a.s / a.t;
-    const int rank = (int)(q0 / per);                        // the queries' rank
+    const int rank = (int)(q0 / per);                               // the queries' rank
     const int T = a.tiles_per_block;
     const int n_tiles = a.t * T;
     // first key row of tile j: block (rank - j / T) mod t, its (j % T)-th tile
@@ -162,6 +176,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int blk = ((rank - j / T) % a.t + a.t) % a.t;
         return (long long)blk * per + (long long)(j % T) * kAttnBN;
     };
+    // score buffer of query tile qt at key tile j, and the phase of its barriers
+    auto sbuf = [](int qt, int j) -> int { return QT == 1 ? (j & 1) : qt; };
+    auto sphase = [](int j) -> uint32_t { return QT == 1 ? (uint32_t)((j >> 1) & 1) : (uint32_t)(j & 1); };
 
     if (threadIdx.x == 0) {
         mbar_init(smem_addr(&tail->q_full), 1);
@@ -171,15 +188,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_init(smem_addr(&tail->v_full[i]), 1);
             mbar_init(smem_addr(&tail->v_empty[i]), 1);
             mbar_init(smem_addr(&tail->s_full[i]), 1);
-            mbar_init(smem_addr(&tail->p_full[i]), 4 * kAttnSplit);   // every softmax warp
+            mbar_init(smem_addr(&tail->p_full[i]), kAttnSoftWarps);   // a query tile's softmax warps
             mbar_init(smem_addr(&tail->o_done[i]), 1);
         }
         mbar_init(smem_addr(&tail->drain), 1);
-        for (int qq = 0; qq < 4; ++qq) {   // every thread of the two warps arrives
-            mbar_init(smem_addr(&tail->pair[qq][0]), 32 * kAttnSplit);
-            mbar_init(smem_addr(&tail->pair[qq][1]), 32 * kAttnSplit);
-            mbar_init(smem_addr(&tail->pair_fin[qq]), 32 * kAttnSplit);
-        }
+        for (int t = 0; t < QT; ++t)
+            for (int qq = 0; qq < 4; ++qq) {   // every thread of the row's warps arrives
+                mbar_init(smem_addr(&tail->pair[t][qq][0]), 32 * kAttnSplit);
+                mbar_init(smem_addr(&tail->pair[t][qq][1]), 32 * kAttnSplit);
+                mbar_init(smem_addr(&tail->pair_fin[t][qq]), 32 * kAttnSplit);
+            }
         tail->abort = 0;
         mbar_init_fence();
     }
@@ -201,11 +219,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol = policy_evict_last();
-            const int qrow = (int)(g * a.s + q0);
             const uint32_t qb = smem_addr(&tail->q_full);
-            mbar_arrive_expect_tx(qb, kAttnTile);
-            tma_load_2d(smem_addr(sq), &maps.q, 0, qrow, qb, pol);
-            tma_load_2d(smem_addr(sq) + kAttnTile / 2, &maps.q, 64, qrow, qb, pol);
+            mbar_arrive_expect_tx(qb, QT * kAttnTile);
+            for (int t = 0; t < QT; ++t) {
+                const int qrow = (int)(g * a.s + q0 + t * kAttnBM);
+                tma_load_2d(smem_addr(sq + (size_t)t * kAttnTile), &maps.q, 0, qrow, qb, pol);
+                tma_load_2d(smem_addr(sq + (size_t)t * kAttnTile) + kAttnTile / 2, &maps.q, 64, qrow,
+                            qb, pol);
+            }
             int issued = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int st = j & 1;
@@ -247,16 +268,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16(kAttnBM, kAttnBN);
             constexpr uint32_t idesc_o = idesc_bf16(kAttnBM, kAttnD) | (1u << 16);  // B MN-major
-            const uint32_t q_s = smem_addr(sq);
             bool ok = mbar_wait(smem_addr(&tail->q_full), 0u, abort, ERR_WAIT_FULL);
-            // S_j = Q K_j^T into buffer j % 2 (after PV_{j-2}, which read P_{j-2} there)
-            auto issue_s = [&](int j) -> bool {
-                const int b = j & 1;
-                if (!mbar_wait(smem_addr(&tail->k_full[b]), (uint32_t)((j >> 1) & 1), abort,
-                               ERR_WAIT_FULL))
+            // S = Q_qt K_j^T into buffer sbuf(qt, j), after the PV that read
+            // the P there; the K tile is freed after its last query tile
+            auto issue_s = [&](int qt, int j) -> bool {
+                const int b = sbuf(qt, j);
+                if (qt == 0 && !mbar_wait(smem_addr(&tail->k_full[j & 1]), (uint32_t)((j >> 1) & 1),
+                                          abort, ERR_WAIT_FULL))
                     return false;
                 tmem_fence_after_sync();
-                const uint32_t k_s = smem_addr(sk + (size_t)b * kAttnTile);
+                const uint32_t q_s = smem_addr(sq + (size_t)qt * kAttnTile);
+                const uint32_t k_s = smem_addr(sk + (size_t)(j & 1) * kAttnTile);
 #pragma unroll
                 for (int kk = 0; kk < kAttnD / 16; ++kk) {
                     // 16 of the 128 head features: chunk kk / 4, 32 bytes each
@@ -264,37 +286,51 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     umma_bf16(tbase + (uint32_t)(b * kAttnBN), sw128_desc(q_s + off),
                               sw128_desc(k_s + off), idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(smem_addr(&tail->k_empty[b]));
+                if (qt == QT - 1) umma_commit(smem_addr(&tail->k_empty[j & 1]));
                 umma_commit(smem_addr(&tail->s_full[b]));
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            if (ok && n_tiles > 1) ok = issue_s(1);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int b = j & 1;
-                if (!mbar_wait(smem_addr(&tail->p_full[b]), (uint32_t)((j >> 1) & 1), abort,
-                               ERR_WAIT_FULL) ||
-                    !mbar_wait(smem_addr(&tail->v_full[b]), (uint32_t)((j >> 1) & 1), abort,
-                               ERR_WAIT_FULL)) {
-                    ok = false;
-                    break;
-                }
+            // O_qt += P V_j, P from buffer sbuf(qt, j); the V tile is freed
+            // after its last query tile
+            auto issue_pv = [&](int qt, int j) -> bool {
+                const int b = sbuf(qt, j);
+                if (!mbar_wait(smem_addr(&tail->p_full[b]), sphase(j), abort, ERR_WAIT_FULL) ||
+                    (qt == 0 && !mbar_wait(smem_addr(&tail->v_full[j & 1]),
+                                           (uint32_t)((j >> 1) & 1), abort, ERR_WAIT_FULL)))
+                    return false;
                 tmem_fence_after_sync();
-                const uint32_t v_s = smem_addr(sv + (size_t)b * kAttnTile);
+                const uint32_t v_s = smem_addr(sv + (size_t)(j & 1) * kAttnTile);
 #pragma unroll
                 for (int kk = 0; kk < kAttnBN / 16; ++kk) {
-                    // keys 16 kk .. 16 kk + 15: P columns 8 kk .. (two bf16 a
-                    // column), V rows 16 kk .. (two 8-row groups of 1024
-                    // bytes, MN-major)
-                    umma_bf16_ts(tbase + 256, tbase + (uint32_t)(b * kAttnBN + 8 * kk),
+                    // keys 16 kk .. 16 kk + 15: P columns (two bf16 a column)
+                    // at the start of the score columns of the slice that
+                    // holds those keys, V rows 16 kk .. (two 8-row groups of
+                    // 1024 bytes, MN-major)
+                    const int slice = (16 * kk) / kAttnCols, kin = 16 * kk - slice * kAttnCols;
+                    umma_bf16_ts(tbase + 256 + (uint32_t)(qt * kAttnD),
+                                 tbase + (uint32_t)(b * kAttnBN + slice * kAttnCols + kin / 2),
                                  sw128_desc_mn(v_s + (uint32_t)kk * 2048, kAttnTile / 2), idesc_o,
                                  (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(smem_addr(&tail->v_empty[b]));
+                if (qt == QT - 1) umma_commit(smem_addr(&tail->v_empty[j & 1]));
                 umma_commit(smem_addr(&tail->o_done[b]));
-                if (j + 2 < n_tiles && !issue_s(j + 2)) {
-                    ok = false;
-                    break;
+                return true;
+            };
+            if constexpr (QT == 1) {
+                if (ok) ok = issue_s(0, 0);
+                if (ok && n_tiles > 1) ok = issue_s(0, 1);
+                for (int j = 0; ok && j < n_tiles; ++j) {
+                    ok = issue_pv(0, j);
+                    if (ok && j + 2 < n_tiles) ok = issue_s(0, j + 2);
+                }
+            } else {
+                if (ok) ok = issue_s(0, 0);
+                if (ok) ok = issue_s(1, 0);
+                for (int j = 0; ok && j < n_tiles; ++j) {
+                    ok = issue_pv(0, j);
+                    if (ok && j + 1 < n_tiles) ok = issue_s(0, j + 1);
+                    if (ok) ok = issue_pv(1, j);
+                    if (ok && j + 1 < n_tiles) ok = issue_s(1, j + 1);
                 }
             }
             // every issued MMA has finished before the CTA tears down
@@ -303,81 +339,87 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             mbar_wait(smem_addr(&tail->drain), 0u, &no_abort, ERR_DRAIN);
         }
     } else {
-        // softmax warps 2 ..: query row 32 (warp % 4) + lane; column slice hf
-        // of the scores (and of O's columns); warps w, w + 4, ... share rows
+        // softmax warps: query tile qt; row 32 (warp % 4) + lane of it; column
+        // slice hf of the scores (and of O's columns); warps w, w + 4, ...
+        // of a tile share rows
+        const int sw = warp - 2;
+        const int qt = sw / kAttnSoftWarps;
         const int q = warp & 3;
-        const int hf = (warp - 2) >> 2;
+        const int hf = (sw % kAttnSoftWarps) >> 2;
         const int row = 32 * q + lane;
         const uint32_t tlane = (uint32_t)(32 * q) << 16;
+        const uint32_t ocol = 256 + (uint32_t)(qt * kAttnD);
         // a bounded wait whose outcome is the same in every lane of the warp,
         // so the warp-collective tensor-memory accesses after it are uniform
         auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
             const bool w = mbar_wait(bar, parity, abort, ERR_WAIT_FULL);
             return __all_sync(0xFFFFFFFFu, w) != 0;
         };
-        float m = -INFINITY, l = 0.f;   // maximum in use (log2 units), this half's sum
+        float m = -INFINITY, l = 0.f;   // maximum in use (log2 units), this slice's sum
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
-            const int b = j & 1;
-            if (!wait_all(smem_addr(&tail->s_full[b]), (uint32_t)((j >> 1) & 1))) {
+            const int b = sbuf(qt, j);
+            const int pb = j & 1;   // parity of the pair exchange
+            if (!wait_all(smem_addr(&tail->s_full[b]), sphase(j))) {
                 ok = false;
                 break;
             }
             tmem_fence_after_sync();
-            uint32_t sc[kAttnCols];
-#pragma unroll
-            for (int c = 0; c < kAttnCols / 32; ++c)
-                tmem_ld32(tbase + tlane + (uint32_t)(b * kAttnBN + kAttnCols * hf + 32 * c), sc + 32 * c);
+            const uint32_t scol = tbase + tlane + (uint32_t)(b * kAttnBN + kAttnCols * hf);
             float mx;
             {
-                // two independent chains of three-input maxima
+                // pass 1: the slice's maximum, 32 scores at a time, two
+                // independent chains of three-input maxima
                 float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < kAttnCols; i += 4) {
-                    m0 = max3f(m0, __uint_as_float(sc[i]), __uint_as_float(sc[i + 1]));
-                    m1 = max3f(m1, __uint_as_float(sc[i + 2]), __uint_as_float(sc[i + 3]));
+                for (int c = 0; c < kAttnCols / 32; ++c) {
+                    uint32_t sc[32];
+                    tmem_ld32(scol + 32 * c, sc);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4) {
+                        m0 = max3f(m0, __uint_as_float(sc[i]), __uint_as_float(sc[i + 1]));
+                        m1 = max3f(m1, __uint_as_float(sc[i + 2]), __uint_as_float(sc[i + 3]));
+                    }
                 }
                 mx = fmaxf(m0, m1);
             }
-            tail->xmax[b][hf][row] = mx;
-            // past this barrier both warps of the row have read their scores,
-            // so either may write P over them
-            tmem_fence_before_sync();
-            mbar_arrive(smem_addr(&tail->pair[q][b]));
-            if (!wait_all(smem_addr(&tail->pair[q][b]), (uint32_t)((j >> 1) & 1))) {
+            tail->xmax[qt][pb][hf][row] = mx;
+            mbar_arrive(smem_addr(&tail->pair[qt][q][pb]));
+            if (!wait_all(smem_addr(&tail->pair[qt][q][pb]), (uint32_t)((j >> 1) & 1))) {
                 ok = false;
                 break;
             }
-            tmem_fence_after_sync();
 #pragma unroll
-            for (int h = 0; h < kAttnSplit; ++h) mx = fmaxf(mx, tail->xmax[b][h][row]);
+            for (int h = 0; h < kAttnSplit; ++h) mx = fmaxf(mx, tail->xmax[qt][pb][h][row]);
             mx *= a.scale_log2;   // the row's maximum
             const bool bump = mx > m + kAttnMaxSlack;   // first tile: m = -inf
             const float alpha = bump ? ex2_approx(m - mx) : 1.0f;   // 0 at the first tile
             if (bump) m = mx;
-            // p = 2^(s * scale - m): the scaling as paired fused multiply-adds,
-            // the sum in two pair lanes
+            // pass 2: p = 2^(s * scale - m), the scaling as paired fused
+            // multiply-adds, the sum in two pair lanes; P as bf16 pairs over
+            // this warp's own score columns (32 scores read, then 16 columns
+            // of P written behind them), so no other warp's scores are touched
             const F2 scale2 = f2(a.scale_log2), negm2 = f2(-m);
             F2 lsum2 = f2(0.f);
-            uint32_t pk[kAttnCols / 2];
 #pragma unroll
-            for (int i = 0; i < kAttnCols / 2; ++i) {
-                const float2 x = halves(fma2(f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])),
-                                             scale2, negm2));
-                const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-                lsum2 = add2(lsum2, f2(p0, p1));
-                pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
+            for (int c = 0; c < kAttnCols / 32; ++c) {
+                uint32_t sc[32], pk[16];
+                tmem_ld32(scol + 32 * c, sc);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 x = halves(fma2(f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])),
+                                                 scale2, negm2));
+                    const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
+                    lsum2 = add2(lsum2, f2(p0, p1));
+                    pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
+                }
+                tmem_st16(scol + 16 * c, pk);
             }
             l = l * alpha + hsum(lsum2);
-            // this slice of the P row: keys kAttnCols hf .. as bf16 pairs,
-            // columns kAttnCols / 2 hf .. of buffer b
-            if constexpr (kAttnCols == 64)
-                tmem_st32(tbase + tlane + (uint32_t)(b * kAttnBN + 32 * hf), pk);
-            else
-                tmem_st16(tbase + tlane + (uint32_t)(b * kAttnBN + 16 * hf), pk);
             if (j > 0 && __any_sync(0xFFFFFFFFu, bump)) {
-                // O of the previous tiles is complete: rescale this half
-                if (!wait_all(smem_addr(&tail->o_done[b ^ 1]), (uint32_t)(((j - 1) >> 1) & 1))) {
+                // O of the previous tiles is complete: rescale this slice
+                const int b_prev = sbuf(qt, j - 1);
+                if (!wait_all(smem_addr(&tail->o_done[b_prev]), sphase(j - 1))) {
                     ok = false;
                     break;
                 }
@@ -385,7 +427,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll 1
                 for (int c = 0; c < kAttnCols / 32; ++c) {
                     uint32_t o[32];
-                    const uint32_t oc = tbase + tlane + 256 + (uint32_t)(kAttnCols * hf + 32 * c);
+                    const uint32_t oc = tbase + tlane + ocol + (uint32_t)(kAttnCols * hf + 32 * c);
                     tmem_ld32(oc, o);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
@@ -397,24 +439,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&tail->p_full[b]));
         }
-        // the row's sum: both halves post theirs (a half that left the loop
-        // early makes the other's bounded wait run out, never hang)
-        tail->xsum[hf][row] = l;
-        mbar_arrive(smem_addr(&tail->pair_fin[q]));
-        if (ok && !wait_all(smem_addr(&tail->pair_fin[q]), 0u)) ok = false;
-        float lt = tail->xsum[0][row];   // the same order, so the same bits, in every warp
+        // the row's sum: every slice posts its own (a warp that left the loop
+        // early makes the others' bounded wait run out, never hang)
+        tail->xsum[qt][hf][row] = l;
+        mbar_arrive(smem_addr(&tail->pair_fin[qt][q]));
+        if (ok && !wait_all(smem_addr(&tail->pair_fin[qt][q]), 0u)) ok = false;
+        float lt = tail->xsum[qt][0][row];   // the same order, so the same bits, in every warp
 #pragma unroll
-        for (int h = 1; h < kAttnSplit; ++h) lt += tail->xsum[h][row];
-        if (ok && wait_all(smem_addr(&tail->o_done[(n_tiles - 1) & 1]),
-                           (uint32_t)(((n_tiles - 1) >> 1) & 1))) {
+        for (int h = 1; h < kAttnSplit; ++h) lt += tail->xsum[qt][h][row];
+        const int b_last = sbuf(qt, n_tiles - 1);
+        if (ok && wait_all(smem_addr(&tail->o_done[b_last]), sphase(n_tiles - 1))) {
             tmem_fence_after_sync();
             const float inv = 1.0f / lt;
+            const long long qrow = q0 + (long long)qt * kAttnBM + row;
             unsigned char* orow = static_cast<unsigned char*>(a.out) +
-                                  ((size_t)g * a.s + q0 + row) * (kAttnD * 2);
+                                  ((size_t)g * a.s + qrow) * (kAttnD * 2);
 #pragma unroll 1
             for (int c = 0; c < kAttnCols / 32; ++c) {
                 uint32_t o[32];
-                tmem_ld32(tbase + tlane + 256 + (uint32_t)(kAttnCols * hf + 32 * c), o);
+                tmem_ld32(tbase + tlane + ocol + (uint32_t)(kAttnCols * hf + 32 * c), o);
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     F2 f[4];
@@ -427,7 +470,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 }
             }
             if (a.lse && hf == 0)
-                a.lse[(size_t)g * a.s + q0 + row] = (m + log2f(lt)) * 0.69314718055994531f;
+                a.lse[(size_t)g * a.s + qrow] = (m + log2f(lt)) * 0.69314718055994531f;
         }
     }
     tmem_fence_before_sync();

@@ -245,9 +245,14 @@ int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const v
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
     a.out = out;
     a.lse = lse;
-    const size_t smem = 1024 + 5 * (size_t)kAttnTile + ((sizeof(AttnTail) + 127) & ~(size_t)127);
+    // two query tiles per CTA when a rank's block holds an even number of
+    // them (both then visit the key tiles in the same ring order)
+    const int qt = per % (2 * kAttnBM) == 0 ? 2 : 1;
+    const size_t smem =
+        1024 + (size_t)(qt + 4) * kAttnTile +
+        (((qt == 2 ? sizeof(AttnTail<2>) : sizeof(AttnTail<1>)) + 127) & ~(size_t)127);
     if (smem > (size_t)dev.smem_optin) return SP_ERR_UNSUPPORTED;
-    const void* kern = (const void*)k_ring_attn;
+    const void* kern = qt == 2 ? (const void*)k_ring_attn<2> : (const void*)k_ring_attn<1>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess) {
         cudaGetLastError();
@@ -257,8 +262,8 @@ int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const v
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3((unsigned)(S / kAttnBM), (unsigned)bh);
-    lc.blockDim = dim3(kAttnThreads);
+    lc.gridDim = dim3((unsigned)(S / (qt * kAttnBM)), (unsigned)bh);
+    lc.blockDim = dim3(attn_threads(qt));
     lc.dynamicSmemBytes = smem;
     lc.stream = static_cast<cudaStream_t>(stream);
     lc.attrs = attr;
