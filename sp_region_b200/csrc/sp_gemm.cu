@@ -75,7 +75,6 @@ int launch_gemm(GemmArgs a, const GemmMaps& maps, const DevInfo& dev, cudaStream
     int S = (int)(((size_t)dev.smem_optin - fixed) / kStage);
     if (S > 16) S = 16;
     a.stages = S;
-    a.tmem_cols = BN <= 128 ? 128 : 256;
     const size_t smem = fixed + (size_t)S * kStage;
     const void* kern = (const void*)k_tp_gemm<BN, EPI>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
@@ -87,7 +86,10 @@ int launch_gemm(GemmArgs a, const GemmMaps& maps, const DevInfo& dev, cudaStream
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((a.N + BN - 1) / BN), (unsigned)((a.M + kGemmBM - 1) / kGemmBM));
+    // persistent: one CTA per SM at most, each looping over tiles
+    const long long tiles = (long long)((a.N + BN - 1) / BN) * ((a.M + kGemmBM - 1) / kGemmBM);
+    if (tiles < 1) return SP_OK;
+    cfg.gridDim = dim3((unsigned)(tiles < dev.sms ? tiles : dev.sms));
     cfg.blockDim = dim3(kGemmThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;

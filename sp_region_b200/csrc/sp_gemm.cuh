@@ -17,15 +17,20 @@
 // column-parallel linear the all-gather becomes the prologue: the A-operand
 // tiles are loaded straight from the t shard buffers.
 //
-// k_tp_gemm: one 128 x BN output tile per CTA.
+// k_tp_gemm: persistent, one CTA per SM; CTA c takes the 128 x BN output
+// tiles c, c + gridDim.x, ... in a grouped order.
 //   warp 0 (one lane)  TMA producer: A and B tiles (K-major, 128-byte
 //                      swizzle, 64 K-elements per stage) into an S-stage ring
+//                      that runs on from one tile into the next
 //   warp 1 (one lane)  MMA issuer: tcgen05.mma kind::f16, M = 128, N = BN,
-//                      K = 16, bf16 x bf16 -> fp32 in tensor memory;
-//                      tcgen05.commit frees each stage and finally signals
-//                      the accumulator
+//                      K = 16, bf16 x bf16 -> fp32 in tensor memory, into one
+//                      of two accumulator stages (2 x BN columns), so the
+//                      epilogue of one tile overlaps the MMAs of the next;
+//                      tcgen05.commit frees each ring stage and signals each
+//                      finished accumulator
 //   warps 2..5         epilogue: tcgen05.ld of the accumulator rows (warp w
-//                      reads lanes 32 (w % 4) .. +32, one row per thread)
+//                      reads lanes 32 (w % 4) .. +32, one row per thread),
+//                      then frees the accumulator stage
 // Every wait is bounded in time; a wait that runs out records an error and
 // the CTA drains what it issued, frees its tensor memory and returns.
 #pragma once
@@ -64,7 +69,6 @@ struct GemmArgs {
     uint32_t off_lo, off_hi;
     uint32_t keys[10][2];
     int dropout;
-    uint32_t tmem_cols;
 };
 
 // Tensor maps (built on the host with cuTensorMapEncodeTiled): B = the
@@ -79,7 +83,9 @@ struct GemmMaps {
 struct GemmTail {
     uint64_t full[16];
     uint64_t empty[16];
-    uint64_t accum;
+    uint64_t acc_full[2];    // an accumulator stage is complete
+    uint64_t acc_empty[2];   // the epilogue has read an accumulator stage
+    uint64_t drain;          // every issued MMA has completed
     uint32_t tmem_base;
     int abort;
 };
@@ -176,12 +182,26 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t r[32])
 
 // ---------------------------------------------------------------------------
 // The kernel.  BN: output features per tile (a multiple of 32, <= 256).
-// EPI 0: row-parallel linear + SP epilogue; EPI 1: plain store.
-// Grid: x = column tiles (ceil(N / BN)), y = row tiles (ceil(M / 128)).
-// Dynamic shared memory: 1024 bytes of alignment slack, stages * (16 KB +
-// BN * 128 B), then GemmTail.  A tile's rows lie in one A map
-// (rows_per_shard is a multiple of 128, or the whole of M).
+// EPI 0: row-parallel linear + SP epilogue; EPI 1: plain store.  Persistent:
+// grid = min(tiles, SMs); CTA c takes tiles c, c + gridDim.x, ...  Dynamic
+// shared memory: 1024 bytes of alignment slack, stages * (16 KB + BN * 128 B),
+// then GemmTail.  A tile's rows lie in one A map (rows_per_shard is a
+// multiple of 128, or the whole of M).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void gemm_tile_coords(long long tile, int Mt, int Nt, int* tm, int* tn)
+{
+    // tile order: the CTAs that run at the same time cover a block of
+    // kGemmGroup row tiles by a few column tiles, so the A and B slabs they
+    // stream (in near lock-step along K) are read from HBM about once and
+    // shared through L2
+    const long long per_group = (long long)kGemmGroup * Nt;
+    const int grp = (int)(tile / per_group);
+    const int in_grp = (int)(tile - (long long)grp * per_group);
+    const int rows_in_grp = min(kGemmGroup, Mt - grp * kGemmGroup);
+    *tm = grp * kGemmGroup + in_grp % rows_in_grp;
+    *tn = in_grp / rows_in_grp;
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_tp_gemm(const __grid_constant__ GemmArgs a, const __grid_constant__ GemmMaps maps)
@@ -189,6 +209,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     constexpr uint32_t kABytes = kGemmBM * kGemmBK * 2;   // 16 KB
     constexpr uint32_t kBBytes = BN * kGemmBK * 2;
     constexpr uint32_t kStage = kABytes + kBBytes;
+    constexpr uint32_t kAccCols = BN <= 128 ? 128 : 256;   // one accumulator stage
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     // the stages need 1024-byte alignment (128-byte swizzle atoms)
     unsigned char* gsm = reinterpret_cast<unsigned char*>(
@@ -197,25 +218,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     GemmTail* tail = reinterpret_cast<GemmTail*>(gsm + (size_t)S * kStage);
     volatile int* abort = &tail->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // tile order: the CTAs that run at the same time cover a block of
-    // kGemmGroup row tiles by a few column tiles, so the A and B slabs they
-    // stream (in near lock-step along K) are each read from HBM once and
-    // shared through L2
-    const int ncol = gridDim.x, nrow = gridDim.y;
-    const long long lin = (long long)blockIdx.y * ncol + blockIdx.x;
-    const long long per_group = (long long)kGemmGroup * ncol;
-    const int grp = (int)(lin / per_group);
-    const int in_grp = (int)(lin - (long long)grp * per_group);
-    const int rows_in_grp = min(kGemmGroup, nrow - grp * kGemmGroup);
-    const int tile_row = grp * kGemmGroup + in_grp % rows_in_grp;
-    const int tile_col = in_grp / rows_in_grp;
-    const int n0 = tile_col * BN;
-    const long long m0 = (long long)tile_row * kGemmBM;
+    const int Mt = (int)((a.M + kGemmBM - 1) / kGemmBM);
+    const int Nt = (a.N + BN - 1) / BN;
+    const long long T = (long long)Mt * Nt;
     const int KB = (a.K + kGemmBK - 1) / kGemmBK;
-    // A rows of this tile come from one shard (rows_per_shard % 128 == 0)
-    const int map_id = (int)(m0 / a.rows_per_shard);
-    const int a_row = (int)(m0 - (long long)map_id * a.rows_per_shard);
-    const CUtensorMap* amap = &maps.a[map_id];
     const CUtensorMap* bmap = &maps.b;
 
     if (threadIdx.x == 0) {
@@ -223,18 +229,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(smem_addr(&tail->full[s]), 1);
             mbar_init(smem_addr(&tail->empty[s]), 1);
         }
-        mbar_init(smem_addr(&tail->accum), 1);
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(smem_addr(&tail->acc_full[q]), 1);
+            mbar_init(smem_addr(&tail->acc_empty[q]), 4);   // the 4 epilogue warps
+        }
+        mbar_init(smem_addr(&tail->drain), 1);
         tail->abort = 0;
         mbar_init_fence();
     }
     if (warp == 1) {
-        tmem_alloc(smem_addr(&tail->tmem_base), a.tmem_cols);
+        tmem_alloc(smem_addr(&tail->tmem_base), 2 * kAccCols);
         tmem_fence_before_sync();
     }
-    if (threadIdx.x == 0) {
-        tma_prefetch_desc(bmap);
-        tma_prefetch_desc(amap);
-    }
+    if (threadIdx.x == 0) tma_prefetch_desc(bmap);
     __syncthreads();
     tmem_fence_after_sync();
     const uint32_t tbase = tail->tmem_base;
@@ -243,27 +250,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // producer: A (x rows) read by every column tile, kept in L2;
-            // B (weight rows) likewise shared by every row tile
+            // producer: A (x rows) is read by every column tile and B (weight
+            // rows) by every row tile: keep both in L2
             const uint64_t pol = policy_evict_last();
-            int issued = 0;
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % S;
-                if (kb >= S &&
-                    !mbar_wait(smem_addr(&tail->empty[s]), (uint32_t)(((kb / S) - 1) & 1), abort,
-                               ERR_WAIT_EMPTY))
-                    break;
-                const uint32_t bar = smem_addr(&tail->full[s]);
-                mbar_arrive_expect_tx(bar, kStage);
-                const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
-                tma_load_2d(sa, amap, kb * kGemmBK, a_row, bar, pol);
-                tma_load_2d(sa + kABytes, bmap, kb * kGemmBK, n0, bar, pol);
-                ++issued;
+            long long g = 0;   // k-steps issued over all tiles
+            bool ok = true;
+            for (long long tile = blockIdx.x; ok && tile < T; tile += gridDim.x) {
+                int tm, tn;
+                gemm_tile_coords(tile, Mt, Nt, &tm, &tn);
+                const long long m0 = (long long)tm * kGemmBM;
+                const int map_id = (int)(m0 / a.rows_per_shard);
+                const int a_row = (int)(m0 - (long long)map_id * a.rows_per_shard);
+                const CUtensorMap* amap = &maps.a[map_id];
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = (int)(g % S);
+                    if (g >= S && !mbar_wait(smem_addr(&tail->empty[s]),
+                                             (uint32_t)(((g / S) - 1) & 1), abort, ERR_WAIT_EMPTY)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar = smem_addr(&tail->full[s]);
+                    mbar_arrive_expect_tx(bar, kStage);
+                    const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
+                    tma_load_2d(sa, amap, kb * kGemmBK, a_row, bar, pol);
+                    tma_load_2d(sa + kABytes, bmap, kb * kGemmBK, tn * BN, bar, pol);
+                }
             }
             if (*abort) {
                 // let every issued copy land before the CTA's memory goes away
-                const int first = issued > S ? issued - S : 0;
-                for (int i = first; i < issued; ++i) {
+                const long long first = g > S ? g - S : 0;
+                for (long long i = first; i < g; ++i) {
                     volatile int no_abort = 0;
                     if (!mbar_wait(smem_addr(&tail->full[i % S]), (uint32_t)((i / S) & 1),
                                    &no_abort, ERR_DRAIN))
@@ -274,94 +290,122 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(kGemmBM, BN);
+            long long g = 0;
             bool ok = true;
-            int kb = 0;
-            for (; kb < KB; ++kb) {
-                const int s = kb % S;
-                if (!mbar_wait(smem_addr(&tail->full[s]), (uint32_t)((kb / S) & 1), abort,
-                               ERR_WAIT_FULL)) {
-                    ok = false;
+            long long it = 0;
+            for (long long tile = blockIdx.x; ok && tile < T; tile += gridDim.x, ++it) {
+                const int as = (int)(it & 1);
+                const uint32_t use = (uint32_t)(it >> 1);
+                // the epilogue has read this accumulator stage's previous tile
+                // (a fresh barrier passes parity 1 at once)
+                if (!mbar_wait(smem_addr(&tail->acc_empty[as]), (use & 1u) ^ 1u, abort,
+                               ERR_WAIT_EMPTY))
                     break;
-                }
                 tmem_fence_after_sync();
-                const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
-                const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + kABytes);
+                const uint32_t tacc = tbase + (uint32_t)as * kAccCols;
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = (int)(g % S);
+                    if (!mbar_wait(smem_addr(&tail->full[s]), (uint32_t)((g / S) & 1), abort,
+                                   ERR_WAIT_FULL)) {
+                        ok = false;
+                        break;
+                    }
+                    tmem_fence_after_sync();
+                    const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
+                    const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sa + kABytes);
 #pragma unroll
-                for (int k = 0; k < kGemmBK / 16; ++k)
-                    // +32 bytes of K per step: +2 in the start-address field
-                    umma_bf16(tbase, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
-                umma_commit(smem_addr(&tail->empty[s]));   // stage s may be refilled
+                    for (int k = 0; k < kGemmBK / 16; ++k)
+                        // +32 bytes of K per step: +2 in the start-address field
+                        umma_bf16(tacc, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(smem_addr(&tail->empty[s]));   // stage s may be refilled
+                }
+                if (!ok) break;
+                umma_commit(smem_addr(&tail->acc_full[as]));   // the accumulator is complete
             }
-            // the accumulator is complete (or, on abort, every issued MMA
-            // has finished reading shared memory)
-            umma_commit(smem_addr(&tail->accum));
-            (void)ok;
+            // every issued MMA has finished reading shared memory and writing
+            // tensor memory
+            umma_commit(smem_addr(&tail->drain));
+            volatile int no_abort = 0;
+            mbar_wait(smem_addr(&tail->drain), 0u, &no_abort, ERR_DRAIN);
         }
     } else {
         // epilogue warps 2..5: warp w owns accumulator lanes 32 (w % 4) ..
         const int q = warp & 3;
-        const long long m = m0 + 32 * q + lane;   // output row of this thread
-        const bool done = mbar_wait(smem_addr(&tail->accum), 0u, abort, ERR_WAIT_FULL);
-        tmem_fence_after_sync();
-        const bool row_ok = done && !*abort && m < a.M;
-        const uint32_t trow = tbase + ((uint32_t)(32 * q) << 16);
+        long long it = 0;
+        for (long long tile = blockIdx.x; tile < T; tile += gridDim.x, ++it) {
+            int tm, tn;
+            gemm_tile_coords(tile, Mt, Nt, &tm, &tn);
+            const int as = (int)(it & 1);
+            const uint32_t use = (uint32_t)(it >> 1);
+            const long long m = (long long)tm * kGemmBM + 32 * q + lane;   // output row of this thread
+            const int n0 = tn * BN;
+            if (!mbar_wait(smem_addr(&tail->acc_full[as]), use & 1u, abort, ERR_WAIT_FULL)) break;
+            tmem_fence_after_sync();
+            const bool row_ok = m < a.M;
+            const uint32_t trow = tbase + ((uint32_t)(32 * q) << 16) + (uint32_t)as * kAccCols;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(trow + (uint32_t)c0, r);   // warp-wide, outside per-thread branches
-            if (!row_ok) continue;
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                if (n0 + c0 >= a.N) break;          // warp-uniform
+                uint32_t r[32];
+                tmem_ld32(trow + (uint32_t)c0, r);   // warp-wide, outside per-thread branches
+                if (!row_ok) continue;
 #pragma unroll
-            for (int v8 = 0; v8 < 4; ++v8) {
-                const int col = n0 + c0 + 8 * v8;   // first feature of this 8-vector
-                if (col >= a.N) continue;           // N % 8 == 0: vectors are whole
-                F2 y[4];
+                for (int v8 = 0; v8 < 4; ++v8) {
+                    const int col = n0 + c0 + 8 * v8;   // first feature of this 8-vector
+                    if (col >= a.N) continue;           // N % 8 == 0: vectors are whole
+                    F2 y[4];
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
-                    y[p] = f2(__uint_as_float(r[8 * v8 + 2 * p]),
-                              __uint_as_float(r[8 * v8 + 2 * p + 1]));
-                if (EPI == 0) {
-                    const long long n = a.row0 + m;   // global token row
-                    if (a.bias) {
-                        F2 b[4];
-                        IO<__nv_bfloat16>::unpack2(load_vec<__nv_bfloat16>(a.bias, col / 8), b);
+                    for (int p = 0; p < 4; ++p)
+                        y[p] = f2(__uint_as_float(r[8 * v8 + 2 * p]),
+                                  __uint_as_float(r[8 * v8 + 2 * p + 1]));
+                    if (EPI == 0) {
+                        const long long n = a.row0 + m;   // global token row
+                        if (a.bias) {
+                            F2 b[4];
+                            IO<__nv_bfloat16>::unpack2(load_vec<__nv_bfloat16>(a.bias, col / 8), b);
 #pragma unroll
-                        for (int p = 0; p < 4; ++p) y[p] = add2(y[p], b[p]);
+                            for (int p = 0; p < 4; ++p) y[p] = add2(y[p], b[p]);
+                        }
+                        uint32_t kb8 = 0xFFu;
+                        if (a.dropout) {
+                            kb8 = keep_bits8((uint32_t)(col / 8), (uint32_t)n, a.off_lo, a.off_hi,
+                                             a.keys, a.thr);
+                            const F2 sc2 = f2(a.scale);
+#pragma unroll
+                            for (int p = 0; p < 4; ++p)
+                                y[p] = keep2(mul2(y[p], sc2), (kb8 >> (2 * p)) & 1u,
+                                             (kb8 >> (2 * p + 1)) & 1u);
+                        }
+                        if (a.mask) a.mask[(size_t)m * a.mask_row_bytes + col / 8] = (uint8_t)kb8;
+                        F2 rs[4];
+                        const unsigned char* rrow =
+                            static_cast<const unsigned char*>(a.residual) + (size_t)m * a.N * 2;
+                        IO<__nv_bfloat16>::unpack2(load_vec<__nv_bfloat16>(rrow, col / 8), rs);
+#pragma unroll
+                        for (int p = 0; p < 4; ++p) y[p] = add2(rs[p], y[p]);
                     }
-                    uint32_t kb8 = 0xFFu;
-                    if (a.dropout) {
-                        kb8 = keep_bits8((uint32_t)(col / 8), (uint32_t)n, a.off_lo, a.off_hi,
-                                         a.keys, a.thr);
-                        const F2 sc2 = f2(a.scale);
-#pragma unroll
-                        for (int p = 0; p < 4; ++p)
-                            y[p] = keep2(mul2(y[p], sc2), (kb8 >> (2 * p)) & 1u,
-                                         (kb8 >> (2 * p + 1)) & 1u);
-                    }
-                    if (a.mask) a.mask[(size_t)m * a.mask_row_bytes + col / 8] = (uint8_t)kb8;
-                    F2 rs[4];
-                    const unsigned char* rrow =
-                        static_cast<const unsigned char*>(a.residual) + (size_t)m * a.N * 2;
-                    IO<__nv_bfloat16>::unpack2(load_vec<__nv_bfloat16>(rrow, col / 8), rs);
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) y[p] = add2(rs[p], y[p]);
+                    unsigned char* orow = static_cast<unsigned char*>(a.out) + (size_t)m * a.N * 2;
+                    store_vec<__nv_bfloat16>(orow, col / 8, IO<__nv_bfloat16>::pack2v(y));
                 }
-                unsigned char* orow = static_cast<unsigned char*>(a.out) + (size_t)m * a.N * 2;
-                store_vec<__nv_bfloat16>(orow, col / 8, IO<__nv_bfloat16>::pack2v(y));
+                if (EPI == 0 && a.mask && n0 + c0 + 32 >= a.N) {
+                    // the row's last features: zero the mask's padding bytes
+                    for (int pb = a.N / 8; pb < a.mask_row_bytes; ++pb)
+                        a.mask[(size_t)m * a.mask_row_bytes + pb] = 0;
+                }
             }
-            if (EPI == 0 && a.mask && n0 + c0 + 32 >= a.N && n0 + c0 < a.N) {
-                // the row's last features: zero the mask's padding bytes
-                for (int pb = a.N / 8; pb < a.mask_row_bytes; ++pb)
-                    a.mask[(size_t)m * a.mask_row_bytes + pb] = 0;
-            }
+            // this warp's reads of the stage are done: the MMA may refill it
+            tmem_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&tail->acc_empty[as]));
         }
     }
-    // every tensor-memory read is done before warp 1 frees the columns
+    // every tensor-memory access is done before warp 1 frees the columns
     tmem_fence_before_sync();
     __syncthreads();
     if (warp == 1) {
         __syncwarp();
         tmem_fence_after_sync();
-        tmem_dealloc(tbase, a.tmem_cols);
+        tmem_dealloc(tbase, 2 * kAccCols);
     }
 }
 
