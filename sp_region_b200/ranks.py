@@ -119,7 +119,7 @@ def peer_buffers(tensor: torch.Tensor, group=None) -> List[torch.Tensor]:
     with torch's symmetric memory (torch.distributed._symmetric_memory.empty):
     this rank's own tensor and every peer's mapped into this process.  The
     kernels read and write peers' buffers through these addresses with plain
-    loads, stores and non-multicast bulk copies."""
+    loads, stores and bulk copies from one source to one destination."""
     import torch.distributed._symmetric_memory as symm_mem
     h = symm_mem.rendezvous(tensor, group or dist.group.WORLD)
     return [tensor if r == h.rank else
