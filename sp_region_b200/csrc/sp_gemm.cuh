@@ -19,9 +19,14 @@
 //
 // k_tp_gemm: persistent, one CTA per SM; CTA c takes the 128 x BN output
 // tiles c, c + gridDim.x, ... in a grouped order.
-//   warp 0 (one lane)  TMA producer: A and B tiles (K-major, 128-byte
-//                      swizzle, 64 K-elements per stage) into an S-stage ring
-//                      that runs on from one tile into the next
+//   warps 0 and 6 (one lane each)  TMA producers: warp 0 the A tile, warp 6
+//                      the B tile of every stage (K-major, 128-byte swizzle,
+//                      64 K-elements per stage) of an S-stage ring that runs on
+//                      from one tile into the next.  Warp 0 arms each stage's
+//                      full barrier for both copies.  Two issuing threads:
+//                      the ring's refill rate is set by how fast requests are
+//                      issued, not by their bytes (one thread issuing both
+//                      copies ran 12-14 % slower)
 //   warp 1 (one lane)  MMA issuer: tcgen05.mma kind::f16, M = 128, N = BN,
 //                      K = 16, bf16 x bf16 -> fp32 in tensor memory, into one
 //                      of two accumulator stages (2 x BN columns), so the
@@ -44,7 +49,7 @@ namespace spk {
 
 constexpr int kGemmBM = 128;           // rows per tile (tcgen05 M)
 constexpr int kGemmBK = 64;            // K elements per stage: one 128-byte row
-constexpr int kGemmThreads = 192;      // producer, MMA, 4 epilogue warps
+constexpr int kGemmThreads = 224;      // A producer, MMA, 4 epilogue warps, B producer
 constexpr int kGemmMaxShards = 16;     // A tensor maps (sequence shards)
 constexpr int kGemmGroup = 16;         // row tiles per group of the tile order
 
@@ -202,6 +207,21 @@ __device__ __forceinline__ void gemm_tile_coords(long long tile, int Mt, int Nt,
     *tn = in_grp / rows_in_grp;
 }
 
+// After an abort: wait (bounded) for the last S of the `issued` stages a
+// producer filled, so no copy lands in shared memory after the CTA is gone.
+// A stage whose barrier was never armed (the other producer stopped first)
+// runs out of its wait; by then that copy has long landed.
+__device__ __forceinline__ void gemm_drain(GemmTail* tail, long long issued, int S)
+{
+    const long long first = issued > S ? issued - S : 0;
+    for (long long i = first; i < issued; ++i) {
+        volatile int no_abort = 0;
+        if (!mbar_wait(smem_addr(&tail->full[i % S]), (uint32_t)((i / S) & 1), &no_abort,
+                       ERR_DRAIN))
+            break;
+    }
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_tp_gemm(const __grid_constant__ GemmArgs a, const __grid_constant__ GemmMaps maps)
@@ -269,23 +289,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ok = false;
                         break;
                     }
+                    // armed for both copies; the B producer's may land first
                     const uint32_t bar = smem_addr(&tail->full[s]);
                     mbar_arrive_expect_tx(bar, kStage);
-                    const uint32_t sa = smem_addr(gsm + (size_t)s * kStage);
-                    tma_load_2d(sa, amap, kb * kGemmBK, a_row, bar, pol);
-                    tma_load_2d(sa + kABytes, bmap, kb * kGemmBK, tn * BN, bar, pol);
+                    tma_load_2d(smem_addr(gsm + (size_t)s * kStage), amap, kb * kGemmBK, a_row,
+                                bar, pol);
                 }
             }
-            if (*abort) {
-                // let every issued copy land before the CTA's memory goes away
-                const long long first = g > S ? g - S : 0;
-                for (long long i = first; i < g; ++i) {
-                    volatile int no_abort = 0;
-                    if (!mbar_wait(smem_addr(&tail->full[i % S]), (uint32_t)((i / S) & 1),
-                                   &no_abort, ERR_DRAIN))
+            if (*abort) gemm_drain(tail, g, S);
+        }
+    } else if (warp == 6) {
+        if (lane == 0) {
+            // B producer: the weight tile of every stage, completing on the
+            // full barrier warp 0 arms
+            const uint64_t pol = policy_evict_last();
+            long long g = 0;
+            bool ok = true;
+            for (long long tile = blockIdx.x; ok && tile < T; tile += gridDim.x) {
+                int tm, tn;
+                gemm_tile_coords(tile, Mt, Nt, &tm, &tn);
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = (int)(g % S);
+                    if (g >= S && !mbar_wait(smem_addr(&tail->empty[s]),
+                                             (uint32_t)(((g / S) - 1) & 1), abort, ERR_WAIT_EMPTY)) {
+                        ok = false;
                         break;
+                    }
+                    tma_load_2d(smem_addr(gsm + (size_t)s * kStage) + kABytes, bmap, kb * kGemmBK,
+                                tn * BN, smem_addr(&tail->full[s]), pol);
                 }
             }
+            if (*abort) gemm_drain(tail, g, S);
         }
     } else if (warp == 1) {
         if (lane == 0) {
