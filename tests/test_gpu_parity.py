@@ -191,6 +191,9 @@ BWD_CASES = {
     "bf16_rms_h8192_p0_nomask": dict(base="C3", s=152, b=1, nomask=True),
     "bf16_ln_h1000_ragged": dict(base="C2", s=111, b=3, h=1000, t=3),
     "bf16_general_h100": dict(base="C2", s=40, b=2, h=100, t=4, drnext=True),
+    # h % 4 != 0: the column sums take their one-column-per-lane form
+    "bf16_general_h90": dict(base="C2", s=48, b=2, h=90, t=3, drnext=True),
+    "f32_general_h30": dict(base="C1", s=30, b=1, h=30, t=3),
     "f32_ln_h512": dict(base="C2", s=64, b=3, h=512, t=2, dtype="f32"),
     "f32_general_worked": dict(base="C1", drnext=True),
     "bf16_ln_no_dbias_dbeta": dict(base="C4", s=64, b=1, h=2048,
