@@ -23,10 +23,10 @@
 //                      the B tile of every stage (K-major, 128-byte swizzle,
 //                      64 K-elements per stage) of an S-stage ring that runs on
 //                      from one tile into the next.  Warp 0 arms each stage's
-//                      full barrier for both copies.  Two issuing threads:
-//                      the ring's refill rate is set by how fast requests are
-//                      issued, not by their bytes (one thread issuing both
-//                      copies ran 12-14 % slower)
+//                      full barrier for both copies.  The stage index and
+//                      parity of every ring step are kept as counters: a 64-bit
+//                      division per step on these threads and on the MMA
+//                      thread cost 9-14 % of the throughput
 //   warp 1 (one lane)  MMA issuer: tcgen05.mma kind::f16, M = 128, N = BN,
 //                      K = 16, bf16 x bf16 -> fp32 in tensor memory, into one
 //                      of two accumulator stages (2 x BN columns), so the
@@ -261,7 +261,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_alloc(smem_addr(&tail->tmem_base), 2 * kAccCols);
         tmem_fence_before_sync();
     }
-    if (threadIdx.x == 0) tma_prefetch_desc(bmap);
+    if (warp == 0 && lane <= a.nmaps) {
+        // the descriptors into the TMA unit's cache: lane 0 the weight's,
+        // lane i the map of shard i - 1
+        tma_prefetch_desc(lane == 0 ? bmap : &maps.a[lane - 1]);
+    }
     __syncthreads();
     tmem_fence_after_sync();
     const uint32_t tbase = tail->tmem_base;
@@ -274,6 +278,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // rows) by every row tile: keep both in L2
             const uint64_t pol = policy_evict_last();
             long long g = 0;   // k-steps issued over all tiles
+            int s = 0;         // stage of step g: g % S
+            uint32_t ph = 0;   // (g / S) & 1; counters, not divisions, on this path
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < T; tile += gridDim.x) {
                 int tm, tn;
@@ -283,9 +289,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int a_row = (int)(m0 - (long long)map_id * a.rows_per_shard);
                 const CUtensorMap* amap = &maps.a[map_id];
                 for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = (int)(g % S);
-                    if (g >= S && !mbar_wait(smem_addr(&tail->empty[s]),
-                                             (uint32_t)(((g / S) - 1) & 1), abort, ERR_WAIT_EMPTY)) {
+                    // the stage's previous fill (step g - S) has been consumed
+                    if (g >= S && !mbar_wait(smem_addr(&tail->empty[s]), ph ^ 1u, abort,
+                                             ERR_WAIT_EMPTY)) {
                         ok = false;
                         break;
                     }
@@ -294,6 +300,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     mbar_arrive_expect_tx(bar, kStage);
                     tma_load_2d(smem_addr(gsm + (size_t)s * kStage), amap, kb * kGemmBK, a_row,
                                 bar, pol);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             if (*abort) gemm_drain(tail, g, S);
@@ -304,19 +314,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // full barrier warp 0 arms
             const uint64_t pol = policy_evict_last();
             long long g = 0;
+            int s = 0;
+            uint32_t ph = 0;
             bool ok = true;
             for (long long tile = blockIdx.x; ok && tile < T; tile += gridDim.x) {
                 int tm, tn;
                 gemm_tile_coords(tile, Mt, Nt, &tm, &tn);
                 for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = (int)(g % S);
-                    if (g >= S && !mbar_wait(smem_addr(&tail->empty[s]),
-                                             (uint32_t)(((g / S) - 1) & 1), abort, ERR_WAIT_EMPTY)) {
+                    if (g >= S && !mbar_wait(smem_addr(&tail->empty[s]), ph ^ 1u, abort,
+                                             ERR_WAIT_EMPTY)) {
                         ok = false;
                         break;
                     }
                     tma_load_2d(smem_addr(gsm + (size_t)s * kStage) + kABytes, bmap, kb * kGemmBK,
                                 tn * BN, smem_addr(&tail->full[s]), pol);
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             if (*abort) gemm_drain(tail, g, S);
@@ -324,7 +339,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_bf16(kGemmBM, BN);
-            long long g = 0;
+            int s = 0;         // stage of the next k-step
+            uint32_t ph = 0;   // parity of its fill
             bool ok = true;
             long long it = 0;
             for (long long tile = blockIdx.x; ok && tile < T; tile += gridDim.x, ++it) {
@@ -337,10 +353,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     break;
                 tmem_fence_after_sync();
                 const uint32_t tacc = tbase + (uint32_t)as * kAccCols;
-                for (int kb = 0; kb < KB; ++kb, ++g) {
-                    const int s = (int)(g % S);
-                    if (!mbar_wait(smem_addr(&tail->full[s]), (uint32_t)((g / S) & 1), abort,
-                                   ERR_WAIT_FULL)) {
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(smem_addr(&tail->full[s]), ph, abort, ERR_WAIT_FULL)) {
                         ok = false;
                         break;
                     }
@@ -352,6 +366,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         // +32 bytes of K per step: +2 in the start-address field
                         umma_bf16(tacc, ad + 2 * k, bd + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
                     umma_commit(smem_addr(&tail->empty[s]));   // stage s may be refilled
+                    if (++s == S) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 umma_commit(smem_addr(&tail->acc_full[as]));   // the accumulator is complete
