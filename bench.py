@@ -667,17 +667,22 @@ def time_ring_attention(args, sp, torch, dev):
     lse = torch.empty((b, heads, s), dtype=torch.float32, device=dev)
     cfg = sp.make_cfg(s, b, heads * d, t, dtype="bf16")
     stream = torch.cuda.current_stream(dev)
-    ms = time_launches(torch, stream, lambda: sp.sp_ring_attention_fwd(
-        cfg, heads, d ** -0.5, q, k, v, out, lse, stream=stream), 3, 3)
+    # the workspace call: the units of the last, partly filled round of SMs
+    # run split over ranges of ring steps (k_attn_merge combines them)
+    nbytes = sp.sp_ring_attention_workspace_bytes(cfg, heads, dev.index)
+    ws = torch.empty(nbytes // 4 + 4, device=dev) if nbytes else None
+    ms = time_launches(torch, stream, lambda: sp.sp_ring_attention_fwd_ws(
+        cfg, heads, d ** -0.5, q, k, v, out, lse, ws, stream=stream), 3, 3)
     assert sp.sp_device_error(dev.index) == 0, "device-side wait timed out"
     flops = 4.0 * s * s * d * heads * b
     tf = flops / (ms * 1e-3) / 1e12
-    del q, k, v, out, lse
+    del q, k, v, out, lse, ws
     gc.collect()
     torch.cuda.empty_cache()
     return {"workload": (f"C5 attention core: s={s}, t={t} ranks of {s // t} tokens, "
                          f"head dim {d}, {heads} heads, b={b}, bf16, full attention"),
-            "kernel": "k_ring_attn", "avg_ms": round(ms, 3), "tflops": round(tf, 1),
+            "kernel": "k_ring_attn + k_attn_merge", "workspace_bytes": nbytes,
+            "avg_ms": round(ms, 3), "tflops": round(tf, 1),
             "frac": round(tf / peak, 4), "peak_tflops": peak, "peak_source": peak_src,
             "flops_per_launch": flops}
 

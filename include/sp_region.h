@@ -407,6 +407,41 @@ int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const v
                           const void* k, const void* v, void* out, float* lse,
                           void* stream);
 
+/*
+ * The same ring attention, with scratch for balancing the last round of work.
+ *
+ * Same definition, arguments and requirements as sp_ring_attention_fwd, plus
+ * a workspace.  One CTA takes a unit (one or two 128-query tiles of one
+ * head) through every ring step, and the GPU runs one CTA per SM.  When the
+ * units do not fill the last round of SMs, the call cuts each unit of that
+ * round into up to 8 contiguous ranges of ring steps (at least 4 key tiles
+ * each). Each range keeps its own online-softmax state (m_i, l_i, o_i), as a
+ * rank does between ring steps. A second kernel then combines the ranges
+ * of every such query in range order:
+ *   m = max m_i,  l = sum exp(m_i - m) l_i,  out = sum exp(m_i - m) o_i / l
+ * which is the online-softmax update of the page applied once per range.
+ * The order of the additions differs from the unsplit call, so results agree
+ * with it to rounding, not bit for bit; repeated calls with the same shape on
+ * the same GPU give the same bits.
+ *
+ *   workspace        device scratch of at least
+ *                    sp_ring_attention_workspace_bytes() bytes, 16-byte
+ *                    aligned, no initial contents; may be NULL when that
+ *                    size is 0.  Calls that overlap on the GPU must not
+ *                    share a workspace.
+ * SP_ERR_INVALID_ARG when the workspace is missing or too small.
+ */
+int sp_ring_attention_fwd_ws(const sp_cfg* cfg, int32_t heads, float scale, const void* q,
+                             const void* k, const void* v, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device scratch sp_ring_attention_fwd_ws needs for cfg and heads
+ * on CUDA device `device` (its SM count sets the split): 0 when the units
+ * fill whole rounds.  Host-only.  The errors of sp_ring_attention_fwd's
+ * shape checks; SP_ERR_INVALID_ARG for bytes == NULL. */
+int sp_ring_attention_workspace_bytes(const sp_cfg* cfg, int32_t heads, int32_t device,
+                                      size_t* bytes);
+
 /* Bytes of device scratch sp_rs_norm_dropout_bwd needs for cfg on CUDA
  * device `device`: the slices of 3*h fp32 parameter-gradient partial sums
  * that the kernel the call picks writes, for 16-byte aligned pointers or for

@@ -36,7 +36,8 @@ EXPORTS = ("sp_rs_bias_dropout_add_norm_fwd", "sp_all_gather",
            "sp_rs_norm_dropout_bwd_noalloc", "sp_norm_all_gather_fwd",
            "sp_rowpar_linear_rs_fwd", "sp_linear_rs_bias_dropout_add_norm_fwd",
            "sp_ag_colpar_linear_fwd", "sp_rs_norm_dropout_bwd_ag",
-           "sp_ring_attention_fwd")
+           "sp_ring_attention_fwd", "sp_ring_attention_fwd_ws",
+           "sp_ring_attention_workspace_bytes")
 
 
 class SPError(RuntimeError):
@@ -93,6 +94,11 @@ def _load() -> ctypes.CDLL:
     lib.sp_ag_colpar_linear_fwd.argtypes = [cfgp, i64, vp, vp, vp, vp]
     lib.sp_ring_attention_fwd.argtypes = [cfgp, i32, ctypes.c_float, vp, vp, vp,
                                           vp, vp, vp]
+    lib.sp_ring_attention_fwd_ws.argtypes = [cfgp, i32, ctypes.c_float, vp, vp,
+                                             vp, vp, vp, vp, ctypes.c_size_t,
+                                             vp]
+    lib.sp_ring_attention_workspace_bytes.argtypes = [
+        cfgp, i32, i32, ctypes.POINTER(ctypes.c_size_t)]
     for f in EXPORTS:
         getattr(lib, f).restype = (ctypes.c_char_p if f == "sp_status_string"
                                    else ctypes.c_int)
@@ -281,6 +287,30 @@ def sp_ring_attention_fwd(cfg: sp_cfg, heads: int, scale: float, q, k, v, out,
            _lib.sp_ring_attention_fwd(ctypes.byref(cfg), heads, scale, _p(q),
                                       _p(k), _p(v), _p(out), _p(lse),
                                       _stream(stream, out)))
+
+
+def sp_ring_attention_workspace_bytes(cfg: sp_cfg, heads: int,
+                                      device=None) -> int:
+    dev = torch.cuda.current_device() if device is None else int(device)
+    n = ctypes.c_size_t(0)
+    _check("sp_ring_attention_workspace_bytes",
+           _lib.sp_ring_attention_workspace_bytes(ctypes.byref(cfg), heads, dev,
+                                                  ctypes.byref(n)))
+    return int(n.value)
+
+
+def sp_ring_attention_fwd_ws(cfg: sp_cfg, heads: int, scale: float, q, k, v,
+                             out, lse=None, workspace=None,
+                             stream=None) -> None:
+    """Ring attention with the last round of units split over the SMs
+    (workspace: sp_ring_attention_workspace_bytes bytes, or None when 0)."""
+    nbytes = 0 if workspace is None else \
+        workspace.numel() * workspace.element_size()
+    _check("sp_ring_attention_fwd_ws",
+           _lib.sp_ring_attention_fwd_ws(ctypes.byref(cfg), heads, scale,
+                                         _p(q), _p(k), _p(v), _p(out), _p(lse),
+                                         _p(workspace), nbytes,
+                                         _stream(stream, out)))
 
 
 def sp_activation_bytes(s: int, b: int, h: int, a: int, t: int, mode: int,

@@ -67,6 +67,15 @@ struct AttnArgs {
     float scale_log2;         // score scale * log2(e)
     void* out;                // [bh][s][128] bf16
     float* lse;               // [bh][s] natural-log sum of exp(scores), or NULL
+    // work items (one CTA each): items [0, full_units) are whole units (QT
+    // query tiles of one head, every ring step); each later unit is split into
+    // `split` contiguous ranges of ring steps whose unnormalised results go to
+    // part_o / part_ml for k_attn_merge
+    int nx;                   // units per head: s / (QT * 128)
+    int full_units;
+    int split;
+    float* part_o;            // [item - full_units][QT * 128][128] fp32: O
+    float* part_ml;           // [item - full_units][QT * 128][2] fp32: maximum in use (log2), sum
 };
 
 struct AttnMaps {
@@ -165,12 +174,22 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
     AttnTail<QT>* tail = reinterpret_cast<AttnTail<QT>*>(sm + (QT + 4) * kAttnTile);
     volatile int* abort = &tail->abort;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long q0 = (long long)blockIdx.x * (QT * kAttnBM);   // first query row
-    const long long g = blockIdx.y;                                 // batch * head index
-    const long long per = a.s / a.t;
-    const int rank = (int)(q0 / per);                               // the queries' rank
     const int T = a.tiles_per_block;
     const int n_tiles = a.t * T;
+    // this CTA's work item: a unit and the ring steps [j0, j0 + n_loc) of it;
+    // slot >= 0: a piece of a split unit, whose result is partial
+    int unit = (int)blockIdx.x, j0 = 0, n_loc = n_tiles, slot = -1;
+    if (unit >= a.full_units) {
+        slot = unit - a.full_units;
+        const int pc = slot % a.split;
+        unit = a.full_units + slot / a.split;
+        j0 = (int)((long long)n_tiles * pc / a.split);
+        n_loc = (int)((long long)n_tiles * (pc + 1) / a.split) - j0;
+    }
+    const long long q0 = (long long)(unit % a.nx) * (QT * kAttnBM);   // first query row
+    const long long g = unit / a.nx;                                  // batch * head index
+    const long long per = a.s / a.t;
+    const int rank = (int)(q0 / per);                                 // the queries' rank
     // first key row of tile j: block (rank - j / T) mod t, its (j % T)-th tile
     auto kv_row = [&](int j) -> long long {
         const int blk = ((rank - j / T) % a.t + a.t) % a.t;
@@ -228,9 +247,9 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
                             qb, pol);
             }
             int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
+            for (int j = 0; j < n_loc; ++j) {   // local step j: ring step j0 + j
                 const int st = j & 1;
-                const int krow = (int)(g * a.s + kv_row(j));
+                const int krow = (int)(g * a.s + kv_row(j0 + j));
                 if (j >= 2 && !mbar_wait(smem_addr(&tail->k_empty[st]),
                                          (uint32_t)(((j >> 1) - 1) & 1), abort, ERR_WAIT_EMPTY))
                     break;
@@ -318,19 +337,19 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
             };
             if constexpr (QT == 1) {
                 if (ok) ok = issue_s(0, 0);
-                if (ok && n_tiles > 1) ok = issue_s(0, 1);
-                for (int j = 0; ok && j < n_tiles; ++j) {
+                if (ok && n_loc > 1) ok = issue_s(0, 1);
+                for (int j = 0; ok && j < n_loc; ++j) {
                     ok = issue_pv(0, j);
-                    if (ok && j + 2 < n_tiles) ok = issue_s(0, j + 2);
+                    if (ok && j + 2 < n_loc) ok = issue_s(0, j + 2);
                 }
             } else {
                 if (ok) ok = issue_s(0, 0);
                 if (ok) ok = issue_s(1, 0);
-                for (int j = 0; ok && j < n_tiles; ++j) {
+                for (int j = 0; ok && j < n_loc; ++j) {
                     ok = issue_pv(0, j);
-                    if (ok && j + 1 < n_tiles) ok = issue_s(0, j + 1);
+                    if (ok && j + 1 < n_loc) ok = issue_s(0, j + 1);
                     if (ok) ok = issue_pv(1, j);
-                    if (ok && j + 1 < n_tiles) ok = issue_s(1, j + 1);
+                    if (ok && j + 1 < n_loc) ok = issue_s(1, j + 1);
                 }
             }
             // every issued MMA has finished before the CTA tears down
@@ -357,7 +376,7 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
         };
         float m = -INFINITY, l = 0.f;   // maximum in use (log2 units), this slice's sum
         bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
+        for (int j = 0; j < n_loc; ++j) {
             const int b = sbuf(qt, j);
             const int pb = j & 1;   // parity of the pair exchange
             if (!wait_all(smem_addr(&tail->s_full[b]), sphase(j))) {
@@ -447,8 +466,26 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
         float lt = tail->xsum[qt][0][row];   // the same order, so the same bits, in every warp
 #pragma unroll
         for (int h = 1; h < kAttnSplit; ++h) lt += tail->xsum[qt][h][row];
-        const int b_last = sbuf(qt, n_tiles - 1);
-        if (ok && wait_all(smem_addr(&tail->o_done[b_last]), sphase(n_tiles - 1))) {
+        const int b_last = sbuf(qt, n_loc - 1);
+        const bool o_ready = ok && wait_all(smem_addr(&tail->o_done[b_last]), sphase(n_loc - 1));
+        if (o_ready && slot >= 0) {
+            // a piece of a split unit: O as accumulated (scaled by 2^-m), m
+            // and the row's sum, for k_attn_merge
+            tmem_fence_after_sync();
+            const size_t prow = (size_t)slot * (QT * kAttnBM) + (size_t)qt * kAttnBM + row;
+            float* po = a.part_o + prow * kAttnD + kAttnCols * hf;
+#pragma unroll 1
+            for (int c = 0; c < kAttnCols / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tbase + tlane + ocol + (uint32_t)(kAttnCols * hf + 32 * c), o);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4*>(po + 32 * c + 4 * u) =
+                        make_float4(__uint_as_float(o[4 * u]), __uint_as_float(o[4 * u + 1]),
+                                    __uint_as_float(o[4 * u + 2]), __uint_as_float(o[4 * u + 3]));
+            }
+            if (hf == 0) *reinterpret_cast<float2*>(a.part_ml + 2 * prow) = make_float2(m, lt);
+        } else if (o_ready) {
             tmem_fence_after_sync();
             const float inv = 1.0f / lt;
             const long long qrow = q0 + (long long)qt * kAttnBM + row;
@@ -480,6 +517,51 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
         tmem_fence_after_sync();
         tmem_dealloc(tbase, 512);
     }
+}
+
+// The pieces of each split unit, combined in piece order: with m_i the
+// maximum a piece's exponentials used (log2 units), l_i its row sum and O_i
+// its accumulated output, M = max m_i, L = sum 2^(m_i - M) l_i and the row's
+// output is sum 2^(m_i - M) O_i / L, its log-sum-exp (M + log2 L) ln 2.  One
+// warp per query row; lane l owns head features 4l .. 4l + 3.
+constexpr int kAttnMergeThreads = 256;
+
+static __global__ void __launch_bounds__(kAttnMergeThreads)
+    k_attn_merge(const __grid_constant__ AttnArgs a, int rows_per_unit, long long rows)
+{
+    grid_dep_launch();
+    grid_dep_wait();   // every piece is written and visible
+    const long long r = (long long)blockIdx.x * (kAttnMergeThreads / 32) + (threadIdx.x >> 5);
+    if (r >= rows) return;   // uniform over the warp
+    const int lane = threadIdx.x & 31;
+    const long long u_t = r / rows_per_unit;   // split unit, counted from the first one
+    const int rr = (int)(r - u_t * rows_per_unit);
+    const long long unit = a.full_units + u_t;
+    const long long g = unit / a.nx;
+    const long long qrow = (unit % a.nx) * rows_per_unit + rr;
+    const size_t prow0 = (size_t)u_t * a.split * rows_per_unit + rr;   // piece 0's row
+    float M = -INFINITY;
+    for (int pc = 0; pc < a.split; ++pc)
+        M = fmaxf(M, a.part_ml[2 * (prow0 + (size_t)pc * rows_per_unit)]);
+    float L = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int pc = 0; pc < a.split; ++pc) {
+        const size_t prow = prow0 + (size_t)pc * rows_per_unit;
+        const float2 ml = *reinterpret_cast<const float2*>(a.part_ml + 2 * prow);
+        const float w = exp2f(ml.x - M);
+        L += w * ml.y;
+        const float4 x = *reinterpret_cast<const float4*>(a.part_o + prow * kAttnD + 4 * lane);
+        o.x += w * x.x;
+        o.y += w * x.y;
+        o.z += w * x.z;
+        o.w += w * x.w;
+    }
+    const float inv = 1.0f / L;
+    const uint2 pk = make_uint2(IO<__nv_bfloat16>::pack2(o.x * inv, o.y * inv),
+                                IO<__nv_bfloat16>::pack2(o.z * inv, o.w * inv));
+    *reinterpret_cast<uint2*>(static_cast<unsigned char*>(a.out) +
+                              ((size_t)g * a.s + qrow) * (kAttnD * 2) + 8 * lane) = pk;
+    if (a.lse && lane == 0) a.lse[(size_t)g * a.s + qrow] = (M + log2f(L)) * 0.69314718055994531f;
 }
 
 }  // namespace spk

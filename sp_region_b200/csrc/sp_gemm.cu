@@ -122,6 +122,159 @@ int check_gemm_cfg(const sp_cfg* cfg)
     return SP_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Ring attention: shape checks, the work split and the launch
+// ---------------------------------------------------------------------------
+
+int check_attn_shape(const sp_cfg* cfg, int heads)
+{
+    int rc = check_gemm_cfg(cfg);
+    if (rc) return rc;
+    if (heads < 1) return SP_ERR_INVALID_ARG;
+    if (!(cfg->row_begin == 0 && cfg->row_end == 0)) return SP_ERR_INVALID_ARG;
+    if (cfg->h != (int64_t)heads * kAttnD) return SP_ERR_UNSUPPORTED;   // head dim 128
+    const long long S = cfg->s, per = S / cfg->t;
+    if (S % kAttnBM || per % kAttnBN) return SP_ERR_UNSUPPORTED;
+    const long long bh = cfg->b * (long long)heads;
+    if (bh * S >= (1LL << 31)) return SP_ERR_UNSUPPORTED;
+    return SP_OK;
+}
+
+constexpr int kAttnMaxSplit = 8;      // pieces per split unit, at most
+constexpr int kAttnMinPiece = 4;      // ring steps (key tiles) per piece, at least
+
+// The work of one call: units of QT query tiles of one head, every ring step.
+// They run one CTA each (one CTA per SM), so `units` CTAs take
+// ceil(units / sms) rounds of the slowest SM.  With `split` allowed, the
+// units of the last, partly filled round are cut into k contiguous ranges of
+// ring steps, the k that leaves the shortest last round (ceil(R k / sms) / k
+// unit times for R leftover units), and combined afterwards.
+struct AttnPlan {
+    int qt;
+    int nx;                  // units per head
+    long long units;
+    long long full_units;    // whole units
+    long long tail_units;    // split units
+    int split;               // pieces per split unit (1: none)
+    size_t ws_bytes;         // partial results of the pieces
+};
+
+void attn_plan(const sp_cfg* cfg, int heads, int sms, bool allow_split, AttnPlan* p)
+{
+    const long long S = cfg->s, per = S / cfg->t;
+    const long long bh = cfg->b * (long long)heads;
+    // two query tiles per CTA when a rank's block holds an even number of
+    // them (both then visit the key tiles in the same ring order)
+    p->qt = per % (2 * kAttnBM) == 0 ? 2 : 1;
+    p->nx = (int)(S / (p->qt * kAttnBM));
+    p->units = (long long)p->nx * bh;
+    p->full_units = p->units;
+    p->tail_units = 0;
+    p->split = 1;
+    p->ws_bytes = 0;
+    const long long rem = sms > 0 ? p->units % sms : 0;
+    if (!allow_split || rem == 0) return;
+    const long long n_tiles = S / kAttnBN;
+    int best_k = 1;
+    double best = 1.0;   // the last round, in unit times, without a split
+    for (int k = 2; k <= kAttnMaxSplit && n_tiles / k >= kAttnMinPiece; ++k) {
+        const double tt = (double)((rem * k + sms - 1) / sms) / k;
+        if (tt < best - 1e-9) {
+            best = tt;
+            best_k = k;
+        }
+    }
+    if (best_k == 1) return;
+    p->split = best_k;
+    p->tail_units = rem;
+    p->full_units = p->units - rem;
+    p->ws_bytes = (size_t)rem * best_k * (size_t)(p->qt * kAttnBM) * (kAttnD + 2) * sizeof(float);
+}
+
+int attn_fwd(const sp_cfg* cfg, int heads, float scale, const void* q, const void* k,
+             const void* v, void* out, float* lse, void* workspace, size_t workspace_bytes,
+             bool allow_split, void* stream)
+{
+    int rc = check_attn_shape(cfg, heads);
+    if (rc) return rc;
+    if (!q || !k || !v || !out || !(scale > 0.0f) || !isfinite(scale)) return SP_ERR_INVALID_ARG;
+    for (const void* p : {q, k, v, (const void*)out})
+        if (!aligned(p, 16)) return SP_ERR_INVALID_ARG;
+    if (lse && !aligned(lse, 4)) return SP_ERR_INVALID_ARG;
+    if (workspace && !aligned(workspace, 16)) return SP_ERR_INVALID_ARG;
+    DevInfo dev;
+    if ((rc = use_device_of(out, &dev))) return rc;
+    AttnPlan pl;
+    attn_plan(cfg, heads, dev.sms, allow_split, &pl);
+    if (pl.ws_bytes && (!workspace || workspace_bytes < pl.ws_bytes)) return SP_ERR_INVALID_ARG;
+
+    const long long S = cfg->s, per = S / cfg->t;
+    const long long bh = cfg->b * (long long)heads;
+    AttnMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (!make_map(&maps.q, q, bh * S, kAttnD, kAttnD, kAttnBM) ||
+        !make_map(&maps.k, k, bh * S, kAttnD, kAttnD, kAttnBN) ||
+        !make_map(&maps.v, v, bh * S, kAttnD, kAttnD, kAttnBN))
+        return SP_ERR_INVALID_ARG;
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.s = S;
+    a.t = cfg->t;
+    a.tiles_per_block = (int)(per / kAttnBN);
+    a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    a.out = out;
+    a.lse = lse;
+    a.nx = pl.nx;
+    a.full_units = (int)pl.full_units;
+    a.split = pl.split;
+    const size_t rows_per_unit = (size_t)pl.qt * kAttnBM;
+    const long long pieces = pl.tail_units * pl.split;
+    if (pieces) {
+        a.part_o = static_cast<float*>(workspace);
+        a.part_ml = a.part_o + (size_t)pieces * rows_per_unit * kAttnD;
+    }
+    const int qt = pl.qt;
+    const size_t smem =
+        1024 + (size_t)(qt + 4) * kAttnTile +
+        (((qt == 2 ? sizeof(AttnTail<2>) : sizeof(AttnTail<1>)) + 127) & ~(size_t)127);
+    if (smem > (size_t)dev.smem_optin) return SP_ERR_UNSUPPORTED;
+    const void* kern = qt == 2 ? (const void*)k_ring_attn<2> : (const void*)k_ring_attn<1>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3((unsigned)(pl.full_units + pieces));
+    lc.blockDim = dim3(attn_threads(qt));
+    lc.dynamicSmemBytes = smem;
+    lc.stream = static_cast<cudaStream_t>(stream);
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    void* params[] = {&a, &maps};
+    if (cudaLaunchKernelExC(&lc, kern, params) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    if (!pieces) return SP_OK;
+    // the split units' rows, one warp each
+    int rpu = (int)rows_per_unit;
+    long long rows = pl.tail_units * (long long)rows_per_unit;
+    constexpr int kWarpsPerBlock = kAttnMergeThreads / 32;
+    lc.gridDim = dim3((unsigned)((rows + kWarpsPerBlock - 1) / kWarpsPerBlock));
+    lc.blockDim = dim3(kAttnMergeThreads);
+    lc.dynamicSmemBytes = 0;
+    void* mparams[] = {&a, &rpu, &rows};
+    if (cudaLaunchKernelExC(&lc, (const void*)k_attn_merge, mparams) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -217,64 +370,31 @@ int sp_ag_colpar_linear_fwd(const sp_cfg* cfg, int64_t f_out, const void* const*
 int sp_ring_attention_fwd(const sp_cfg* cfg, int32_t heads, float scale, const void* q,
                           const void* k, const void* v, void* out, float* lse, void* stream)
 {
-    int rc = check_gemm_cfg(cfg);
-    if (rc) return rc;
-    if (!q || !k || !v || !out || heads < 1 || !(scale > 0.0f) || !isfinite(scale))
-        return SP_ERR_INVALID_ARG;
-    if (!(cfg->row_begin == 0 && cfg->row_end == 0)) return SP_ERR_INVALID_ARG;
-    if (cfg->h != (int64_t)heads * kAttnD) return SP_ERR_UNSUPPORTED;   // head dim 128
-    const long long S = cfg->s, per = S / cfg->t;
-    if (S % kAttnBM || per % kAttnBN) return SP_ERR_UNSUPPORTED;
-    const long long bh = cfg->b * (long long)heads;
-    if (bh * S >= (1LL << 31) || bh > 65535) return SP_ERR_UNSUPPORTED;
-    for (const void* p : {q, k, v, (const void*)out})
-        if (!aligned(p, 16)) return SP_ERR_INVALID_ARG;
-    if (lse && !aligned(lse, 4)) return SP_ERR_INVALID_ARG;
-    DevInfo dev;
-    if ((rc = use_device_of(out, &dev))) return rc;
+    return attn_fwd(cfg, heads, scale, q, k, v, out, lse, nullptr, 0, false, stream);
+}
 
-    AttnMaps maps;
-    memset(&maps, 0, sizeof(maps));
-    if (!make_map(&maps.q, q, bh * S, kAttnD, kAttnD, kAttnBM) ||
-        !make_map(&maps.k, k, bh * S, kAttnD, kAttnD, kAttnBN) ||
-        !make_map(&maps.v, v, bh * S, kAttnD, kAttnD, kAttnBN))
-        return SP_ERR_INVALID_ARG;
-    AttnArgs a;
-    memset(&a, 0, sizeof(a));
-    a.s = S;
-    a.t = cfg->t;
-    a.tiles_per_block = (int)(per / kAttnBN);
-    a.scale_log2 = (float)((double)scale * 1.4426950408889634);
-    a.out = out;
-    a.lse = lse;
-    // two query tiles per CTA when a rank's block holds an even number of
-    // them (both then visit the key tiles in the same ring order)
-    const int qt = per % (2 * kAttnBM) == 0 ? 2 : 1;
-    const size_t smem =
-        1024 + (size_t)(qt + 4) * kAttnTile +
-        (((qt == 2 ? sizeof(AttnTail<2>) : sizeof(AttnTail<1>)) + 127) & ~(size_t)127);
-    if (smem > (size_t)dev.smem_optin) return SP_ERR_UNSUPPORTED;
-    const void* kern = qt == 2 ? (const void*)k_ring_attn<2> : (const void*)k_ring_attn<1>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess) {
+int sp_ring_attention_fwd_ws(const sp_cfg* cfg, int32_t heads, float scale, const void* q,
+                             const void* k, const void* v, void* out, float* lse,
+                             void* workspace, size_t workspace_bytes, void* stream)
+{
+    return attn_fwd(cfg, heads, scale, q, k, v, out, lse, workspace, workspace_bytes, true,
+                    stream);
+}
+
+int sp_ring_attention_workspace_bytes(const sp_cfg* cfg, int32_t heads, int32_t device,
+                                      size_t* bytes)
+{
+    int rc = check_attn_shape(cfg, heads);
+    if (rc) return rc;
+    if (!bytes) return SP_ERR_INVALID_ARG;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) {
         cudaGetLastError();
         return SP_ERR_CUDA;
     }
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3((unsigned)(S / (qt * kAttnBM)), (unsigned)bh);
-    lc.blockDim = dim3(attn_threads(qt));
-    lc.dynamicSmemBytes = smem;
-    lc.stream = static_cast<cudaStream_t>(stream);
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-    void* params[] = {&a, &maps};
-    if (cudaLaunchKernelExC(&lc, kern, params) != cudaSuccess) {
-        cudaGetLastError();
-        return SP_ERR_CUDA;
-    }
+    AttnPlan pl;
+    attn_plan(cfg, heads, sms, true, &pl);
+    *bytes = pl.ws_bytes;
     return SP_OK;
 }
 
