@@ -28,5 +28,16 @@ int main(void)
     cfg.dtype = SP_BF16; cfg.norm = SP_LAYERNORM; cfg.eps = 1e-5f;
     size_t ws = 0;
     printf("bad_cfg %d\n", sp_bwd_workspace_bytes(&cfg, 0, &ws));
+
+    /* ring attention's workspace query: shapes it does not take, and a NULL
+     * result pointer, are answered before any device query */
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.s = 384; cfg.b = 1; cfg.h = 128; cfg.t = 2;   /* s / t = 192 */
+    cfg.dtype = SP_BF16; cfg.norm = SP_LAYERNORM; cfg.eps = 1e-5f;
+    printf("attn_ragged %d\n", sp_ring_attention_workspace_bytes(&cfg, 1, 0, &ws));
+    cfg.s = 256; cfg.t = 1; cfg.h = 64;                /* head dimension 64 */
+    printf("attn_head64 %d\n", sp_ring_attention_workspace_bytes(&cfg, 1, 0, &ws));
+    cfg.h = 128;
+    printf("attn_null %d\n", sp_ring_attention_workspace_bytes(&cfg, 1, 0, NULL));
     return 0;
 }

@@ -30,3 +30,6 @@ def test_c_program_links_and_calls_the_abi(tmp_path, orc):
     assert int(got["bad_mode"]) == sp.SP_ERR_INVALID_ARG
     assert got["status"] == sp.sp_status_string(sp.SP_ERR_INVALID_ARG)
     assert int(got["bad_cfg"]) == sp.SP_ERR_INVALID_ARG
+    assert int(got["attn_ragged"]) == sp.SP_ERR_UNSUPPORTED
+    assert int(got["attn_head64"]) == sp.SP_ERR_UNSUPPORTED
+    assert int(got["attn_null"]) == sp.SP_ERR_INVALID_ARG
