@@ -40,8 +40,10 @@
 //                      units): the probabilities then stay below 2^8, and O is
 //                      rescaled in tensor memory only on those tiles, so in
 //                      most tiles the softmax never waits for the previous
-//                      PV.  P goes to tensor memory as bf16 pairs; at the end
-//                      O / l to global memory and the log-sum-exp
+//                      PV.  One exponential pair in 8 is a cubic on the FMA
+//                      pipe, the rest the transcendental unit's.  P goes to
+//                      tensor memory as bf16 pairs; at the end O / l to
+//                      global memory and the log-sum-exp
 // Tensor memory: QT = 1: S0/P0 [0, 128), S1/P1 [128, 256), O [256, 384);
 // QT = 2: S/P of tile A [0, 128), of tile B [128, 256), O_A [256, 384), O_B
 // [384, 512).
@@ -139,6 +141,27 @@ __device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, u
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
         "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// 2^x for both halves on the FMA pipe: x = n + f with n the nearest integer
+// (the 1.5 * 2^23 rounding constant) and f in [-1/2, 1/2]; 2^f by a cubic
+// fitted to it in relative error on that interval (at most 7.5e-5, far
+// below the bf16 rounding P gets); 2^n added to the exponent field.  x is
+// clamped at -125, where the result (2^-125) is negligible against the row
+// sum, so the exponent field never underflows.
+__device__ __forceinline__ F2 exp2_poly2(F2 x)
+{
+    const float2 xs = halves(x);
+    const F2 xc = f2(fmaxf(xs.x, -125.0f), fmaxf(xs.y, -125.0f));
+    const F2 sh = add2(xc, f2(12582912.0f));
+    const F2 n = sub2(sh, f2(12582912.0f));
+    const F2 fr = sub2(xc, n);
+    F2 p = fma2(f2(0x1.c3f610p-5f), fr, f2(0x1.f0de1cp-3f));
+    p = fma2(p, fr, f2(0x1.62f31ep-1f));
+    p = fma2(p, fr, f2(0x1.fff692p-1f));
+    const float2 ps = halves(p), ss = halves(sh);
+    return f2(__int_as_float(__float_as_int(ps.x) + (__float_as_int(ss.x) << 23)),
+              __int_as_float(__float_as_int(ps.y) + (__float_as_int(ss.y) << 23)));
 }
 
 // 2^x by the transcendental unit's approximation (PTX ex2.approx.ftz: at most
@@ -426,11 +449,22 @@ __global__ void __launch_bounds__(attn_threads(QT), 1)
                 tmem_ld32(scol + 32 * c, sc);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float2 x = halves(fma2(f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])),
-                                                 scale2, negm2));
-                    const float p0 = ex2_approx(x.x), p1 = ex2_approx(x.y);
-                    lsum2 = add2(lsum2, f2(p0, p1));
-                    pk[i] = IO<__nv_bfloat16>::pack2(p0, p1);
+                    const F2 x2 = fma2(f2(__uint_as_float(sc[2 * i]), __uint_as_float(sc[2 * i + 1])),
+                                       scale2, negm2);
+                    F2 p2;
+                    if ((i & 7) == 7) {
+                        // one pair in 8 on the FMA pipe: the transcendental
+                        // unit is the softmax's critical resource (16384
+                        // exponentials a tile against the other query tile's
+                        // MMAs); more than 1 in 8 costs more issue than it saves
+                        p2 = exp2_poly2(x2);
+                    } else {
+                        const float2 x = halves(x2);
+                        p2 = f2(ex2_approx(x.x), ex2_approx(x.y));
+                    }
+                    lsum2 = add2(lsum2, p2);
+                    const float2 pp = halves(p2);
+                    pk[i] = IO<__nv_bfloat16>::pack2(pp.x, pp.y);
                 }
                 tmem_st16(scol + 16 * c, pk);
             }

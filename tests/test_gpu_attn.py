@@ -5,14 +5,16 @@ section "Context parallelism and ring attention").
 Tolerance.  The kernel's scores are fp32 sums of d = 128 products
 accumulated in tensor memory, |ds| <= (d/16 + 16) 2^-23 scale sum_c |q_c k_c|.
 The probabilities enter the second product as bf16 (relative error up to
-2^-9, plus exp2's few ulps), while the normaliser l sums them in fp32, and
-the output accumulates over all s keys in fp32.  So an output element passes
-when
+2^-9, plus exp2's few ulps; one pair in 8 comes from a cubic whose relative
+error is at most 7.5e-5), while the normaliser l sums them in fp32 (so l is
+off by at most 7.5e-5 relative), and the output accumulates over all s keys
+in fp32.  So an output element passes when
 
   |out - ref| <= ulp_bf16(ref) + (2^-8 + 2 max|ds| + (s/16 + 16) 2^-23) W,
 
-W = sum_j softmax_j |v_j| (the attention-weighted mean of |v|, float64),
-and the log-sum-exp when |lse - ref| <= 2 max|ds| + 1e-5 (1 + |ref|).
+W = sum_j softmax_j |v_j| (the attention-weighted mean of |v|, float64;
+2^-8 covers 2^-9 + 2 * 7.5e-5), and the log-sum-exp when
+|lse - ref| <= 2 max|ds| + 1e-5 (1 + |ref|) + 7.5e-5.
 """
 import concurrent.futures
 import gc
@@ -31,6 +33,7 @@ import sp_region_b200 as sp
 pytestmark = pytest.mark.gpu
 
 D = 128
+EXP2_POLY_REL = 7.5e-5   # the kernel's cubic for 2^f, f in [-1/2, 1/2]: max relative error
 
 
 @pytest.fixture(autouse=True)
@@ -103,7 +106,7 @@ def _check(out, lse, ref, ref_lse, q, k, v, scale):
     bad = ~(np.abs(g - r) <= tol)
     assert not bad.any(), (f"out: {int(bad.sum())} of {bad.size} outside; first "
                            f"{np.argwhere(bad)[:3].tolist()}")
-    lt = 2 * ds[..., 0] + 1e-5 * (1 + np.abs(ref_lse))
+    lt = 2 * ds[..., 0] + 1e-5 * (1 + np.abs(ref_lse)) + EXP2_POLY_REL
     bad = ~(np.abs(np.asarray(lse, np.float64) - ref_lse) <= lt)
     assert not bad.any(), f"lse: {int(bad.sum())} of {bad.size} outside"
 
