@@ -129,12 +129,21 @@ def measured_tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback (no MEASURED_PEAKS.json)"
 
 
+# the translation units of the streaming kernels (k_fwd_tma, k_bwd_tma,
+# k_colreduce, k_norm_ag) and every file they include: the recorded traffic
+# depends on these and on nothing else (the linears and ring attention are
+# built in their own unit)
+STREAMING_SOURCES = ("sp_region.cu", "sp_inst_fwd.cu", "sp_inst_bwd.cu", "sp_bwd.cuh",
+                     "sp_device.cuh", "sp_entry.cuh", "sp_fwd.cuh", "sp_gather.cuh",
+                     "sp_host.h", "sp_plans.h")
+
+
 def kernel_sources_sha():
-    """Hash of every source the library is built from (csrc/*, the header)."""
+    """Hash of the sources the streaming kernels are built from (their csrc
+    files and the header)."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "sp_region_b200", "csrc")
-    files = sorted(os.path.join(csrc, f) for f in os.listdir(csrc)
-                   if f.endswith((".cu", ".cuh", ".h")))
+    files = [os.path.join(csrc, f) for f in sorted(STREAMING_SOURCES)]
     for f in files + [os.path.join(ROOT, "include", "sp_region.h")]:
         with open(f, "rb") as fh:
             h.update(fh.read())

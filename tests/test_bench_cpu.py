@@ -1,7 +1,12 @@
 """bench.py's CPU baselines (the oracle timed on the host cores): one core,
-and one spawned process per core, on a small workload."""
+and one spawned process per core, on a small workload; and the source set
+that keys the recorded traffic."""
+import os
+
 import bench
 from sp_synth import WORKLOADS
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_cpu_baselines_report_their_sample_and_cores():
@@ -32,3 +37,20 @@ def test_algorithmic_bytes_follow_the_stated_formulas():
     # the entry: read x, write the gathered rows
     e = bench.entry_fwd_bytes(w)
     assert e == 2 * sbh + 2 * 2 * h + 2 * sbh + 8 * N
+
+
+def test_traffic_hash_covers_the_streaming_kernels_sources():
+    """The recorded DRAM traffic is keyed by a hash of the files the streaming
+    kernels are built from: their translation units and every file those
+    include, transitively, and nothing else."""
+    import re
+    csrc = os.path.join(ROOT, "sp_region_b200", "csrc")
+    todo, seen = ["sp_region.cu", "sp_inst_fwd.cu", "sp_inst_bwd.cu"], set()
+    while todo:
+        f = todo.pop()
+        path = os.path.join(csrc, f)
+        if f in seen or not os.path.exists(path):
+            continue
+        seen.add(f)
+        todo += re.findall(r'#include "([^"]+)"', open(path).read())
+    assert seen == set(bench.STREAMING_SOURCES)
