@@ -11,6 +11,7 @@
 
 #include "sp_attn.cuh"
 #include "sp_gemm.cuh"
+#include "sp_gemm2.cuh"
 #include "sp_host.h"
 #include "sp_plans.h"
 #include "sp_region.h"
@@ -103,15 +104,71 @@ int launch_gemm(GemmArgs a, const GemmMaps& maps, const DevInfo& dev, cudaStream
     return SP_OK;
 }
 
+// Persistent launch of k_tp_gemm2: as many CTA pairs as can be resident at
+// once (a pair needs two SMs of one TPC), at most one per 256 x 256 tile.
+template <int EPI>
+int launch_gemm2(GemmArgs a, const GemmMaps& maps, const DevInfo& dev, cudaStream_t st)
+{
+    constexpr size_t kStage = (size_t)(kGemmBM + kGemm2HalfN) * kGemmBK * 2;
+    const size_t fixed = 1024 + ((sizeof(GemmTail2) + 127) & ~(size_t)127);
+    if ((size_t)dev.smem_optin <= fixed + 2 * kStage) return SP_ERR_UNSUPPORTED;
+    int S = (int)(((size_t)dev.smem_optin - fixed) / kStage);
+    if (S > kGemm2MaxStages) S = kGemm2MaxStages;
+    a.stages = S;
+    const size_t smem = fixed + (size_t)S * kStage;
+    const void* kern = (const void*)k_tp_gemm2<EPI>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kGemm2Threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;   // the occupancy query takes the cluster shape alone
+    cfg.gridDim = dim3((unsigned)(dev.sms & ~1));
+    static int pairs_cache[64][2];
+    int pairs = dev.id >= 0 && dev.id < 64 ? pairs_cache[dev.id][EPI] : 0;
+    if (pairs <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess || pairs <= 0) {
+            cudaGetLastError();
+            return SP_ERR_UNSUPPORTED;
+        }
+        if (dev.id >= 0 && dev.id < 64) pairs_cache[dev.id][EPI] = pairs;
+    }
+    const long long tiles = ((a.M + 2 * kGemmBM - 1) / (2 * kGemmBM)) *
+                            (long long)((a.N + kGemm2BN - 1) / kGemm2BN);
+    if (tiles < 1) return SP_OK;
+    const long long np = tiles < pairs ? tiles : pairs;
+    cfg.gridDim = dim3((unsigned)(2 * np));
+    cfg.numAttrs = 2;
+    void* params[] = {&a, const_cast<GemmMaps*>(&maps)};
+    if (cudaLaunchKernelExC(&cfg, kern, params) != cudaSuccess) {
+        cudaGetLastError();
+        return SP_ERR_CUDA;
+    }
+    return SP_OK;
+}
+
 template <int EPI>
 int launch_gemm_bn(const GemmArgs& a, const GemmMaps& maps, const DevInfo& dev, cudaStream_t st,
                    int bn)
 {
-    return bn == 256 ? launch_gemm<256, EPI>(a, maps, dev, st)
+    return bn == 256 ? launch_gemm2<EPI>(a, maps, dev, st)
                      : launch_gemm<128, EPI>(a, maps, dev, st);
 }
 
-// output features per tile: 256 unless the output is narrower
+// output features per tile: 256 (a CTA pair, k_tp_gemm2) unless the output
+// is narrower (one CTA, k_tp_gemm with 128-feature tiles)
 int pick_bn(long long n) { return n >= 256 ? 256 : 128; }
 
 int check_gemm_cfg(const sp_cfg* cfg)
@@ -303,7 +360,8 @@ int sp_rowpar_linear_rs_fwd(const sp_cfg* cfg, int64_t f, const void* x, const v
     memset(&maps, 0, sizeof(maps));
     // x: this call's rows [rows][f]; the t ranks' slices are its column
     // blocks, so one map covers every rank
-    if (!make_map(&maps.a[0], x, rows, f, f, kGemmBM) || !make_map(&maps.b, w, h, f, f, bn))
+    if (!make_map(&maps.a[0], x, rows, f, f, kGemmBM) ||
+        !make_map(&maps.b, w, h, f, f, bn == 256 ? kGemm2HalfN : bn))
         return SP_ERR_INVALID_ARG;
     GemmArgs a;
     memset(&a, 0, sizeof(a));
@@ -355,7 +413,7 @@ int sp_ag_colpar_linear_fwd(const sp_cfg* cfg, int64_t f_out, const void* const*
     memset(&maps, 0, sizeof(maps));
     for (int r = 0; r < t; ++r)
         if (!make_map(&maps.a[r], shards[r], per, h, h, kGemmBM)) return SP_ERR_INVALID_ARG;
-    if (!make_map(&maps.b, w, f_out, h, h, bn)) return SP_ERR_INVALID_ARG;
+    if (!make_map(&maps.b, w, f_out, h, h, bn == 256 ? kGemm2HalfN : bn)) return SP_ERR_INVALID_ARG;
     GemmArgs a;
     memset(&a, 0, sizeof(a));
     a.M = N;
