@@ -83,6 +83,8 @@ CASES = [
     ("two_col_tiles_rms_p0", 192, 512, 384, 4, 0.0, False, "rmsnorm"),
     ("c2_width_t8", 256, 1024, 6144, 8, 0.1, True, "layernorm"),
     ("t1", 128, 136, 128, 1, 0.25, True, "layernorm"),
+    # 80 CTA-pair tiles: more than a B200's 74 clusters take in one round
+    ("two_rounds_of_pair_tiles", 2048, 256, 2560, 4, 0.1, True, "layernorm"),
 ]
 
 
@@ -154,6 +156,7 @@ AG_CASES = [
     ("t4_ragged_cols", 1024, 512, 264, 4),
     ("t1_ragged_rows_k", 300, 520, 128, 1),
     ("t8", 1024, 1024, 512, 8),
+    ("two_rounds_of_pair_tiles", 2048, 256, 2560, 4),
 ]
 
 
