@@ -649,10 +649,10 @@ def time_linears(args, sp, torch, dev):
                      f"down-projection f={f} -> h, then the SP boundary (LN, p=0.1, "
                      f"bias); column-parallel up-projection h -> {fo}; bf16"),
         "peak_tflops": peak, "peak_source": peak_src,
-        "fused": rec("k_tp_gemm (SP epilogue) + k_norm_ag", fused_ms),
-        "gemm": rec("k_tp_gemm (SP epilogue)", gemm_ms),
-        "unfused": rec(f"{t} x k_tp_gemm (partials to HBM) + k_fwd_tma", unfused_ms),
-        "colpar": rec("k_tp_gemm (all-gather prologue)", col_ms, 2.0 * N * h * fo),
+        "fused": rec("k_tp_gemm2 (CTA pairs, SP epilogue) + k_norm_ag", fused_ms),
+        "gemm": rec("k_tp_gemm2 (CTA pairs, SP epilogue)", gemm_ms),
+        "unfused": rec(f"{t} x k_tp_gemm2 (partials to HBM) + k_fwd_tma", unfused_ms),
+        "colpar": rec("k_tp_gemm2 (CTA pairs, all-gather prologue)", col_ms, 2.0 * N * h * fo),
         "fused_speedup": round(unfused_ms / fused_ms, 3),
     }
     del w_in, z, out, rout, res
