@@ -277,3 +277,21 @@ def test_ring_attention_ws_rejects_a_short_workspace():
     with pytest.raises(sp.SPError) as e:
         sp.sp_ring_attention_workspace_bytes(sp.make_cfg(384, 1, D, 2), 1)
     assert e.value.status == sp.SP_ERR_UNSUPPORTED
+
+
+def test_ring_attention_ws_without_lse():
+    """The workspace call with no log-sum-exp output: the split units' merge
+    skips it and writes the same output bits as with it."""
+    b, heads, s, t = 1, 10, 4096, 4   # 160 units: whole and split ones
+    q, k, v = _qkv(b, heads, s, 12, device="cuda")
+    cfg = sp.make_cfg(s, b, heads * D, t, dtype="bf16")
+    nbytes = sp.sp_ring_attention_workspace_bytes(cfg, heads)
+    ws = torch.empty(nbytes // 4 + 4, device="cuda") if nbytes else None
+    out1 = torch.empty_like(q)
+    lse = torch.empty((b, heads, s), dtype=torch.float32, device="cuda")
+    sp.sp_ring_attention_fwd_ws(cfg, heads, D ** -0.5, q, k, v, out1, lse, ws)
+    out2 = torch.full_like(q, float("nan"))
+    sp.sp_ring_attention_fwd_ws(cfg, heads, D ** -0.5, q, k, v, out2, None, ws)
+    torch.cuda.synchronize()
+    assert sp.sp_device_error() == 0
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
