@@ -774,6 +774,22 @@ int sp_all_gather(const sp_cfg* cfg, const void* const* shards, void* const* out
     a.n_out = n_out;
     a.unit_bytes = vec ? 16 : E;
     a.shard_units = shard_bytes / a.unit_bytes;
+    if (vec) {
+        // bulk copies through shared memory, one issuing thread per SM
+        const long long chunks =
+            (shard_bytes + kAgChunk - 1) / kAgChunk * (long long)cfg->t;
+        if (chunks < 1) return SP_OK;
+        const size_t smem = (size_t)kAgSlots * kAgChunk;
+        if (smem > (size_t)dev.smem_optin) return SP_ERR_UNSUPPORTED;
+        const void* kern = (const void*)k_all_gather_bulk;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess) {
+            cudaGetLastError();
+            return SP_ERR_CUDA;
+        }
+        const int grid = (int)(chunks < dev.sms ? chunks : dev.sms);
+        return launch_kernel(kern, grid, 32, smem, static_cast<cudaStream_t>(stream), &a);
+    }
     const long long total = a.shard_units * a.t;
     long long grid = (total + 511) / 512;
     const long long cap = (long long)dev.sms * 4;
