@@ -542,7 +542,7 @@ def time_workloads(args, sp, torch, dev, peak):
                       for r in range(t)]
             ms = time_launches(torch, stream, lambda: sp.sp_all_gather(
                 cfg, shards, gath[1:], stream=stream), K, 3)
-            rec["all_gather"] = entry(f"k_all_gather ({t - 1} replicas)",
+            rec["all_gather"] = entry(f"k_all_gather_bulk ({t - 1} replicas)",
                                       all_gather_bytes(w, t - 1), ms)
         del parts
         gc.collect()
