@@ -2,8 +2,9 @@
 // tensors ("SP: Partition Activations Alongside TP", section "Change layouts
 // between SP and TP": the shards of the SP region combine into the same
 // input X on every GPU).  On one GPU this is a copy of each shard into its
-// row range of every output; each 16-byte vector is read once and written
-// n_out times.
+// row range of every output: each shard is read once and written n_out
+// times, by bulk copies through shared memory when every buffer is 16-byte
+// aligned (k_all_gather_bulk), else element by element (k_all_gather).
 #pragma once
 
 #include "sp_device.cuh"

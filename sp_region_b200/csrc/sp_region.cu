@@ -795,9 +795,9 @@ int sp_all_gather(const sp_cfg* cfg, const void* const* shards, void* const* out
     const long long cap = (long long)dev.sms * 4;
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
-    const void* kern = vec ? (const void*)k_all_gather<uint4>
-                           : (E == 4 ? (const void*)k_all_gather<uint32_t>
-                                     : (const void*)k_all_gather<uint16_t>);
+    // unaligned buffers: the element-wise copy
+    const void* kern = E == 4 ? (const void*)k_all_gather<uint32_t>
+                              : (const void*)k_all_gather<uint16_t>;
     return launch_kernel(kern, (int)grid, 512, 0, static_cast<cudaStream_t>(stream), &a);
 }
 
