@@ -163,6 +163,30 @@ def test_all_gather_validation(lib):
         sp.SP_ERR_INVALID_ARG
 
 
+def test_ring_attention_validation(lib):
+    """Both attention calls reject bad shapes, NULL or misaligned pointers, a
+    bad scale and a misaligned workspace before any device query."""
+    import sp_region_b200 as sp
+    vp, f = ctypes.c_void_p, ctypes.c_float
+    lib.sp_ring_attention_fwd.argtypes = [ctypes.c_void_p, ctypes.c_int32, f, vp, vp, vp, vp,
+                                          vp, vp]
+    lib.sp_ring_attention_fwd_ws.argtypes = [ctypes.c_void_p, ctypes.c_int32, f, vp, vp, vp,
+                                             vp, vp, vp, ctypes.c_size_t, vp]
+    cfg = sp.make_cfg(256, 1, 128, 2, dtype="bf16")
+    ok, odd = vp(0x1000), vp(0x1008)
+    ws_args = lambda *p: lib.sp_ring_attention_fwd_ws(ctypes.byref(cfg), 1, 0.1, *p)
+    assert ws_args(None, ok, ok, ok, None, ok, 1 << 20, None) == sp.SP_ERR_INVALID_ARG
+    assert ws_args(ok, ok, ok, odd, None, ok, 1 << 20, None) == sp.SP_ERR_INVALID_ARG
+    assert ws_args(ok, ok, ok, ok, None, odd, 1 << 20, None) == sp.SP_ERR_INVALID_ARG
+    assert lib.sp_ring_attention_fwd_ws(ctypes.byref(cfg), 1, -1.0, ok, ok, ok, ok, None, ok,
+                                        1 << 20, None) == sp.SP_ERR_INVALID_ARG
+    assert lib.sp_ring_attention_fwd(ctypes.byref(cfg), 0, 0.1, ok, ok, ok, ok, None,
+                                     None) == sp.SP_ERR_INVALID_ARG
+    bad = sp.make_cfg(384, 1, 128, 2, dtype="bf16")   # s / t = 192: not a 128-key tile
+    assert lib.sp_ring_attention_fwd_ws(ctypes.byref(bad), 1, 0.1, ok, ok, ok, ok, None, ok,
+                                        1 << 20, None) == sp.SP_ERR_UNSUPPORTED
+
+
 def test_fp32_residual_stream_needs_fp32_alignment(lib):
     """With res_f32 the residual-stream tensors are fp32: a pointer aligned
     for bf16 only is rejected before any launch, forward and backward."""
