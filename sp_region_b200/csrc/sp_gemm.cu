@@ -3,11 +3,13 @@
 // accumulation, with the SP region's bias, dropout and residual add in its
 // epilogue; the column-parallel linear whose all-gather is its A-operand
 // prologue; and ring attention over the context-parallel ranks.  Argument
-// validation, tensor maps and launch; the arithmetic is in sp_gemm.cuh and
-// sp_attn.cuh.
+// validation, tensor maps and launch; the arithmetic is in sp_gemm2.cuh (CTA
+// pairs), sp_gemm.cuh (one CTA, narrow outputs) and sp_attn.cuh.
 #include <cuda.h>
 #include <math.h>
 #include <string.h>
+
+#include <atomic>
 
 #include "sp_attn.cuh"
 #include "sp_gemm.cuh"
@@ -136,14 +138,16 @@ int launch_gemm2(GemmArgs a, const GemmMaps& maps, const DevInfo& dev, cudaStrea
     cfg.attrs = attr;
     cfg.numAttrs = 1;   // the occupancy query takes the cluster shape alone
     cfg.gridDim = dim3((unsigned)(dev.sms & ~1));
-    static int pairs_cache[64][2];
-    int pairs = dev.id >= 0 && dev.id < 64 ? pairs_cache[dev.id][EPI] : 0;
+    // clusters resident at once, per device and kernel (host threads may
+    // race to fill an entry; they store the same value)
+    static std::atomic<int> pairs_cache[64][2];
+    int pairs = dev.id >= 0 && dev.id < 64 ? pairs_cache[dev.id][EPI].load() : 0;
     if (pairs <= 0) {
         if (cudaOccupancyMaxActiveClusters(&pairs, kern, &cfg) != cudaSuccess || pairs <= 0) {
             cudaGetLastError();
             return SP_ERR_UNSUPPORTED;
         }
-        if (dev.id >= 0 && dev.id < 64) pairs_cache[dev.id][EPI] = pairs;
+        if (dev.id >= 0 && dev.id < 64) pairs_cache[dev.id][EPI].store(pairs);
     }
     const long long tiles = ((a.M + 2 * kGemmBM - 1) / (2 * kGemmBM)) *
                             (long long)((a.N + kGemm2BN - 1) / kGemm2BN);
