@@ -187,6 +187,38 @@ def test_ring_attention_validation(lib):
                                         1 << 20, None) == sp.SP_ERR_UNSUPPORTED
 
 
+def test_linears_validation(lib):
+    """The tensor-core linears reject missing or misaligned operands, an inner
+    dimension the ranks cannot split, shapes no kernel takes, and a missing
+    dropout mask, before any device query."""
+    import sp_region_b200 as sp
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.sp_rowpar_linear_rs_fwd.argtypes = [vp, i64, vp, vp, vp, vp, vp, vp, vp]
+    lib.sp_ag_colpar_linear_fwd.argtypes = [vp, i64, vp, vp, vp, vp]
+    ok, odd = vp(0x1000), vp(0x1008)
+    cfg = sp.make_cfg(256, 1, 256, 4, dtype="bf16", p_drop=0.1)
+    row = lambda f, x, w, res, rout, mask: lib.sp_rowpar_linear_rs_fwd(
+        ctypes.byref(cfg), f, x, w, None, res, rout, mask, None)
+    assert row(512, None, ok, ok, ok, ok) == sp.SP_ERR_INVALID_ARG    # no x
+    assert row(510, ok, ok, ok, ok, ok) == sp.SP_ERR_INVALID_ARG      # f % t != 0
+    assert row(516, ok, ok, ok, ok, ok) == sp.SP_ERR_UNSUPPORTED      # f % 8 != 0
+    assert row(512, ok, ok, ok, ok, None) == sp.SP_ERR_INVALID_ARG    # p > 0, no mask
+    assert row(512, odd, ok, ok, ok, ok) == sp.SP_ERR_INVALID_ARG     # misaligned x
+    f32 = sp.make_cfg(256, 1, 256, 4, dtype="f32")
+    assert lib.sp_rowpar_linear_rs_fwd(ctypes.byref(f32), 512, ok, ok, None, ok, ok, None,
+                                       None) == sp.SP_ERR_UNSUPPORTED  # bf16 only
+    cfg_c = sp.make_cfg(256, 1, 256, 4, dtype="bf16")
+    shards = (vp * 4)(*([0x1000] * 4))
+    col = lambda f_out, sh, w, out: lib.sp_ag_colpar_linear_fwd(
+        ctypes.byref(cfg_c), f_out, sh, w, out, None)
+    assert col(512, None, ok, ok) == sp.SP_ERR_INVALID_ARG           # no shards
+    assert col(0, shards, ok, ok) == sp.SP_ERR_INVALID_ARG           # no output features
+    assert col(516, shards, ok, ok) == sp.SP_ERR_UNSUPPORTED         # f_out % 8 != 0
+    ragged = sp.make_cfg(384, 1, 256, 4, dtype="bf16")               # 96 rows a shard
+    assert lib.sp_ag_colpar_linear_fwd(ctypes.byref(ragged), 512, shards, ok, ok,
+                                       None) == sp.SP_ERR_UNSUPPORTED
+
+
 def test_fp32_residual_stream_needs_fp32_alignment(lib):
     """With res_f32 the residual-stream tensors are fp32: a pointer aligned
     for bf16 only is rejected before any launch, forward and backward."""
